@@ -1,0 +1,246 @@
+/*
+ * pagedkv.h -- C ABI of the paged FP8-KV decode library for NVIDIA B200
+ * (sm_100a).
+ *
+ * The calls follow the problem as the source pages state it: a pool of
+ * physical KV-cache pages; per request a page table (logical page ->
+ * physical page); per page a uint32 tag that changes whenever the page is
+ * reallocated; per request the tags it expects; and a check, run as a
+ * separate batched step before a supported decode op reads the cache, that
+ * aborts any request whose page table names a page whose tag no longer
+ * matches.  Pages cited below:
+ *   [T] "大模型推理优化：量化、压缩与安全验证" (Chinese translation of the
+ *       first-party post), sections "量化 KV cache" and "保护共享 KV cache";
+ *   [S] siami.tw editorial on Cloudflare's Kimi/GLM inference, sections
+ *       "KV 快取量化" (Table 1) and "共享 KV 快取的完整性檢查" (Table 3);
+ *   [R] remio.ai commentary "Cloudflare 小型模型服务降低内存占用，但安全性成为考验",
+ *       section "共享 KV 缓存安全性成为生产问题".
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Memory: every array argument is DEVICE memory owned by the caller.  The
+ *    library allocates nothing, frees nothing and keeps no per-call state;
+ *    its only state is a thread-local error string and a per-device cache of
+ *    launch limits.
+ *  - bf16 values are passed as their 16-bit patterns (uint16_t); FP8 values
+ *    are E4M3 codes (uint8_t): 1 sign bit, 4 exponent bits with bias 7,
+ *    3 mantissa bits, S.1111.111 = NaN, no infinities, largest value 448.
+ *  - KV pools are laid out [num_pages][num_kv_heads][page_size][head_dim],
+ *    so one (page, KV head) tile is contiguous.  K and V live in separate
+ *    pools of the same shape.
+ *  - page_table and expected_tags are [batch][max_pages] (row stride
+ *    max_pages); only the first ceil(seq_lens[b] / page_size) entries of a
+ *    row are ever read.
+ *  - seq_lens[b] counts the request's new token: the new token sits at
+ *    position seq_lens[b] - 1.
+ *  - abort is a [batch] uint8 mask (nonzero = aborted); it may be NULL
+ *    wherever it is an input, meaning "no request is aborted" (the
+ *    integrity check switched off; [T] "保护共享 KV cache": the default path
+ *    is a no-op tracker with no measurable cost).
+ *  - Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).
+ *    Every call only enqueues work: it returns before the GPU runs it, and
+ *    never synchronises.
+ *  - Launch chaining: every kernel is launched with programmatic dependent
+ *    launch, so it may be scheduled while the previous kernel on the stream
+ *    is still running.  Each kernel waits for that kernel to finish before it
+ *    touches memory that kernel may write, with one exception documented at
+ *    paged_decode_attn_fp8: before waiting, attention reads q, seq_lens and
+ *    page_table and prefetches K/V pages into L2 (nothing it reads before
+ *    the wait reaches its outputs).
+ *  - Errors: a status code is returned.  Invalid arguments are detected on
+ *    the host before anything is enqueued (PKV_ERR_INVALID_ARG,
+ *    PKV_ERR_WORKSPACE, PKV_ERR_UNSUPPORTED); a failed launch returns
+ *    PKV_ERR_CUDA.  pkv_last_error() describes the last non-OK status on the
+ *    calling thread.  Bad DEVICE data never traps a kernel: a page id outside
+ *    [0, num_pages) or a length outside [1, max_pages * page_size] makes the
+ *    request behave as aborted.
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PKV_API __attribute__((visibility("default")))
+#else
+#define PKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t pkv_status;
+#define PKV_OK 0
+#define PKV_ERR_INVALID_ARG 1   /* bad pointer, size, shape or alignment   */
+#define PKV_ERR_WORKSPACE 2     /* workspace missing or too small          */
+#define PKV_ERR_UNSUPPORTED 3   /* valid but not implemented (e.g. D=96)   */
+#define PKV_ERR_CUDA 4          /* a CUDA runtime call or launch failed     */
+
+#define PKV_KV_FP8 0
+#define PKV_KV_BF16 1
+
+/* Supported shapes: head_dim in {64, 128}; page_size in {16, 32, 64, 128};
+ * num_q_heads a multiple of num_kv_heads with a group of at most 16;
+ * num_pages * num_kv_heads * page_size < 2^31. */
+
+/*
+ * kv_tag_check -- batched page-tag integrity check.
+ * [T] "保护共享 KV cache"; [S] "共享 KV 快取的完整性檢查"; [R] "共享 KV 缓存安全性成为生产问题":
+ * each physical page has a tag that changes on reallocation; the server
+ * records each request's expected pages and tags; before a supported decode
+ * op reads the cache the mapping is checked, and a mismatching request is
+ * aborted instead of returning data from the wrong page.  The check is its
+ * own batched kernel, not fused into attention ([S] Table 3 discussion).
+ *
+ * For each request b:
+ *   abort_out[b] = 1 if seq_lens[b] is outside [1, max_pages * page_size], or
+ *   if some entry j < ceil(seq_lens[b] / page_size) has page_table[b][j]
+ *   outside [0, num_pages) or page_tags[page_table[b][j]] !=
+ *   expected_tags[b][j]; otherwise 0.  Every abort_out[b] is written.
+ *   Entries past the used ones are never read.
+ * page_tags [num_pages] uint32; page_table [batch][max_pages] int32;
+ * expected_tags [batch][max_pages] uint32; seq_lens [batch] int32;
+ * abort_out [batch] uint8 (written); num_aborted: NULL or one int32 that
+ * receives the number of aborted requests (it is zeroed on the stream first).
+ */
+PKV_API pkv_status kv_tag_check(const uint32_t* page_tags, int32_t num_pages,
+                        const int32_t* page_table, const uint32_t* expected_tags,
+                        int32_t max_pages, const int32_t* seq_lens, int32_t batch,
+                        int32_t page_size, uint8_t* abort_out, int32_t* num_aborted,
+                        void* stream);
+
+/*
+ * kv_append_fp8 -- quantise each request's new K/V token to E4M3 and write
+ * it into its physical page.  [T] "量化 KV cache" / [S] "KV 快取量化": the KV
+ * cache is stored as FP8 e4m3, halving it against BF16.
+ *
+ * For request b with L = seq_lens[b] and pos = L - 1, every element x of
+ * k_new[b] (resp. v_new[b]) is written to
+ *   k_cache[page_table[b][pos / page_size]][h][pos % page_size][d]
+ * as the E4M3 code of y = x / k_scale, where y is the correctly rounded
+ * binary32 quotient and the code is y rounded to nearest, ties to even,
+ * with |y| > 448 (Inf included) saturated to +-448, NaN written as
+ * S.1111.111 keeping its sign, and signed zeros kept.
+ * Requests with abort[b] != 0 (abort may be NULL), a length outside
+ * [1, max_pages * page_size] or a page id outside [0, num_pages) are
+ * skipped.  k_new, v_new: [batch][num_kv_heads][head_dim] bf16, 16-byte
+ * aligned.  k_scale, v_scale: finite and > 0 (per-tensor scales).
+ */
+PKV_API pkv_status kv_append_fp8(const uint16_t* k_new, const uint16_t* v_new,
+                         const int32_t* page_table, int32_t max_pages,
+                         const int32_t* seq_lens, int32_t batch, int32_t num_kv_heads,
+                         int32_t head_dim, int32_t page_size, float k_scale, float v_scale,
+                         uint8_t* k_cache, uint8_t* v_cache, int32_t num_pages,
+                         const uint8_t* abort, void* stream);
+
+/*
+ * kv_append_bf16 -- the same write for a BF16 cache (the value is stored
+ * unchanged).  The BF16 cache is the comparison point of [S] Table 1.
+ */
+PKV_API pkv_status kv_append_bf16(const uint16_t* k_new, const uint16_t* v_new,
+                          const int32_t* page_table, int32_t max_pages,
+                          const int32_t* seq_lens, int32_t batch, int32_t num_kv_heads,
+                          int32_t head_dim, int32_t page_size,
+                          uint16_t* k_cache, uint16_t* v_cache, int32_t num_pages,
+                          const uint8_t* abort, void* stream);
+
+/*
+ * kv_requant_pages_fp8 -- BF16 -> FP8 page handoff.  [S] "KV 快取量化" and
+ * [T] "量化 KV cache": the prefill pool keeps a BF16 cache while the decode
+ * pool stores FP8.  Page src_pages[i] of the BF16 pool is re-quantised into
+ * page dst_pages[i] of the FP8 pool, element by element with exactly the
+ * rounding of kv_append_fp8.  Pairs naming an id outside their pool are
+ * skipped.  src_pool [src_num_pages][Hkv][P][D] bf16; dst_pool
+ * [dst_num_pages][Hkv][P][D] uint8; src_pages, dst_pages [num_pairs] int32.
+ * Call once for K (with k_scale) and once for V (with v_scale).
+ */
+PKV_API pkv_status kv_requant_pages_fp8(const uint16_t* src_pool, int32_t src_num_pages,
+                                const int32_t* src_pages, uint8_t* dst_pool,
+                                int32_t dst_num_pages, const int32_t* dst_pages,
+                                int32_t num_pairs, int32_t num_kv_heads, int32_t page_size,
+                                int32_t head_dim, float scale, void* stream);
+
+/*
+ * paged_decode_attn_workspace_size -- bytes of device workspace the
+ * attention calls need for these sizes.  kv_dtype is PKV_KV_FP8 or
+ * PKV_KV_BF16; num_ctas is the split-K grid size passed to the attention
+ * call (0 = the default, one full wave of resident CTAs on the current
+ * device).  Returns 0 on invalid arguments (see pkv_last_error).  The
+ * workspace holds a status word, the per-request chunk offsets and the
+ * split-K partial results; its first 4 bytes are a status word that the
+ * kernels set nonzero only if an internal bounded wait expires (never
+ * expected); the caller may read it after the stream has finished.
+ */
+PKV_API size_t paged_decode_attn_workspace_size(int32_t kv_dtype, int32_t batch, int32_t num_q_heads,
+                                        int32_t num_kv_heads, int32_t head_dim,
+                                        int32_t num_ctas);
+
+/*
+ * paged_decode_attn_fp8 -- decode attention of one new query token per
+ * request over a paged FP8 E4M3 cache, converting on every read ([T]
+ * "量化 KV cache": the FP8 attention kernel converts values as it reads
+ * them; [S] "KV 快取量化", Table 1).
+ *
+ * For every request b not aborted and every query head h (KV head
+ * h / (num_q_heads / num_kv_heads)):
+ *   s_t = sm_scale * sum_d q[b][h][d] * (decode(K_t[d]) * k_scale), t < L
+ *   lse[b][h] = ln sum_t exp(s_t)        (natural log, scaled scores)
+ *   out[b][h] = bf16( sum_t exp(s_t - lse[b][h]) * decode(V_t) * v_scale )
+ * where token t of request b lives in page page_table[b][t / page_size],
+ * slot t % page_size.  Aborted requests (abort[b] != 0), requests whose
+ * length is outside [1, max_pages * page_size] and requests whose used
+ * page-table entries name a page outside [0, num_pages) get out = 0 and
+ * lse = -inf; the cache pages of an aborted request are never read into
+ * the computation.
+ *
+ * q [batch][num_q_heads][head_dim] bf16 (16-byte aligned); caches as above
+ * (16-byte aligned); out [batch][num_q_heads][head_dim] bf16; lse
+ * [batch][num_q_heads] fp32.  workspace: device memory of at least
+ * paged_decode_attn_workspace_size(PKV_KV_FP8, ...) bytes, 256-byte
+ * aligned, not shared with a concurrently running attention call; its
+ * contents need no initialisation.  num_ctas: split-K grid size (0 =
+ * default); any value >= 1 gives the same result up to rounding.
+ *
+ * Work split: the (request, KV head, 64-token chunk) units are divided
+ * evenly over the CTAs of one persistent wave; a request split over several
+ * CTAs is combined by a log-sum-exp merge kernel.  Before its grid
+ * dependency wait the kernel reads q, seq_lens and page_table and prefetches
+ * its first K/V tiles into L2; everything else (abort, the cache contents)
+ * is read after the preceding kernel on the stream has finished.
+ */
+PKV_API pkv_status paged_decode_attn_fp8(const uint16_t* q, const uint8_t* k_cache,
+                                 const uint8_t* v_cache, float k_scale, float v_scale,
+                                 const int32_t* page_table, int32_t max_pages,
+                                 const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
+                                 int32_t num_kv_heads, int32_t head_dim, int32_t page_size,
+                                 int32_t num_pages, float sm_scale, const uint8_t* abort,
+                                 uint16_t* out, float* lse, void* workspace,
+                                 size_t workspace_bytes, int32_t num_ctas, void* stream);
+
+/*
+ * paged_decode_attn_bf16 -- the same attention over a BF16 cache (no
+ * scales), the comparison kernel of [S] Table 1.  Workspace from
+ * paged_decode_attn_workspace_size(PKV_KV_BF16, ...).
+ */
+PKV_API pkv_status paged_decode_attn_bf16(const uint16_t* q, const uint16_t* k_cache,
+                                  const uint16_t* v_cache, const int32_t* page_table,
+                                  int32_t max_pages, const int32_t* seq_lens, int32_t batch,
+                                  int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                  int32_t page_size, int32_t num_pages, float sm_scale,
+                                  const uint8_t* abort, uint16_t* out, float* lse,
+                                  void* workspace, size_t workspace_bytes, int32_t num_ctas,
+                                  void* stream);
+
+/* Message describing the last non-OK status returned on this thread. */
+PKV_API const char* pkv_last_error(void);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+PKV_API int32_t pkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H */

@@ -1,0 +1,399 @@
+// api.cu -- the extern "C" entry points declared in include/pagedkv.h:
+// host-side argument validation, TMA descriptor encoding, workspace layout
+// and kernel launches.  No call allocates, frees or synchronises.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "internal.h"
+#include "pagedkv.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+pkv_status fail(pkv_status code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+pkv_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(PKV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+bool supported_head_dim(int32_t d) { return d == 64 || d == 128; }
+bool supported_page_size(int32_t p) { return p == 16 || p == 32 || p == 64 || p == 128; }
+
+// ---------------------------------------------------------------------------
+// per-device launch limits (SM count, resident attention CTAs per SM)
+// ---------------------------------------------------------------------------
+constexpr int kMaxDevices = 64;
+struct DeviceInfo {
+    bool ready = false;
+    int sms = 0;
+    int occupancy[2][2][2] = {};   // [fp8][d128][gp16]
+};
+std::mutex g_dev_mutex;
+DeviceInfo g_dev[kMaxDevices];
+
+pkv_status device_info(const DeviceInfo** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(PKV_ERR_UNSUPPORTED, "device index %d", dev);
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    DeviceInfo& info = g_dev[dev];
+    if (!info.ready) {
+        e = cudaDeviceGetAttribute(&info.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+        for (int f = 0; f < 2; ++f)
+            for (int d = 0; d < 2; ++d)
+                for (int gp = 0; gp < 2; ++gp) {
+                    const bool fp8 = f == 1;
+                    const int hd = d ? 128 : 64, gpad = gp ? 16 : 8;
+                    e = pkv::attn_set_smem_attr(fp8, hd, gpad);
+                    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+                    int blocks = 0;
+                    e = pkv::attn_occupancy(fp8, hd, gpad, &blocks);
+                    if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
+                    info.occupancy[f][d][gp] = blocks < 1 ? 1 : blocks;
+                }
+        info.ready = true;
+    }
+    *out = &info;
+    return PKV_OK;
+}
+
+int group_pad_of(int group) { return group <= 8 ? 8 : 16; }
+
+pkv_status default_ctas(bool fp8, int head_dim, int group, int* ctas) {
+    const DeviceInfo* info = nullptr;
+    pkv_status st = device_info(&info);
+    if (st != PKV_OK) return st;
+    *ctas = info->sms * info->occupancy[fp8 ? 1 : 0][head_dim == 128][group > 8];
+    return PKV_OK;
+}
+
+// ---------------------------------------------------------------------------
+// TMA descriptors for the K / V pools viewed as 2-D [rows][head_dim]
+// ---------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+pkv_status get_encoder(EncodeTiledFn* fn) {
+    static std::once_flag once;
+    static EncodeTiledFn cached = nullptr;
+    static cudaError_t err = cudaSuccess;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+        if (err == cudaSuccess && q == cudaDriverEntryPointSuccess)
+            cached = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    if (cached == nullptr)
+        return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorString(err));
+    *fn = cached;
+    return PKV_OK;
+}
+
+pkv_status encode_pool_map(CUtensorMap* map, const void* pool, bool fp8, int head_dim,
+                           int64_t rows, int box_rows) {
+    EncodeTiledFn encode = nullptr;
+    pkv_status st = get_encoder(&encode);
+    if (st != PKV_OK) return st;
+    const int esize = fp8 ? 1 : 2;
+    const int box_inner = fp8 ? head_dim : 64;  // elements; 64 or 128 bytes
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(head_dim) * esize};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapSwizzle sw =
+        (box_inner * esize == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    CUresult r = encode(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                        2, const_cast<void*>(pool), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return PKV_OK;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+pkv_status check_common_kv(int32_t batch, int32_t num_kv_heads, int32_t head_dim,
+                           int32_t page_size, int32_t num_pages, int32_t max_pages) {
+    if (batch < 0) return fail(PKV_ERR_INVALID_ARG, "batch must be >= 0 (got %d)", batch);
+    if (num_kv_heads < 1) return fail(PKV_ERR_INVALID_ARG, "num_kv_heads must be >= 1");
+    if (!supported_head_dim(head_dim))
+        return fail(PKV_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", head_dim);
+    if (!supported_page_size(page_size))
+        return fail(PKV_ERR_UNSUPPORTED, "page_size %d not supported (16, 32, 64, 128)", page_size);
+    if (num_pages < 1) return fail(PKV_ERR_INVALID_ARG, "num_pages must be >= 1");
+    if (max_pages < 1) return fail(PKV_ERR_INVALID_ARG, "max_pages must be >= 1");
+    const int64_t rows = static_cast<int64_t>(num_pages) * num_kv_heads * page_size;
+    if (rows >= (int64_t(1) << 31))
+        return fail(PKV_ERR_UNSUPPORTED, "num_pages * num_kv_heads * page_size must be < 2^31");
+    return PKV_OK;
+}
+
+pkv_status attn_impl(bool fp8, const uint16_t* q, const void* k_cache, const void* v_cache,
+                     float k_scale, float v_scale, const int32_t* page_table, int32_t max_pages,
+                     const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
+                     int32_t num_kv_heads, int32_t head_dim, int32_t page_size, int32_t num_pages,
+                     float sm_scale, const uint8_t* abort, uint16_t* out, float* lse,
+                     void* workspace, size_t workspace_bytes, int32_t num_ctas, void* stream) {
+    pkv_status st = check_common_kv(batch, num_kv_heads, head_dim, page_size, num_pages, max_pages);
+    if (st != PKV_OK) return st;
+    if (num_q_heads < 1 || num_q_heads % num_kv_heads != 0)
+        return fail(PKV_ERR_INVALID_ARG, "num_q_heads (%d) must be a positive multiple of "
+                    "num_kv_heads (%d)", num_q_heads, num_kv_heads);
+    const int group = num_q_heads / num_kv_heads;
+    if (group > 16) return fail(PKV_ERR_UNSUPPORTED, "GQA group %d > 16 not supported", group);
+    if (!(std::isfinite(sm_scale)))
+        return fail(PKV_ERR_INVALID_ARG, "sm_scale must be finite");
+    if (fp8 && (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) ||
+                !std::isfinite(v_scale)))
+        return fail(PKV_ERR_INVALID_ARG, "k_scale and v_scale must be finite and > 0");
+    if (num_ctas < 0) return fail(PKV_ERR_INVALID_ARG, "num_ctas must be >= 0");
+    if (batch == 0) return PKV_OK;
+    if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !out || !lse)
+        return fail(PKV_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 4) ||
+        !aligned(lse, 4) || !aligned(page_table, 4) || !aligned(seq_lens, 4))
+        return fail(PKV_ERR_INVALID_ARG, "misaligned pointer (q and caches need 16 bytes)");
+    if (!workspace || !aligned(workspace, 256))
+        return fail(PKV_ERR_WORKSPACE, "workspace must be non-null and 256-byte aligned");
+
+    int grid = num_ctas;
+    if (grid == 0) {
+        st = default_ctas(fp8, head_dim, group, &grid);
+        if (st != PKV_OK) return st;
+    } else {
+        const DeviceInfo* info = nullptr;
+        st = device_info(&info);  // sets the shared-memory attribute
+        if (st != PKV_OK) return st;
+    }
+    const pkv::WorkspaceLayout wl =
+        pkv::workspace_layout(batch, group, num_kv_heads, head_dim, grid);
+    if (workspace_bytes < wl.total)
+        return fail(PKV_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes,
+                    wl.total);
+
+    const int box_rows = page_size < pkv::kChunkTokens ? page_size : pkv::kChunkTokens;
+    const int64_t rows = static_cast<int64_t>(num_pages) * num_kv_heads * page_size;
+    CUtensorMap tk, tv;
+    st = encode_pool_map(&tk, k_cache, fp8, head_dim, rows, box_rows);
+    if (st != PKV_OK) return st;
+    st = encode_pool_map(&tv, v_cache, fp8, head_dim, rows, box_rows);
+    if (st != PKV_OK) return st;
+
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    pkv::AttnArgs a{};
+    a.q = q;
+    a.page_table = page_table;
+    a.seq_lens = seq_lens;
+    a.abort = abort;
+    a.out = out;
+    a.lse = lse;
+    a.ws_status = reinterpret_cast<uint32_t*>(ws);
+    a.ws_prefix = reinterpret_cast<int32_t*>(ws + wl.prefix_off);
+    a.ws_ml = reinterpret_cast<float*>(ws + wl.ml_off);
+    a.ws_o = reinterpret_cast<float*>(ws + wl.o_off);
+    a.batch = batch;
+    a.max_pages = max_pages;
+    a.num_q_heads = num_q_heads;
+    a.num_kv_heads = num_kv_heads;
+    a.group = group;
+    a.page_size = page_size;
+    a.num_pages = num_pages;
+    a.num_ctas = grid;
+    a.box_rows = box_rows;
+    a.qk_scale = sm_scale * (fp8 ? k_scale : 1.f) * 1.4426950408889634f;
+    a.v_scale = fp8 ? v_scale : 1.f;
+
+    cudaError_t e = pkv::launch_attn_partial(fp8, head_dim, group_pad_of(group), grid,
+                                             as_stream(stream), tk, tv, a);
+    if (e != cudaSuccess) return cuda_fail(e, "attention partial launch");
+    e = pkv::launch_attn_merge(head_dim, as_stream(stream), a);
+    if (e != cudaSuccess) return cuda_fail(e, "attention merge launch");
+    return PKV_OK;
+}
+
+}  // namespace
+
+namespace pkv {
+WorkspaceLayout workspace_layout(int32_t batch, int32_t group, int32_t num_kv_heads,
+                                 int32_t head_dim, int32_t num_ctas) {
+    WorkspaceLayout l{};
+    l.prefix_off = 256;
+    const size_t slots = static_cast<size_t>(num_ctas) + static_cast<size_t>(batch) * num_kv_heads;
+    l.ml_off = round_up(l.prefix_off + (static_cast<size_t>(batch) + 1) * 4, 256);
+    l.o_off = round_up(l.ml_off + slots * group * 2 * 4, 256);
+    l.total = round_up(l.o_off + slots * group * head_dim * 4, 256);
+    return l;
+}
+}  // namespace pkv
+
+extern "C" {
+
+const char* pkv_last_error(void) { return g_last_error.c_str(); }
+
+int32_t pkv_version(void) { return 100; }
+
+pkv_status kv_tag_check(const uint32_t* page_tags, int32_t num_pages, const int32_t* page_table,
+                        const uint32_t* expected_tags, int32_t max_pages, const int32_t* seq_lens,
+                        int32_t batch, int32_t page_size, uint8_t* abort_out,
+                        int32_t* num_aborted, void* stream) {
+    if (batch < 0) return fail(PKV_ERR_INVALID_ARG, "batch must be >= 0");
+    if (num_pages < 1 || max_pages < 1 || page_size < 1)
+        return fail(PKV_ERR_INVALID_ARG, "num_pages, max_pages and page_size must be >= 1");
+    if (batch > 0 && (!page_tags || !page_table || !expected_tags || !seq_lens || !abort_out))
+        return fail(PKV_ERR_INVALID_ARG, "null pointer argument");
+    if (num_aborted) {
+        cudaError_t e = cudaMemsetAsync(num_aborted, 0, sizeof(int32_t), as_stream(stream));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(num_aborted)");
+    }
+    if (batch == 0) return PKV_OK;
+    cudaError_t e = pkv::launch_tag_check(page_tags, num_pages, page_table, expected_tags,
+                                          max_pages, seq_lens, batch, page_size, abort_out,
+                                          num_aborted, as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "tag check launch");
+    return PKV_OK;
+}
+
+static pkv_status append_impl(bool fp8, const uint16_t* k_new, const uint16_t* v_new,
+                              const int32_t* page_table, int32_t max_pages,
+                              const int32_t* seq_lens, int32_t batch, int32_t num_kv_heads,
+                              int32_t head_dim, int32_t page_size, float k_scale, float v_scale,
+                              void* k_cache, void* v_cache, int32_t num_pages,
+                              const uint8_t* abort, void* stream) {
+    pkv_status st = check_common_kv(batch, num_kv_heads, head_dim, page_size, num_pages, max_pages);
+    if (st != PKV_OK) return st;
+    if (fp8 && (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) ||
+                !std::isfinite(v_scale)))
+        return fail(PKV_ERR_INVALID_ARG, "k_scale and v_scale must be finite and > 0");
+    if (batch == 0) return PKV_OK;
+    if (!k_new || !v_new || !page_table || !seq_lens || !k_cache || !v_cache)
+        return fail(PKV_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) ||
+        !aligned(v_cache, 16))
+        return fail(PKV_ERR_INVALID_ARG, "k_new, v_new and the caches must be 16-byte aligned");
+    cudaError_t e = pkv::launch_append(fp8, k_new, v_new, page_table, max_pages, seq_lens, batch,
+                                       num_kv_heads, head_dim, page_size, k_scale, v_scale,
+                                       k_cache, v_cache, num_pages, abort, as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "append launch");
+    return PKV_OK;
+}
+
+pkv_status kv_append_fp8(const uint16_t* k_new, const uint16_t* v_new, const int32_t* page_table,
+                         int32_t max_pages, const int32_t* seq_lens, int32_t batch,
+                         int32_t num_kv_heads, int32_t head_dim, int32_t page_size, float k_scale,
+                         float v_scale, uint8_t* k_cache, uint8_t* v_cache, int32_t num_pages,
+                         const uint8_t* abort, void* stream) {
+    return append_impl(true, k_new, v_new, page_table, max_pages, seq_lens, batch, num_kv_heads,
+                       head_dim, page_size, k_scale, v_scale, k_cache, v_cache, num_pages, abort,
+                       stream);
+}
+
+pkv_status kv_append_bf16(const uint16_t* k_new, const uint16_t* v_new,
+                          const int32_t* page_table, int32_t max_pages, const int32_t* seq_lens,
+                          int32_t batch, int32_t num_kv_heads, int32_t head_dim,
+                          int32_t page_size, uint16_t* k_cache, uint16_t* v_cache,
+                          int32_t num_pages, const uint8_t* abort, void* stream) {
+    return append_impl(false, k_new, v_new, page_table, max_pages, seq_lens, batch, num_kv_heads,
+                       head_dim, page_size, 1.f, 1.f, k_cache, v_cache, num_pages, abort, stream);
+}
+
+pkv_status kv_requant_pages_fp8(const uint16_t* src_pool, int32_t src_num_pages,
+                                const int32_t* src_pages, uint8_t* dst_pool,
+                                int32_t dst_num_pages, const int32_t* dst_pages,
+                                int32_t num_pairs, int32_t num_kv_heads, int32_t page_size,
+                                int32_t head_dim, float scale, void* stream) {
+    if (num_pairs < 0) return fail(PKV_ERR_INVALID_ARG, "num_pairs must be >= 0");
+    if (src_num_pages < 1 || dst_num_pages < 1 || num_kv_heads < 1)
+        return fail(PKV_ERR_INVALID_ARG, "pool sizes and num_kv_heads must be >= 1");
+    if (!supported_head_dim(head_dim))
+        return fail(PKV_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", head_dim);
+    if (!supported_page_size(page_size))
+        return fail(PKV_ERR_UNSUPPORTED, "page_size %d not supported", page_size);
+    if (!(scale > 0.f) || !std::isfinite(scale))
+        return fail(PKV_ERR_INVALID_ARG, "scale must be finite and > 0");
+    if (num_pairs == 0) return PKV_OK;
+    if (!src_pool || !src_pages || !dst_pool || !dst_pages)
+        return fail(PKV_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned(src_pool, 16) || !aligned(dst_pool, 16))
+        return fail(PKV_ERR_INVALID_ARG, "pools must be 16-byte aligned");
+    const int64_t page_elems = static_cast<int64_t>(num_kv_heads) * page_size * head_dim;
+    cudaError_t e = pkv::launch_requant(src_pool, src_num_pages, src_pages, dst_pool,
+                                        dst_num_pages, dst_pages, num_pairs, page_elems, scale,
+                                        as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "requant launch");
+    return PKV_OK;
+}
+
+size_t paged_decode_attn_workspace_size(int32_t kv_dtype, int32_t batch, int32_t num_q_heads,
+                                        int32_t num_kv_heads, int32_t head_dim,
+                                        int32_t num_ctas) {
+    if (kv_dtype != PKV_KV_FP8 && kv_dtype != PKV_KV_BF16) {
+        fail(PKV_ERR_INVALID_ARG, "kv_dtype must be PKV_KV_FP8 or PKV_KV_BF16");
+        return 0;
+    }
+    if (batch < 0 || num_kv_heads < 1 || num_q_heads < 1 || num_q_heads % num_kv_heads != 0 ||
+        !supported_head_dim(head_dim) || num_ctas < 0) {
+        fail(PKV_ERR_INVALID_ARG, "invalid sizes for the workspace query");
+        return 0;
+    }
+    const int group = num_q_heads / num_kv_heads;
+    if (group > 16) {
+        fail(PKV_ERR_UNSUPPORTED, "GQA group %d > 16 not supported", group);
+        return 0;
+    }
+    int grid = num_ctas;
+    if (grid == 0 && default_ctas(kv_dtype == PKV_KV_FP8, head_dim, group, &grid) != PKV_OK)
+        return 0;
+    return pkv::workspace_layout(batch, group, num_kv_heads, head_dim, grid).total;
+}
+
+pkv_status paged_decode_attn_fp8(const uint16_t* q, const uint8_t* k_cache,
+                                 const uint8_t* v_cache, float k_scale, float v_scale,
+                                 const int32_t* page_table, int32_t max_pages,
+                                 const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
+                                 int32_t num_kv_heads, int32_t head_dim, int32_t page_size,
+                                 int32_t num_pages, float sm_scale, const uint8_t* abort,
+                                 uint16_t* out, float* lse, void* workspace,
+                                 size_t workspace_bytes, int32_t num_ctas, void* stream) {
+    return attn_impl(true, q, k_cache, v_cache, k_scale, v_scale, page_table, max_pages, seq_lens,
+                     batch, num_q_heads, num_kv_heads, head_dim, page_size, num_pages, sm_scale,
+                     abort, out, lse, workspace, workspace_bytes, num_ctas, stream);
+}
+
+pkv_status paged_decode_attn_bf16(const uint16_t* q, const uint16_t* k_cache,
+                                  const uint16_t* v_cache, const int32_t* page_table,
+                                  int32_t max_pages, const int32_t* seq_lens, int32_t batch,
+                                  int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                  int32_t page_size, int32_t num_pages, float sm_scale,
+                                  const uint8_t* abort, uint16_t* out, float* lse,
+                                  void* workspace, size_t workspace_bytes, int32_t num_ctas,
+                                  void* stream) {
+    return attn_impl(false, q, k_cache, v_cache, 1.f, 1.f, page_table, max_pages, seq_lens, batch,
+                     num_q_heads, num_kv_heads, head_dim, page_size, num_pages, sm_scale, abort,
+                     out, lse, workspace, workspace_bytes, num_ctas, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,811 @@
+// attention.cu -- paged decode attention over an FP8 E4M3 or BF16 KV cache
+// for sm_100a: split-K partial kernel plus log-sum-exp merge kernel.
+//
+// Source pages: "大模型推理优化：量化、压缩与安全验证", section "量化 KV cache"
+// (FP8 e4m3 cache; the FP8 attention kernel converts values on every read);
+// siami.tw editorial, section "KV 快取量化" (Table 1: FP8 vs BF16 KV decode
+// throughput); remio.ai commentary, section "小型缓存胜过单纯的速度" (decode
+// is memory-bound).  The pages give no kernel design; the one here is:
+//
+//  * Work: units are (request, KV head, 64-token chunk).  The units of the
+//    whole batch are cut into num_ctas equal contiguous ranges, one per CTA
+//    of a single persistent wave, so long and short requests balance.  A CTA
+//    walks its range as "segments" (maximal runs inside one (request, KV
+//    head) item).  A segment covering a whole item writes the final output;
+//    otherwise it writes an fp32 partial (m, l, O) to workspace slot
+//    cta + item (unique because the partition is monotone) and the merge
+//    kernel combines the partials of that item.
+//  * Pipeline: warp 4 is the producer.  Its lane 0 streams the K and V tiles
+//    of each chunk from the [page][kv_head][slot][dim] pools into a ring of
+//    shared-memory stages with 2-D TMA tensor loads (128-byte swizzle)
+//    completing on mbarriers; consumers release a stage through a second
+//    mbarrier.  Before its grid-dependency wait the producer prefetches its
+//    first stages into L2 so the preceding kernels (tag check, append)
+//    overlap with DRAM traffic.
+//  * Math: warps 0-3 each own a 16-token slice of every chunk and keep their
+//    own online-softmax state.  Scores S = Q K^T and the output O = P V run on
+//    tensor cores as m16n8k16 MMAs with the query heads of one KV head (the
+//    GQA group, padded to 8 or 16) as the M dimension.  FP8 codes are turned
+//    into f16 in registers with the hardware E4M3 conversion (exact); the
+//    per-tensor scales are folded into the score scale and into the output.
+//    For the FP8 path each query head is scaled by a power of two so that
+//    its largest |q| lies in [128, 256), which keeps the bf16 -> f16
+//    conversion exact; the power of two is undone in the score scale.
+//  * Layout tricks: the token order inside each 8-row group and the order of
+//    the head dimension inside the QK contraction are permuted (both are
+//    free: softmax and the contraction are invariant under them) so that
+//    each thread's shared-memory reads are 16-byte (K) or 4-byte (V) words
+//    that hit 32 distinct banks under the TMA swizzle.
+//  * Lazy rescaling: a warp rescales O only when a head's running maximum
+//    grows by more than 8 (log2 units); P is then at most 2^8, exact enough
+//    in f16 and far from overflow.
+#include "device.cuh"
+#include "internal.h"
+
+namespace pkv {
+
+constexpr int kConsumerWarps = 4;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;
+constexpr float kNegInf = -__builtin_huge_valf();
+
+template <bool kFp8, int kD, int kGP>
+struct AttnCfg {
+    static constexpr int kElem = kFp8 ? 1 : 2;
+    static constexpr int kRowBytes = kD * kElem;                 // 64, 128 or 256
+    static constexpr int kBoxBytes = kFp8 ? kRowBytes : 128;     // TMA box inner bytes
+    static constexpr int kSubTiles = kRowBytes / kBoxBytes;      // 2 for BF16 D=128
+    static constexpr int kSwizzle = kBoxBytes;                   // 128 or 64
+    static constexpr int kSubTileBytes = kChunkTokens * kBoxBytes;
+    static constexpr int kTileBytes = kChunkTokens * kRowBytes;  // one of K or V per stage
+    static constexpr int kStageBytes = 2 * kTileBytes;
+    static constexpr int kStages =
+        kFp8 ? (kD == 128 ? 5 : 8) : (kD == 128 ? (kGP == 8 ? 3 : 2) : 5);
+    static constexpr int kRedOff = kStages * kStageBytes;
+    static constexpr int kRedFloats = kConsumerWarps * kGP * (kD + 2);
+    static constexpr int kBarOff = kRedOff + kRedFloats * 4;
+    static constexpr int kFlagOff = kBarOff + 2 * kStages * 8;
+    static constexpr int kScratchOff = kFlagOff + kStages * 4;
+    static constexpr int kSmemBytes = kScratchOff + 16 * 4 + 1024;  // + alignment slack
+    static_assert(kD == 64 || kD == 128, "head_dim");
+    static_assert(kGP == 8 || kGP == 16, "group pad");
+};
+
+// Token permutation inside an 8-row group: row tau(n) feeds MMA column n.
+__device__ __forceinline__ int tau(int n) { return n ^ ((n & 1) << 2); }
+
+struct Segment {
+    int b, h, c0, c1, n, L;
+};
+
+// Walks a CTA's unit range [u, u_hi) segment by segment.  Every warp runs an
+// identical copy, so producer and consumers agree without communicating.
+struct Walker {
+    const int32_t* seq_lens;
+    int64_t max_tokens;
+    int num_kv_heads;
+    int batch;
+    int b, h, ch, n, L;
+    int64_t u, u_hi;
+
+    __device__ __forceinline__ int chunks_of(int32_t len) const {
+        return (len >= 1 && static_cast<int64_t>(len) <= max_tokens)
+                   ? (len + kChunkTokens - 1) / kChunkTokens
+                   : 0;
+    }
+    __device__ __forceinline__ void init(int b0, int pre0, int64_t ulo, int64_t uhi) {
+        u = ulo;
+        u_hi = uhi;
+        b = b0;
+        h = ch = n = L = 0;
+        if (u < u_hi) {
+            L = seq_lens[b];
+            n = chunks_of(L);
+            const int64_t off = ulo - static_cast<int64_t>(num_kv_heads) * pre0;
+            h = static_cast<int>(off / n);
+            ch = static_cast<int>(off % n);
+        }
+    }
+    __device__ __forceinline__ bool next(Segment& s) {
+        if (u >= u_hi || ch >= n) {   // ch >= n only if the batch changed under us
+            u = u_hi;
+            return false;
+        }
+        const int64_t left = u_hi - u;
+        const int take = static_cast<int>(left < (n - ch) ? left : (n - ch));
+        s.b = b;
+        s.h = h;
+        s.c0 = ch;
+        s.c1 = ch + take;
+        s.n = n;
+        s.L = L;
+        u += take;
+        ch += take;
+        if (u < u_hi && ch == n) {
+            ch = 0;
+            if (++h == num_kv_heads) {
+                h = 0;
+                do {
+                    ++b;
+                    L = seq_lens[b];
+                    n = chunks_of(L);
+                } while (n == 0 && b + 1 < batch);
+            }
+        }
+        return true;
+    }
+};
+
+__device__ __forceinline__ void record_timeout(const AttnArgs& a, volatile int* cta_failed) {
+    *cta_failed = 1;
+    atomicOr(a.ws_status, 1u);
+}
+// Bounded mbarrier wait.  After a timeout in this CTA every later wait
+// returns at once, so the kernel always runs to completion; the workspace
+// status word reports the failure.
+__device__ __forceinline__ void wait_or_give_up(uint64_t* bar, uint32_t parity, const AttnArgs& a,
+                                                volatile int* cta_failed) {
+    if (*cta_failed) return;
+    if (!mbar_wait(bar, parity)) record_timeout(a, cta_failed);
+}
+
+// Page id of entry j of a row, read through a 32-entry window held across
+// the producer warp's lanes (one coalesced load per 32 pages).
+struct PageWindow {
+    const int32_t* row;
+    int base;
+    int32_t mine;
+    __device__ __forceinline__ void reset(const int32_t* r) {
+        row = r;
+        base = -(1 << 30);
+    }
+    __device__ __forceinline__ int32_t get(int j, int limit, int lane) {
+        if (j < base || j >= base + 32) {
+            base = j;
+            mine = (j + lane < limit) ? row[j + lane] : -1;
+        }
+        return __shfl_sync(0xffffffffu, mine, j - base);
+    }
+};
+
+// ---------------------------------------------------------------------------
+// the split-K partial kernel
+// ---------------------------------------------------------------------------
+template <bool kFp8, int kD, int kGP>
+__global__ void __launch_bounds__(kAttnThreads, 2)
+attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                    const __grid_constant__ CUtensorMap tmap_v, const AttnArgs a) {
+    using C = AttnCfg<kFp8, kD, kGP>;
+    constexpr int S = C::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    float* red_o = reinterpret_cast<float*>(smem + C::kRedOff);
+    float* red_m = red_o + kConsumerWarps * kGP * kD;
+    float* red_l = red_m + kConsumerWarps * kGP;
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+    uint64_t* empty_bar = full_bar + S;
+    volatile int* stage_bad = reinterpret_cast<volatile int*>(smem + C::kFlagOff);
+    int* scratch = reinterpret_cast<int*>(smem + C::kScratchOff);
+    volatile int* cta_failed = scratch + 10;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int B = a.batch;
+    const int Hkv = a.num_kv_heads;
+    const int64_t max_tokens = static_cast<int64_t>(a.max_pages) * a.page_size;
+
+    launch_dependents();
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], kConsumerWarps);
+        }
+        *cta_failed = 0;
+        fence_barrier_init();
+    }
+
+    // ---- partition: exclusive scan of chunk counts over the batch --------
+    Walker walk;
+    walk.seq_lens = a.seq_lens;
+    walk.max_tokens = max_tokens;
+    walk.num_kv_heads = Hkv;
+    walk.batch = B;
+    const int per = (B + kAttnThreads - 1) / kAttnThreads;
+    const int b_lo = min(B, tid * per);
+    const int b_hi = min(B, b_lo + per);
+    int local = 0;
+    for (int b = b_lo; b < b_hi; ++b) local += walk.chunks_of(a.seq_lens[b]);
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+    }
+    if (lane == 31) scratch[warp] = incl;
+    __syncthreads();
+    int warp_base = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kAttnThreads / 32; ++w) {
+        const int t = scratch[w];
+        if (w < warp) warp_base += t;
+        total += t;
+    }
+    const int64_t U = static_cast<int64_t>(Hkv) * total;
+    const int64_t u_lo = static_cast<int64_t>(blockIdx.x) * U / a.num_ctas;
+    const int64_t u_hi = static_cast<int64_t>(blockIdx.x + 1) * U / a.num_ctas;
+    {
+        int run = warp_base + incl - local;
+        for (int b = b_lo; b < b_hi; ++b) {
+            const int n = walk.chunks_of(a.seq_lens[b]);
+            if (blockIdx.x == 0) a.ws_prefix[b] = run;
+            if (n > 0 && u_lo < u_hi && static_cast<int64_t>(Hkv) * run <= u_lo &&
+                u_lo < static_cast<int64_t>(Hkv) * (run + n)) {
+                scratch[8] = b;
+                scratch[9] = run;
+            }
+            run += n;
+        }
+        if (blockIdx.x == 0 && tid == 0) a.ws_prefix[B] = total;
+    }
+    __syncthreads();
+    if (u_lo >= u_hi) return;
+    walk.init(scratch[8], scratch[9], u_lo, u_hi);
+
+    const int P = a.page_size;
+    const int box_rows = a.box_rows;
+    const int boxes = kChunkTokens / box_rows;
+
+    if (warp == kConsumerWarps) {
+        // ================= producer warp =================
+        prefetch_tensormap(&tmap_k);
+        prefetch_tensormap(&tmap_v);
+        PageWindow win;
+        // L2 prefetch of the first S chunks, before the dependency wait.
+        {
+            Walker w2 = walk;
+            Segment s;
+            int count = 0;
+            while (count < S && w2.next(s)) {
+                win.reset(a.page_table + static_cast<int64_t>(s.b) * a.max_pages);
+                const int npages = (s.L + P - 1) / P;
+                for (int ch = s.c0; ch < s.c1 && count < S; ++ch, ++count) {
+                    for (int i = 0; i < boxes; ++i) {
+                        const int tok0 = ch * kChunkTokens + i * box_rows;
+                        const int j = tok0 / P;
+                        if (j >= npages) break;
+                        const int32_t pid = win.get(j, npages, lane);
+                        if (lane == 0 && pid >= 0 && pid < a.num_pages) {
+                            const int32_t y = (pid * Hkv + s.h) * P + (tok0 % P);
+                            for (int st = 0; st < C::kSubTiles; ++st) {
+                                tma_prefetch_l2_2d(&tmap_k, st * 64, y);
+                                tma_prefetch_l2_2d(&tmap_v, st * 64, y);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+        grid_dependency_wait();
+        uint32_t it = 0;
+        Segment s;
+        while (walk.next(s)) {
+            if (a.abort != nullptr && a.abort[s.b] != 0) continue;
+            win.reset(a.page_table + static_cast<int64_t>(s.b) * a.max_pages);
+            const int npages = (s.L + P - 1) / P;
+            for (int ch = s.c0; ch < s.c1; ++ch, ++it) {
+                const int stage = it % S;
+                if (it >= static_cast<uint32_t>(S)) {
+                    if (lane == 0) wait_or_give_up(&empty_bar[stage], ((it / S) + 1) & 1, a, cta_failed);
+                    __syncwarp();
+                }
+                const uint32_t kdst = smem_addr(smem + stage * C::kStageBytes);
+                const uint32_t vdst = kdst + C::kTileBytes;
+                uint32_t bytes = 0;
+                int bad = 0;
+                int32_t pids[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    pids[i] = -1;
+                    if (i < boxes) {
+                        const int tok0 = ch * kChunkTokens + i * box_rows;
+                        const int j = tok0 / P;
+                        if (j < npages) {
+                            pids[i] = win.get(j, npages, lane);
+                            if (pids[i] < 0 || pids[i] >= a.num_pages) {
+                                bad = 1;
+                                pids[i] = -1;
+                            } else {
+                                bytes += 2u * C::kSubTiles * box_rows * C::kBoxBytes;
+                            }
+                        }
+                    }
+                }
+                if (lane == 0) {
+                    stage_bad[stage] = bad;
+                    mbar_arrive_expect_tx(&full_bar[stage], bytes);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        if (pids[i] < 0) continue;
+                        const int tok0 = ch * kChunkTokens + i * box_rows;
+                        const int32_t y = (pids[i] * Hkv + s.h) * P + (tok0 % P);
+                        for (int st = 0; st < C::kSubTiles; ++st) {
+                            const uint32_t off = st * C::kSubTileBytes + i * box_rows * C::kBoxBytes;
+                            tma_load_2d(kdst + off, &tmap_k, st * 64, y, &full_bar[stage]);
+                            tma_load_2d(vdst + off, &tmap_v, st * 64, y, &full_bar[stage]);
+                        }
+                    }
+                }
+                __syncwarp();
+            }
+        }
+        return;
+    }
+
+    // ================= consumer warps =================
+    grid_dependency_wait();
+    const int g = lane >> 2;   // MMA group id: head row g (and g + 8)
+    const int c = lane & 3;    // thread in group
+    const int G = a.group;
+    const int rb = warp * 16;  // this warp's rows of each chunk
+    constexpr int kNB = kD / 8;       // n-blocks of the output
+    constexpr int kKS = kD / 16;      // k-steps of the QK contraction
+
+    uint32_t it = 0;
+    Segment s;
+    while (walk.next(s)) {
+        const int item = s.b * Hkv + s.h;
+        const bool whole = (s.c0 == 0 && s.c1 == s.n);
+        const int64_t slot = static_cast<int64_t>(blockIdx.x) + item;
+        const int64_t head0 = static_cast<int64_t>(s.b) * a.num_q_heads + s.h * G;
+
+        if (a.abort != nullptr && a.abort[s.b] != 0) {
+            for (int e = tid; e < G * kD; e += kConsumerThreads) {
+                const int hq = e / kD, d = e % kD;
+                if (whole) {
+                    a.out[(head0 + hq) * kD + d] = 0;
+                    if (d == 0) a.lse[head0 + hq] = kNegInf;
+                } else {
+                    a.ws_o[(slot * G + hq) * kD + d] = 0.f;
+                    if (d == 0) {
+                        a.ws_ml[(slot * G + hq) * 2 + 0] = kNegInf;
+                        a.ws_ml[(slot * G + hq) * 2 + 1] = -1.f;
+                    }
+                }
+            }
+            continue;
+        }
+
+        // ---- query fragments (A operand, rows = heads g and g + 8) -------
+        uint32_t qa[kKS][4];
+        float qk0 = 0.f, qk1 = 0.f;
+#pragma unroll
+        for (int half = 0; half < (kGP == 16 ? 2 : 1); ++half) {
+            const int hh = g + 8 * half;
+            const bool valid = hh < G;
+            const uint16_t* qrow = a.q + (head0 + (valid ? hh : 0)) * kD;
+            if constexpr (kFp8) {
+                // this thread's dims: [16c, 16c+16) and, for D=128, [64+16c, 64+16c+16)
+                float v[kD / 4];
+#pragma unroll
+                for (int part = 0; part < kD / 64; ++part) {
+                    const uint4* src = reinterpret_cast<const uint4*>(qrow + part * 64 + 16 * c);
+                    const uint4 w0 = src[0], w1 = src[1];
+                    const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        v[part * 16 + 2 * k] = valid ? bf16_bits_to_f32(ws[k] & 0xFFFFu) : 0.f;
+                        v[part * 16 + 2 * k + 1] = valid ? bf16_bits_to_f32(ws[k] >> 16) : 0.f;
+                    }
+                }
+                float amax = 0.f;
+#pragma unroll
+                for (int k = 0; k < kD / 4; ++k) amax = fmaxf(amax, fabsf(v[k]));
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+                int e = 0;
+                int shift = 0;
+                if (amax > 0.f && isfinite(amax)) {
+                    frexpf(amax, &e);
+                    shift = min(60, max(-126, 8 - e));
+                }
+#pragma unroll
+                for (int j = 0; j < kKS; ++j) {
+                    qa[j][half] = pack_f16x2(ldexpf(v[4 * j], shift), ldexpf(v[4 * j + 1], shift));
+                    qa[j][2 + half] =
+                        pack_f16x2(ldexpf(v[4 * j + 2], shift), ldexpf(v[4 * j + 3], shift));
+                }
+                const float qs = a.qk_scale * ldexpf(1.f, -shift);
+                if (half == 0) qk0 = qs; else qk1 = qs;
+            } else {
+#pragma unroll
+                for (int j = 0; j < kKS; ++j) {
+                    const uint32_t* src = reinterpret_cast<const uint32_t*>(qrow + 16 * j + 2 * c);
+                    qa[j][half] = valid ? src[0] : 0u;
+                    qa[j][2 + half] = valid ? src[4] : 0u;
+                }
+                if (half == 0) qk0 = a.qk_scale; else qk1 = a.qk_scale;
+            }
+        }
+        if constexpr (kGP == 8) {
+#pragma unroll
+            for (int j = 0; j < kKS; ++j) qa[j][1] = qa[j][3] = 0u;
+        }
+
+        float o[kNB][4];
+#pragma unroll
+        for (int nb = 0; nb < kNB; ++nb) o[nb][0] = o[nb][1] = o[nb][2] = o[nb][3] = 0.f;
+        float m0 = kNegInf, m1 = kNegInf, l0 = 0.f, l1 = 0.f;
+        int poisoned = 0;
+
+        for (int ch = s.c0; ch < s.c1; ++ch, ++it) {
+            const int stage = it % S;
+            wait_or_give_up(&full_bar[stage], (it / S) & 1, a, cta_failed);
+            poisoned |= stage_bad[stage];
+            const int n_valid = min(kChunkTokens, s.L - ch * kChunkTokens);
+            const bool tail = n_valid < kChunkTokens;
+            const uint32_t kb = smem_addr(smem + stage * C::kStageBytes);
+            const uint32_t vb = kb + C::kTileBytes;
+
+            // ---- S = Q K^T: two n-blocks of 8 tokens -------------------
+            float sc[2][4];
+#pragma unroll
+            for (int nb = 0; nb < 2; ++nb) sc[nb][0] = sc[nb][1] = sc[nb][2] = sc[nb][3] = 0.f;
+            if constexpr (kFp8) {
+#pragma unroll
+                for (int nb = 0; nb < 2; ++nb) {
+                    const int r = rb + 8 * nb + tau(g);
+                    uint32_t wk[kKS];
+                    const uint4 lo = lds128(kb + swz<C::kRowBytes, C::kSwizzle>(r, 16 * c));
+                    wk[0] = lo.x; wk[1] = lo.y; wk[2] = lo.z; wk[3] = lo.w;
+                    if constexpr (kD == 128) {
+                        const uint4 hi = lds128(kb + swz<C::kRowBytes, C::kSwizzle>(r, 16 * (4 + c)));
+                        wk[4] = hi.x; wk[5] = hi.y; wk[6] = hi.z; wk[7] = hi.w;
+                    }
+#pragma unroll
+                    for (int j = 0; j < kKS; ++j) {
+                        const uint32_t b0 = e4m3x2_to_f16x2(wk[j] & 0xFFFFu);
+                        const uint32_t b1 = e4m3x2_to_f16x2(wk[j] >> 16);
+                        mma_f16(sc[nb], qa[j][0], qa[j][1], qa[j][2], qa[j][3], b0, b1);
+                    }
+                }
+            } else {
+                const int q8 = lane >> 3;
+                const int row = rb + 8 * (q8 >> 1) + (lane & 7);
+#pragma unroll
+                for (int j = 0; j < kKS; ++j) {
+                    const int chunk16 = 2 * j + (q8 & 1);
+                    const uint32_t addr = kb + (chunk16 >> 3) * C::kSubTileBytes +
+                                          swz<128, 128>(row, (chunk16 & 7) * 16);
+                    uint32_t r0, r1, r2, r3;
+                    ldsm_x4(addr, r0, r1, r2, r3);
+                    mma_bf16(sc[0], qa[j][0], qa[j][1], qa[j][2], qa[j][3], r0, r1);
+                    mma_bf16(sc[1], qa[j][0], qa[j][1], qa[j][2], qa[j][3], r2, r3);
+                }
+            }
+
+            // ---- online softmax (log2 domain) ---------------------------
+            float p[2][4];
+#pragma unroll
+            for (int nb = 0; nb < 2; ++nb) {
+                p[nb][0] = sc[nb][0] * qk0;
+                p[nb][1] = sc[nb][1] * qk0;
+                p[nb][2] = sc[nb][2] * qk1;
+                p[nb][3] = sc[nb][3] * qk1;
+            }
+            if (tail) {
+#pragma unroll
+                for (int nb = 0; nb < 2; ++nb) {
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const int tok = kFp8 ? (rb + 8 * nb + tau(2 * c + i)) : (rb + 8 * nb + 2 * c + i);
+                        if (tok >= n_valid) p[nb][i] = p[nb][i + 2] = kNegInf;
+                    }
+                }
+            }
+            float mx0 = fmaxf(fmaxf(p[0][0], p[0][1]), fmaxf(p[1][0], p[1][1]));
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+            float mx1 = kNegInf;
+            if constexpr (kGP == 16) {
+                mx1 = fmaxf(fmaxf(p[0][2], p[0][3]), fmaxf(p[1][2], p[1][3]));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+            }
+            const bool need = (mx0 > m0 + kRescaleThreshold) || (mx1 > m1 + kRescaleThreshold);
+            if (__any_sync(0xffffffffu, need)) {
+                const float n0 = fmaxf(m0, mx0);
+                const float a0 = (n0 == kNegInf) ? 1.f : exp2f(m0 - n0);
+                m0 = n0;
+                l0 *= a0;
+                float a1 = 1.f;
+                if constexpr (kGP == 16) {
+                    const float n1 = fmaxf(m1, mx1);
+                    a1 = (n1 == kNegInf) ? 1.f : exp2f(m1 - n1);
+                    m1 = n1;
+                    l1 *= a1;
+                }
+#pragma unroll
+                for (int nb = 0; nb < kNB; ++nb) {
+                    o[nb][0] *= a0;
+                    o[nb][1] *= a0;
+                    if constexpr (kGP == 16) {
+                        o[nb][2] *= a1;
+                        o[nb][3] *= a1;
+                    }
+                }
+            }
+            const float ref0 = (m0 == kNegInf) ? 0.f : m0;
+            const float ref1 = (m1 == kNegInf) ? 0.f : m1;
+#pragma unroll
+            for (int nb = 0; nb < 2; ++nb) {
+                p[nb][0] = exp2f(p[nb][0] - ref0);
+                p[nb][1] = exp2f(p[nb][1] - ref0);
+                l0 += p[nb][0] + p[nb][1];
+                if constexpr (kGP == 16) {
+                    p[nb][2] = exp2f(p[nb][2] - ref1);
+                    p[nb][3] = exp2f(p[nb][3] - ref1);
+                    l1 += p[nb][2] + p[nb][3];
+                }
+            }
+
+            // ---- O += P V ------------------------------------------------
+            if constexpr (kFp8) {
+                const uint32_t pa0 = pack_f16x2(p[0][0], p[0][1]);
+                const uint32_t pa2 = pack_f16x2(p[1][0], p[1][1]);
+                const uint32_t pa1 = (kGP == 16) ? pack_f16x2(p[0][2], p[0][3]) : 0u;
+                const uint32_t pa3 = (kGP == 16) ? pack_f16x2(p[1][2], p[1][3]) : 0u;
+                const int r0 = rb + tau(2 * c), r1 = rb + tau(2 * c + 1);
+                const int r2 = r0 + 8, r3 = r1 + 8;
+#pragma unroll
+                for (int blk = 0; blk < kD / 32; ++blk) {
+                    const int off = 32 * blk + 4 * g;
+                    uint32_t x0 = lds32(vb + swz<C::kRowBytes, C::kSwizzle>(r0, off));
+                    uint32_t x1 = lds32(vb + swz<C::kRowBytes, C::kSwizzle>(r1, off));
+                    uint32_t x2 = lds32(vb + swz<C::kRowBytes, C::kSwizzle>(r2, off));
+                    uint32_t x3 = lds32(vb + swz<C::kRowBytes, C::kSwizzle>(r3, off));
+                    if (tail) {
+                        x0 = r0 < n_valid ? x0 : 0u;
+                        x1 = r1 < n_valid ? x1 : 0u;
+                        x2 = r2 < n_valid ? x2 : 0u;
+                        x3 = r3 < n_valid ? x3 : 0u;
+                    }
+                    const uint32_t lo01 = prmt(x0, x1, 0x5140u), hi01 = prmt(x0, x1, 0x7362u);
+                    const uint32_t lo23 = prmt(x2, x3, 0x5140u), hi23 = prmt(x2, x3, 0x7362u);
+                    mma_f16(o[4 * blk + 0], pa0, pa1, pa2, pa3, e4m3x2_to_f16x2(lo01 & 0xFFFFu),
+                            e4m3x2_to_f16x2(lo23 & 0xFFFFu));
+                    mma_f16(o[4 * blk + 1], pa0, pa1, pa2, pa3, e4m3x2_to_f16x2(lo01 >> 16),
+                            e4m3x2_to_f16x2(lo23 >> 16));
+                    mma_f16(o[4 * blk + 2], pa0, pa1, pa2, pa3, e4m3x2_to_f16x2(hi01 & 0xFFFFu),
+                            e4m3x2_to_f16x2(hi23 & 0xFFFFu));
+                    mma_f16(o[4 * blk + 3], pa0, pa1, pa2, pa3, e4m3x2_to_f16x2(hi01 >> 16),
+                            e4m3x2_to_f16x2(hi23 >> 16));
+                }
+            } else {
+                const uint32_t pa0 = pack_bf16x2(p[0][0], p[0][1]);
+                const uint32_t pa2 = pack_bf16x2(p[1][0], p[1][1]);
+                const uint32_t pa1 = (kGP == 16) ? pack_bf16x2(p[0][2], p[0][3]) : 0u;
+                const uint32_t pa3 = (kGP == 16) ? pack_bf16x2(p[1][2], p[1][3]) : 0u;
+                const int q8 = lane >> 3;
+                const int row = rb + 8 * (q8 & 1) + (lane & 7);
+                // rows of this thread's B fragments, for masking the tail
+                const int t0 = rb + 2 * c, t1 = t0 + 1, t2 = t0 + 8, t3 = t0 + 9;
+#pragma unroll
+                for (int m = 0; m < kD / 16; ++m) {
+                    const int chunk16 = 2 * m + (q8 >> 1);
+                    const uint32_t addr = vb + (chunk16 >> 3) * C::kSubTileBytes +
+                                          swz<128, 128>(row, (chunk16 & 7) * 16);
+                    uint32_t v0, v1, v2, v3;
+                    ldsm_x4_trans(addr, v0, v1, v2, v3);
+                    if (tail) {
+                        const uint32_t m01 = (t0 < n_valid ? 0x0000FFFFu : 0u) | (t1 < n_valid ? 0xFFFF0000u : 0u);
+                        const uint32_t m23 = (t2 < n_valid ? 0x0000FFFFu : 0u) | (t3 < n_valid ? 0xFFFF0000u : 0u);
+                        v0 &= m01; v2 &= m01;
+                        v1 &= m23; v3 &= m23;
+                    }
+                    mma_bf16(o[2 * m + 0], pa0, pa1, pa2, pa3, v0, v1);
+                    mma_bf16(o[2 * m + 1], pa0, pa1, pa2, pa3, v2, v3);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty_bar[stage]);
+        }
+
+        // ---- epilogue: combine the four warps, then write ---------------
+        l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+        l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+        if constexpr (kGP == 16) {
+            l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+        }
+        if (c == 0) {
+            red_m[warp * kGP + g] = m0;
+            red_l[warp * kGP + g] = l0;
+            if constexpr (kGP == 16) {
+                red_m[warp * kGP + g + 8] = m1;
+                red_l[warp * kGP + g + 8] = l1;
+            }
+        }
+#pragma unroll
+        for (int nb = 0; nb < kNB; ++nb) {
+            int d0, d1;
+            if constexpr (kFp8) {
+                // n-block 4*blk + i, column n  <->  dim 32*blk + 4*n + i
+                const int blk = nb >> 2, i = nb & 3;
+                d0 = 32 * blk + 8 * c + i;
+                d1 = d0 + 4;
+            } else {
+                d0 = 8 * nb + 2 * c;
+                d1 = d0 + 1;
+            }
+            float* dst = red_o + (warp * kGP + g) * kD;
+            dst[d0] = o[nb][0];
+            dst[d1] = o[nb][1];
+            if constexpr (kGP == 16) {
+                dst[8 * kD + d0] = o[nb][2];
+                dst[8 * kD + d1] = o[nb][3];
+            }
+        }
+        named_barrier_sync(1, kConsumerThreads);
+        for (int e = tid; e < G * kD; e += kConsumerThreads) {
+            const int hq = e / kD, d = e % kD;
+            float M = kNegInf;
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red_m[w * kGP + hq]);
+            float Lsum = 0.f, O = 0.f;
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) {
+                const float mw = red_m[w * kGP + hq];
+                const float wt = (mw == kNegInf) ? 0.f : exp2f(mw - M);
+                Lsum += wt * red_l[w * kGP + hq];
+                O += wt * red_o[(w * kGP + hq) * kD + d];
+            }
+            if (whole) {
+                if (poisoned) {
+                    a.out[(head0 + hq) * kD + d] = 0;
+                    if (d == 0) a.lse[head0 + hq] = kNegInf;
+                } else {
+                    const float val = O * a.v_scale / Lsum;
+                    a.out[(head0 + hq) * kD + d] = f32_to_bf16_bits(val);
+                    if (d == 0) a.lse[head0 + hq] = (M + log2f(Lsum)) * kLn2;
+                }
+            } else {
+                a.ws_o[(slot * G + hq) * kD + d] = poisoned ? 0.f : O * a.v_scale;
+                if (d == 0) {
+                    a.ws_ml[(slot * G + hq) * 2 + 0] = poisoned ? kNegInf : M;
+                    a.ws_ml[(slot * G + hq) * 2 + 1] = poisoned ? -1.f : Lsum;
+                }
+            }
+        }
+        named_barrier_sync(1, kConsumerThreads);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// merge: one CTA per (request, KV head) item
+// ---------------------------------------------------------------------------
+constexpr int kMergeThreads = 128;
+
+__device__ __forceinline__ int64_t cta_of_unit(int64_t u, int64_t U, int N) {
+    // largest c with floor(c * U / N) <= u
+    return ((u + 1) * N + U - 1) / U - 1;
+}
+
+template <int kD>
+__global__ void __launch_bounds__(kMergeThreads)
+attn_merge_kernel(const AttnArgs a) {
+    launch_dependents();
+    grid_dependency_wait();
+    const int Hkv = a.num_kv_heads;
+    const int item = blockIdx.x;
+    const int b = item / Hkv, h = item % Hkv;
+    const int G = a.group;
+    const int64_t head0 = static_cast<int64_t>(b) * a.num_q_heads + h * G;
+    const int32_t pre = a.ws_prefix[b];
+    const int32_t n = a.ws_prefix[b + 1] - pre;
+    if (n == 0) {
+        for (int e = threadIdx.x; e < G * kD; e += kMergeThreads) {
+            const int hq = e / kD, d = e % kD;
+            a.out[(head0 + hq) * kD + d] = 0;
+            if (d == 0) a.lse[head0 + hq] = kNegInf;
+        }
+        return;
+    }
+    const int64_t U = static_cast<int64_t>(Hkv) * a.ws_prefix[a.batch];
+    const int64_t u0 = static_cast<int64_t>(Hkv) * pre + static_cast<int64_t>(h) * n;
+    const int64_t c0 = cta_of_unit(u0, U, a.num_ctas);
+    const int64_t c1 = cta_of_unit(u0 + n - 1, U, a.num_ctas);
+    if (c0 == c1) return;   // finished by the partial kernel
+    for (int e = threadIdx.x; e < G * kD; e += kMergeThreads) {
+        const int hq = e / kD, d = e % kD;
+        float M = kNegInf;
+        bool dead = false;
+        for (int64_t cc = c0; cc <= c1; ++cc) {
+            const int64_t slot = cc + item;
+            M = fmaxf(M, a.ws_ml[(slot * G + hq) * 2 + 0]);
+            dead |= a.ws_ml[(slot * G + hq) * 2 + 1] < 0.f;
+        }
+        float Lsum = 0.f, O = 0.f;
+        for (int64_t cc = c0; cc <= c1; ++cc) {
+            const int64_t slot = cc + item;
+            const float ms = a.ws_ml[(slot * G + hq) * 2 + 0];
+            const float wt = (ms == kNegInf) ? 0.f : exp2f(ms - M);
+            Lsum += wt * a.ws_ml[(slot * G + hq) * 2 + 1];
+            O += wt * a.ws_o[(slot * G + hq) * kD + d];
+        }
+        if (dead) {
+            a.out[(head0 + hq) * kD + d] = 0;
+            if (d == 0) a.lse[head0 + hq] = kNegInf;
+        } else {
+            a.out[(head0 + hq) * kD + d] = f32_to_bf16_bits(O / Lsum);
+            if (d == 0) a.lse[head0 + hq] = (M + log2f(Lsum)) * kLn2;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host-side dispatch
+// ---------------------------------------------------------------------------
+template <bool kFp8, int kD, int kGP>
+static cudaError_t launch_variant(int grid, cudaStream_t stream, const CUtensorMap& tk,
+                                  const CUtensorMap& tv, const AttnArgs& args) {
+    using C = AttnCfg<kFp8, kD, kGP>;
+    PdlLaunch l(dim3(grid), dim3(kAttnThreads), C::kSmemBytes, stream);
+    return cudaLaunchKernelEx(&l.cfg, attn_partial_kernel<kFp8, kD, kGP>, tk, tv, args);
+}
+
+#define PKV_FOR_EACH_VARIANT(X) \
+    X(true, 64, 8) X(true, 64, 16) X(true, 128, 8) X(true, 128, 16) \
+    X(false, 64, 8) X(false, 64, 16) X(false, 128, 8) X(false, 128, 16)
+
+size_t attn_partial_smem_bytes(bool fp8, int head_dim, int group_pad) {
+#define X(F, D, GP) \
+    if (fp8 == F && head_dim == D && group_pad == GP) return AttnCfg<F, D, GP>::kSmemBytes;
+    PKV_FOR_EACH_VARIANT(X)
+#undef X
+    return 0;
+}
+
+cudaError_t attn_set_smem_attr(bool fp8, int head_dim, int group_pad) {
+#define X(F, D, GP)                                                                        \
+    if (fp8 == F && head_dim == D && group_pad == GP)                                       \
+        return cudaFuncSetAttribute(attn_partial_kernel<F, D, GP>,                          \
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,            \
+                                    AttnCfg<F, D, GP>::kSmemBytes);
+    PKV_FOR_EACH_VARIANT(X)
+#undef X
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t attn_occupancy(bool fp8, int head_dim, int group_pad, int* blocks_per_sm) {
+#define X(F, D, GP)                                                                         \
+    if (fp8 == F && head_dim == D && group_pad == GP)                                        \
+        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(                                \
+            blocks_per_sm, attn_partial_kernel<F, D, GP>, kAttnThreads,                      \
+            AttnCfg<F, D, GP>::kSmemBytes);
+    PKV_FOR_EACH_VARIANT(X)
+#undef X
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attn_partial(bool fp8, int head_dim, int group_pad, int grid,
+                                cudaStream_t stream, const CUtensorMap& tmap_k,
+                                const CUtensorMap& tmap_v, const AttnArgs& args) {
+#define X(F, D, GP) \
+    if (fp8 == F && head_dim == D && group_pad == GP) \
+        return launch_variant<F, D, GP>(grid, stream, tmap_k, tmap_v, args);
+    PKV_FOR_EACH_VARIANT(X)
+#undef X
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attn_merge(int head_dim, cudaStream_t stream, const AttnArgs& args) {
+    PdlLaunch l(dim3(args.batch * args.num_kv_heads), dim3(kMergeThreads), 0, stream);
+    if (head_dim == 64) return cudaLaunchKernelEx(&l.cfg, attn_merge_kernel<64>, args);
+    return cudaLaunchKernelEx(&l.cfg, attn_merge_kernel<128>, args);
+}
+
+}  // namespace pkv

@@ -1,0 +1,93 @@
+// internal.h -- declarations shared by the host API and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace pkv {
+
+// Tokens per pipeline stage of the attention kernels (one "chunk").
+constexpr int kChunkTokens = 64;
+
+// Arguments of the split-K partial and merge kernels (passed by value).
+struct AttnArgs {
+    const uint16_t* q;          // [B][Hq][D] bf16
+    const int32_t* page_table;  // [B][MP]
+    const int32_t* seq_lens;    // [B]
+    const uint8_t* abort;       // [B] or null
+    uint16_t* out;              // [B][Hq][D] bf16
+    float* lse;                 // [B][Hq]
+    uint32_t* ws_status;        // workspace word 0
+    int32_t* ws_prefix;         // [B + 1] chunk offsets (written by CTA 0)
+    float* ws_ml;               // [slots][G][2]  (running max in log2 units, sum)
+    float* ws_o;                // [slots][G][D]  (unnormalised, V scale applied)
+    int32_t batch;
+    int32_t max_pages;
+    int32_t num_q_heads;
+    int32_t num_kv_heads;
+    int32_t group;
+    int32_t page_size;
+    int32_t num_pages;
+    int32_t num_ctas;
+    int32_t box_rows;           // rows per TMA box = min(page_size, 64)
+    float qk_scale;             // sm_scale * k_scale * log2(e)
+    float v_scale;              // per-tensor V scale (1 for BF16)
+};
+
+// Workspace layout for given sizes and grid.
+struct WorkspaceLayout {
+    size_t prefix_off, ml_off, o_off, total;
+};
+WorkspaceLayout workspace_layout(int32_t batch, int32_t group, int32_t num_kv_heads,
+                                 int32_t head_dim, int32_t num_ctas);
+
+// Attention variant properties: dynamic shared memory bytes.  Returns 0 if
+// the combination is not compiled.
+size_t attn_partial_smem_bytes(bool fp8, int head_dim, int group_pad);
+cudaError_t attn_set_smem_attr(bool fp8, int head_dim, int group_pad);
+cudaError_t attn_occupancy(bool fp8, int head_dim, int group_pad, int* blocks_per_sm);
+constexpr int kAttnThreads = 160;   // 4 consumer warps + 1 producer warp
+
+cudaError_t launch_attn_partial(bool fp8, int head_dim, int group_pad, int grid,
+                                cudaStream_t stream, const CUtensorMap& tmap_k,
+                                const CUtensorMap& tmap_v, const AttnArgs& args);
+cudaError_t launch_attn_merge(int head_dim, cudaStream_t stream, const AttnArgs& args);
+
+cudaError_t launch_tag_check(const uint32_t* page_tags, int32_t num_pages,
+                             const int32_t* page_table, const uint32_t* expected_tags,
+                             int32_t max_pages, const int32_t* seq_lens, int32_t batch,
+                             int32_t page_size, uint8_t* abort_out, int32_t* num_aborted,
+                             cudaStream_t stream);
+
+cudaError_t launch_append(bool fp8, const uint16_t* k_new, const uint16_t* v_new,
+                          const int32_t* page_table, int32_t max_pages, const int32_t* seq_lens,
+                          int32_t batch, int32_t num_kv_heads, int32_t head_dim,
+                          int32_t page_size, float k_scale, float v_scale, void* k_cache,
+                          void* v_cache, int32_t num_pages, const uint8_t* abort,
+                          cudaStream_t stream);
+
+cudaError_t launch_requant(const uint16_t* src_pool, int32_t src_num_pages,
+                           const int32_t* src_pages, uint8_t* dst_pool, int32_t dst_num_pages,
+                           const int32_t* dst_pages, int32_t num_pairs, int64_t page_elems,
+                           float scale, cudaStream_t stream);
+
+// Launch configuration with the programmatic-stream-serialisation attribute.
+struct PdlLaunch {
+    cudaLaunchConfig_t cfg;
+    cudaLaunchAttribute attr[1];
+    PdlLaunch(dim3 grid, dim3 block, size_t smem, cudaStream_t stream) {
+        cfg = cudaLaunchConfig_t{};
+        cfg.gridDim = grid;
+        cfg.blockDim = block;
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+};
+
+}  // namespace pkv

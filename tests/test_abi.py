@@ -1,0 +1,73 @@
+"""CPU checks of the C-ABI library: it builds for sm_100a, loads without a
+GPU, exports every symbol the header declares, and rejects bad arguments on
+the host before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import paged_fp8_kv_attn_b200 as pkv
+from paged_fp8_kv_attn_b200 import build as pkv_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pagedkv.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*PKV_API\s+(?:const\s+)?[a-z_0-9]+\s*\*?\s*([a-z_][a-z_0-9]*)\s*\(", text, re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pkv_build.build()
+    return pkv.library()
+
+
+def test_header_declares_the_hot_path(lib):
+    names = _declared_functions()
+    for want in ("kv_tag_check", "kv_append_fp8", "paged_decode_attn_fp8",
+                 "paged_decode_attn_bf16", "paged_decode_attn_workspace_size", "pkv_last_error"):
+        assert want in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_library_is_built_for_sm100a():
+    log = open(os.path.join(ROOT, "paged_fp8_kv_attn_b200", "build.log")).read()
+    assert "arch=compute_100a,code=sm_100a" in log
+    assert "sm_100a" in log
+
+
+def test_version_and_error_string(lib):
+    assert pkv.version() >= 100
+    assert isinstance(lib.pkv_last_error(), bytes)
+
+
+def test_host_validation_without_a_gpu(lib):
+    P = ctypes.c_void_p
+    # unsupported head_dim is rejected before any device work
+    st = lib.kv_append_fp8(P(16), P(16), P(16), 4, P(16), 1, 1, 96, 16, 1.0, 1.0, P(16), P(16),
+                           4, None, None)
+    assert st == 3
+    assert b"head_dim" in lib.pkv_last_error()
+    # non-positive scale
+    st = lib.kv_append_fp8(P(16), P(16), P(16), 4, P(16), 1, 1, 64, 16, 0.0, 1.0, P(16), P(16),
+                           4, None, None)
+    assert st == 1
+    # GQA group not a divisor
+    st = lib.paged_decode_attn_bf16(P(16), P(16), P(16), P(16), 4, P(16), 1, 6, 4, 64, 16, 8,
+                                    0.1, None, P(16), P(16), P(256), 1 << 20, 1, None)
+    assert st == 1
+    # empty batch is a no-op
+    assert lib.kv_tag_check(None, 1, None, None, 1, None, 0, 16, None, None, None) == 0
+    # workspace query with invalid sizes returns 0
+    assert lib.paged_decode_attn_workspace_size(0, 4, 6, 4, 64, 10) == 0
+    # explicit grid: size is computable without a device
+    assert lib.paged_decode_attn_workspace_size(0, 4, 64, 8, 128, 296) > 0

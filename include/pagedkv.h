@@ -121,8 +121,8 @@ PKV_API pkv_status kv_tag_check(const uint32_t* page_tags, int32_t num_pages,
  *   k_cache[page_table[b][pos / page_size]][h][pos % page_size][d]
  * as the E4M3 code of y = x / k_scale, where y is the correctly rounded
  * binary32 quotient and the code is y rounded to nearest, ties to even,
- * with |y| > 448 (Inf included) saturated to +-448, NaN written as
- * S.1111.111 keeping its sign, and signed zeros kept.
+ * with |y| > 448 (Inf included) saturated to +-448, a NaN x written as
+ * S.1111.111 with the sign bit of x, and signed zeros kept.
  * Requests with abort[b] != 0 (abort may be NULL), a length outside
  * [1, max_pages * page_size] or a page id outside [0, num_pages) are
  * skipped.  k_new, v_new: [batch][num_kv_heads][head_dim] bf16, 16-byte

@@ -27,8 +27,9 @@
  *   - Scale granularity: one fp32 scale for K and one for V (per tensor).
  *   - Quantise: y = fp32(x) / fp32(scale) as one correctly rounded fp32
  *     division, then round y to E4M3 with round-to-nearest-even; any |y|
- *     above 448 saturates to +-448 (Inf included); NaN keeps its sign bit
- *     and becomes S.1111.111; a zero keeps its sign.
+ *     above 448 saturates to +-448 (Inf included); a NaN input x becomes
+ *     S.1111.111 with the sign bit of x (the sign of a NaN quotient is not
+ *     fixed by IEEE 754); a zero keeps its sign.
  *   - Dequantise: x = decode(code) * scale, in fp64.
  *   - Attention: s_t = sm_scale * q . k_t over t < L (L counts the new
  *     token), LSE = m + ln(sum exp(s_t - m)), o = sum exp(s_t - LSE) v_t.
@@ -141,6 +142,11 @@ uint8_t orc_quantize_bf16(uint16_t x_bits, float scale)
     uint32_t w = (uint32_t)x_bits << 16;
     float x;
     memcpy(&x, &w, sizeof x);
+    /* IEEE 754 leaves the sign of a NaN produced by an operation unspecified,
+     * so the NaN rule is stated on the input: a NaN x becomes S.1111.111 with
+     * the sign bit of x. */
+    if (isnan(x))
+        return signbit(x) ? 0xFFu : 0x7Fu;
     volatile float y = x / scale;
     return orc_e4m3_encode(y);
 }

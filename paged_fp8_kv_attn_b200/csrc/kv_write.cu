@@ -63,14 +63,16 @@ cudaError_t launch_tag_check(const uint32_t* page_tags, int32_t num_pages,
 // ---------------------------------------------------------------------------
 // E4M3 quantisation of bf16 values: y = x / scale as one correctly rounded
 // binary32 division, then the hardware's round-to-nearest-even conversion
-// with saturation to +-448; a NaN becomes S.1111.111 with its sign kept.
+// with saturation to +-448; a NaN input becomes S.1111.111 with its sign.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t quantize_pair(float x_lo, float x_hi, float scale) {
     const float y_lo = __fdiv_rn(x_lo, scale);
     const float y_hi = __fdiv_rn(x_hi, scale);
     uint32_t p = f32x2_to_e4m3x2(y_hi, y_lo);
-    if (isnan(y_lo)) p = (p & 0xFF00u) | (signbit(y_lo) ? 0xFFu : 0x7Fu);
-    if (isnan(y_hi)) p = (p & 0x00FFu) | ((signbit(y_hi) ? 0xFFu : 0x7Fu) << 8);
+    // The quotient of a NaN is a NaN of unspecified sign; the code takes the
+    // sign of the input (a finite, positive scale makes y NaN iff x is).
+    if (isnan(x_lo)) p = (p & 0xFF00u) | (signbit(x_lo) ? 0xFFu : 0x7Fu);
+    if (isnan(x_hi)) p = (p & 0x00FFu) | ((signbit(x_hi) ? 0xFFu : 0x7Fu) << 8);
     return p;
 }
 // 8 bf16 values (one 16-byte word) -> 8 codes (two 32-bit words).

@@ -164,3 +164,15 @@ def test_quantize_exact_quotients_on_midpoints(scale):
     lower = np.arange(0x7E, dtype=np.uint8)[exact]
     want = np.where(lower % 2 == 0, lower, lower + 1).astype(np.uint8)
     assert np.array_equal(oracle.quantize_bf16(bits, scale), want)
+
+
+def test_quantize_nan_takes_the_input_sign():
+    """IEEE 754 does not fix the sign of a NaN quotient, so the quantiser's
+    NaN rule is stated on its input: every NaN bf16 pattern becomes
+    S.1111.111 with the sign bit of the input, for any scale."""
+    nans = np.array([b for b in range(65536) if (b & 0x7F80) == 0x7F80 and (b & 0x7F)],
+                    dtype=np.uint16)
+    assert nans.size == 254
+    for scale in (1.0, 0.0137, 3.0):
+        got = oracle.quantize_bf16(nans, scale)
+        assert np.array_equal(got, np.where(nans & 0x8000, 0xFF, 0x7F).astype(np.uint8))

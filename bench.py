@@ -1,0 +1,629 @@
+"""Benchmark: paged FP8-KV decode attention tokens/s and HBM GB/s vs concurrency.
+
+One "step" is one pass of the whole decode hot path for one layer over one
+batch: the batched page-tag check, the FP8 quantise-and-append of every
+request's new K/V token, and paged decode attention (split-K partial + LSE
+merge), all through the C ABI on one stream.  The headline workload is the
+concurrency sweep's largest batch: 64 requests x 8,192 tokens of context,
+page size 64, 64 query heads / 8 KV heads, head_dim 128, FP8 E4M3 KV with
+per-tensor scales (synthetic, seeded).  tokens/s = requests / step time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  N > 1 runs N independent replicas (one per
+GPU, each with its own batch; no data-path collective) and reports the
+aggregate over ranks with the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged FP8-KV decode attention tokens/s & HBM GB/s (% peak) vs concurrency"
+UNIT = "tokens/s"
+HEADLINE_BATCH = 64
+CONTEXT = 8192
+SWEEP = (1, 8, 16, 32, 64)
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 2**20
+
+
+# --------------------------------------------------------------------------
+# small host-side helpers (also exercised by the CPU tests)
+# --------------------------------------------------------------------------
+
+def kv_bytes_per_step(seq_lens, num_kv_heads, head_dim, elem_bytes):
+    """Algorithmic K+V bytes attention reads in one step."""
+    return int(sum(int(L) for L in seq_lens)) * num_kv_heads * head_dim * 2 * elem_bytes
+
+
+def attn_algorithmic_bytes(seq_lens, page_size, num_q_heads, num_kv_heads, head_dim,
+                           elem_bytes):
+    """KV + q/out/lse + page-table bytes of one attention call."""
+    B = len(seq_lens)
+    kv = kv_bytes_per_step(seq_lens, num_kv_heads, head_dim, elem_bytes)
+    qo = B * num_q_heads * (2 * head_dim * 2 + 4)
+    pt = sum((int(L) + page_size - 1) // page_size for L in seq_lens) * 4
+    return kv + qo + pt
+
+
+def reduce_max_time(local_ms: float, world: int) -> float:
+    """Max of a per-rank time over the process group (identity if world == 1)."""
+    if world <= 1:
+        return local_ms
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([local_ms], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_seed(base: int, rank: int) -> int:
+    """Each replica draws its own batch."""
+    return base + 1000 * rank
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_hash(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+ATTN_SOURCES = [os.path.join(ROOT, "paged_fp8_kv_attn_b200", "csrc", n)
+                for n in ("attention.cu", "device.cuh", "internal.h")]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fp8_traffic.json")
+
+
+def ncu_traffic_per_launch(num_kv_tokens):
+    """DRAM bytes per attention launch from the committed ncu capture, scaled to
+    this launch by KV tokens; None if no capture exists or the kernel source
+    changed since it was taken."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("source_hash") != source_hash(ATTN_SOURCES):
+        return None
+    per_token = float(rec["dram_bytes_per_launch"]) / float(rec["kv_tokens"])
+    return per_token * num_kv_tokens
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------
+# GPU arm
+# --------------------------------------------------------------------------
+
+class Step:
+    """Device buffers and the C-ABI calls of one decode step."""
+
+    def __init__(self, wl, kv="fp8"):
+        import numpy as np
+        import torch
+        import paged_fp8_kv_attn_b200 as pkv
+        self.pkv = pkv
+        self.wl = wl
+        self.kv = kv
+        dev = torch.device("cuda")
+        self.q = wl.q.to(dev).contiguous()
+        self.k_new = wl.k_new.to(dev).contiguous()
+        self.v_new = wl.v_new.to(dev).contiguous()
+        self.page_table = torch.from_numpy(wl.page_table).to(dev)
+        self.seq_lens = torch.from_numpy(wl.seq_lens).to(dev)
+        self.page_tags = torch.from_numpy(wl.page_tags.view(np.int32)).to(dev)
+        self.expected = torch.from_numpy(wl.expected_tags.view(np.int32)).to(dev)
+        B, Hq, D = wl.q.shape
+        self.out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+        self.abort = torch.zeros(B, dtype=torch.uint8, device=dev)
+        if kv == "fp8":
+            self.k_cache = torch.empty(wl.k_pool.shape, dtype=torch.uint8, device=dev)
+            self.v_cache = torch.empty(wl.v_pool.shape, dtype=torch.uint8, device=dev)
+            ids = torch.arange(wl.num_pages, dtype=torch.int32, device=dev)
+            pkv.kv_requant_pages_fp8(wl.k_pool, ids, self.k_cache, ids, wl.k_scale)
+            pkv.kv_requant_pages_fp8(wl.v_pool, ids, self.v_cache, ids, wl.v_scale)
+            code = pkv.PKV_KV_FP8
+        else:
+            self.k_cache = wl.k_pool
+            self.v_cache = wl.v_pool
+            code = pkv.PKV_KV_BF16
+        self.ws = pkv.alloc_workspace(code, B, Hq, wl.num_kv_heads, D, device=dev)
+        torch.cuda.synchronize()
+
+    def check(self):
+        wl = self.wl
+        self.pkv.kv_tag_check(self.page_tags, self.page_table, self.expected, self.seq_lens,
+                              wl.page_size, self.abort)
+
+    def append(self, checked=True):
+        wl = self.wl
+        ab = self.abort if checked else None
+        if self.kv == "fp8":
+            self.pkv.kv_append_fp8(self.k_new, self.v_new, self.page_table, self.seq_lens,
+                                   wl.page_size, wl.k_scale, wl.v_scale, self.k_cache,
+                                   self.v_cache, ab)
+        else:
+            self.pkv.kv_append_bf16(self.k_new, self.v_new, self.page_table, self.seq_lens,
+                                    wl.page_size, self.k_cache, self.v_cache, ab)
+
+    def attend(self, checked=True):
+        wl = self.wl
+        ab = self.abort if checked else None
+        if self.kv == "fp8":
+            self.pkv.paged_decode_attn_fp8(self.q, self.k_cache, self.v_cache, wl.k_scale,
+                                           wl.v_scale, self.page_table, self.seq_lens,
+                                           wl.sm_scale, self.out, self.lse, self.ws, abort=ab)
+        else:
+            self.pkv.paged_decode_attn_bf16(self.q, self.k_cache, self.v_cache, self.page_table,
+                                            self.seq_lens, wl.sm_scale, self.out, self.lse,
+                                            self.ws, abort=ab)
+
+    def full(self):
+        self.check()
+        self.append(True)
+        self.attend(True)
+
+    def unchecked(self):
+        self.append(False)
+        self.attend(False)
+
+
+def _graph(fn):
+    import torch
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()                         # warm the library's per-device set-up outside capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def time_per_call(fn, steps, warmup, flush=None):
+    """Median/mean device time (us) of fn, one CUDA-event pair per call on the
+    current stream; an optional L2 flush between calls is outside the events."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps):
+        if flush is not None:
+            flush.add_(1)
+        starts[i].record()
+        fn()
+        ends[i].record()
+    torch.cuda.synchronize()
+    ts = [s.elapsed_time(e) * 1e3 for s, e in zip(starts, ends)]
+    return statistics.median(ts), sum(ts) / len(ts)
+
+
+def gpu_arm(args, rank, world):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import workloads
+
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+    props = torch.cuda.get_device_properties(torch.cuda.current_device())
+    try:
+        gpu_index = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+    except AttributeError:
+        gpu_index = str(torch.cuda.current_device())
+    peak, peak_kind = load_peaks()
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+
+    # ---- headline: full step on the B=64 batch, CUDA-graph replays ------
+    wl = workloads.concurrency_sweep(HEADLINE_BATCH, seed=replica_seed(2, rank), device="cuda")
+    st = Step(wl, "fp8")
+    g_full = _graph(st.full)
+    g_unchecked = _graph(st.unchecked)
+    for _ in range(args.warmup):
+        g_full.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = ClockSampler(gpu_index)
+    clocks.start()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        g_full.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    local_ms = e0.elapsed_time(e1)
+    clk = clocks.stop()
+    total_ms = reduce_max_time(local_ms, world)
+    ms_per_step = total_ms / args.steps
+    value = world * HEADLINE_BATCH / (ms_per_step / 1e3)
+    kv_bytes = kv_bytes_per_step(wl.seq_lens, wl.num_kv_heads, wl.head_dim, 1)
+
+    # ---- roofline of the dominant kernel: the FP8 attention call ------------
+    attn_bytes = attn_algorithmic_bytes(wl.seq_lens, wl.page_size, wl.num_q_heads,
+                                        wl.num_kv_heads, wl.head_dim, 1)
+    attn_med, attn_mean = time_per_call(lambda: st.attend(True), args.steps, args.warmup)
+    achieved = attn_bytes / (attn_mean * 1e-6) / 1e9
+    traffic = ncu_traffic_per_launch(wl.logical_tokens() * wl.num_kv_heads)
+
+    # ---- tag-check overhead: full step vs step without the check ---------
+    t_full, _ = time_per_call(g_full.replay, args.steps, args.warmup)
+    t_unch, _ = time_per_call(g_unchecked.replay, args.steps, args.warmup)
+    overhead_pct = 100.0 * (t_full - t_unch) / t_unch
+
+    # ---- end to end through the public API with host buffers -------------
+    B = HEADLINE_BATCH
+    pin = lambda t: t.detach().cpu().pin_memory()
+    h_in = {"q": pin(st.q), "k_new": pin(st.k_new), "v_new": pin(st.v_new),
+            "seq_lens": pin(st.seq_lens), "page_table": pin(st.page_table),
+            "expected": pin(st.expected)}
+    h_out = {"out": torch.empty_like(st.out, device="cpu").pin_memory(),
+             "lse": torch.empty_like(st.lse, device="cpu").pin_memory(),
+             "abort": torch.empty_like(st.abort, device="cpu").pin_memory()}
+    h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+
+    def e2e_step():
+        st.q.copy_(h_in["q"], non_blocking=True)
+        st.k_new.copy_(h_in["k_new"], non_blocking=True)
+        st.v_new.copy_(h_in["v_new"], non_blocking=True)
+        st.seq_lens.copy_(h_in["seq_lens"], non_blocking=True)
+        st.page_table.copy_(h_in["page_table"], non_blocking=True)
+        st.expected.copy_(h_in["expected"], non_blocking=True)
+        st.full()
+        h_out["out"].copy_(st.out, non_blocking=True)
+        h_out["lse"].copy_(st.lse, non_blocking=True)
+        h_out["abort"].copy_(st.abort, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max_time(e0.elapsed_time(e1), world) / args.steps
+    e2e_value = world * B / (e2e_ms / 1e3)
+    assert pkv_status_ok(st)
+    del g_full, g_unchecked, st
+    torch.cuda.empty_cache()
+
+    # ---- concurrency sweep, FP8 and BF16 side by side ---------------------
+    sweep = []
+    if not args.no_sweep:
+        for b in SWEEP:
+            wlb = workloads.concurrency_sweep(b, seed=replica_seed(2, rank), device="cuda")
+            row = {"batch": b}
+            for kv in ("fp8", "bf16"):
+                sb = Step(wlb, kv)
+                eb = 1 if kv == "fp8" else 2
+                byts = attn_algorithmic_bytes(wlb.seq_lens, wlb.page_size, wlb.num_q_heads,
+                                              wlb.num_kv_heads, wlb.head_dim, eb)
+                small = byts < 2 * L2_BYTES
+                gf = _graph(sb.full)
+                gu = _graph(sb.unchecked)
+                ga = _graph(lambda: sb.attend(True))
+                steps = max(args.steps, 20)
+                fl = flush if small else None
+                t_step, _ = time_per_call(gf.replay, steps, args.warmup, fl)
+                t_u, _ = time_per_call(gu.replay, steps, args.warmup, fl)
+                t_a, _ = time_per_call(ga.replay, steps, args.warmup, fl)
+                row[kv] = {"step_us": round(t_step, 2), "tokens_per_s": round(b / (t_step * 1e-6), 1),
+                           "attn_us": round(t_a, 2),
+                           "attn_gbs": round(byts / (t_a * 1e-6) / 1e9, 1),
+                           "attn_frac_of_measured": round(byts / (t_a * 1e-6) / 1e9 / peak, 4),
+                           "attn_frac_of_8tbs": round(byts / (t_a * 1e-6) / 1e9 / NOMINAL_HBM_GBS, 4),
+                           "check_overhead_pct": round(100.0 * (t_step - t_u) / t_u, 3),
+                           "l2": "flushed between calls" if small else "inputs larger than L2"}
+                del gf, gu, ga, sb
+                torch.cuda.empty_cache()
+            sweep.append(row)
+            del wlb
+            torch.cuda.empty_cache()
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3 cache; f16 tensor-core products, f32 accumulate",
+        "data": "synthetic (seeded; Q~N(0,1), K/V~N(0,1) with 1% x20 outliers, bf16 -> e4m3 at amax/448)",
+        "config": {"workload": f"concurrency sweep, batch {HEADLINE_BATCH} x context {CONTEXT}, "
+                               "page 64, 64 q heads / 8 kv heads, head_dim 128, FP8 E4M3 KV",
+                   "step": "tag check + FP8 append + paged attention (partial + merge), one layer",
+                   "global_batch": world * HEADLINE_BATCH, "seq_len": CONTEXT,
+                   "kv_dtype": "fp8_e4m3", "parallelism": f"replicas x{world}",
+                   "launch": "CUDA graph of the step (programmatic dependent launch)",
+                   "l2": f"inputs larger than L2 ({kv_bytes / 1e9:.2f} GB of KV per step)"},
+        "step_kv_gbs": round(kv_bytes / (ms_per_step * 1e-3) / 1e9, 1),
+        "step_kv_frac_of_8tbs": round(kv_bytes / (ms_per_step * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 4),
+        "check_overhead_pct": round(overhead_pct, 3),
+        "roofline": {"kernel": "paged_decode_attn_fp8 (split-K partial + LSE merge)",
+                     "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "peak_kind": f"{peak_kind} (copy bandwidth)",
+                     "traffic": None if traffic is None else round(traffic),
+                     "algorithmic_bytes_per_launch": attn_bytes,
+                     "launch_us_mean": round(attn_mean, 2)},
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "api": "python binding -> C ABI, eager calls, pinned host buffers"},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk,
+        "sweep": sweep,
+    }
+    return line
+
+
+def pkv_status_ok(st) -> bool:
+    return st.pkv.workspace_status(st.ws) == 0
+
+
+# --------------------------------------------------------------------------
+# CPU oracle (baseline leg and reference arm)
+# --------------------------------------------------------------------------
+
+class OracleSampler:
+    """The CPU oracle, as it stands, on a bounded sample of the headline
+    workload: R requests with the headline's per-request shape (8,192 tokens,
+    64 q heads / 8 KV heads, D=128, P=64, FP8).  One timed oracle step is the
+    tag check and the append of those requests plus attention over their
+    (request, KV head) items, run on all host cores; the time per item is
+    scaled to the 512 items of the batch-64 step."""
+
+    def __init__(self, requests: int, seed: int = 2):
+        import numpy as np
+        import oracle
+        import workloads
+        from workloads import bf16_bits
+        self.oracle = oracle
+        self.np = np
+        self.threads = os.cpu_count() or 1
+        wl = workloads.concurrency_sweep(requests, seed=seed, device="cpu", context=CONTEXT)
+        self.wl = wl
+        self.kbits, self.vbits = bf16_bits(wl.k_pool), bf16_bits(wl.v_pool)
+        self.kc = self._quantize(self.kbits, wl.k_scale)
+        self.vc = self._quantize(self.vbits, wl.v_scale)
+        self.q = bf16_bits(wl.q)
+        self.kn, self.vn = bf16_bits(wl.k_new), bf16_bits(wl.v_new)
+
+    def _quantize(self, bits, scale):
+        from concurrent.futures import ThreadPoolExecutor
+        flat = bits.reshape(-1)
+        parts = self.np.array_split(self.np.arange(flat.size), self.threads)
+        out = self.np.empty(flat.size, dtype=self.np.uint8)
+
+        def job(ix):
+            out[ix[0]: ix[-1] + 1] = self.oracle.quantize_bf16(flat[ix[0]: ix[-1] + 1], scale)
+
+        with ThreadPoolExecutor(self.threads) as ex:
+            list(ex.map(job, [p for p in parts if p.size]))
+        return out.reshape(bits.shape)
+
+    def step(self, n_items=None):
+        """Seconds of one oracle step over the first n_items items."""
+        wl, o = self.wl, self.oracle
+        total = wl.batch * wl.num_kv_heads
+        items = self.np.arange(total if n_items is None else min(n_items, total),
+                               dtype=self.np.int32)
+        t0 = time.perf_counter()
+        abort, _ = o.kv_tag_check(wl.page_tags, wl.page_table, wl.expected_tags, wl.seq_lens,
+                                  wl.page_size)
+        o.kv_append_fp8(self.kn, self.vn, wl.page_table, wl.seq_lens, wl.page_size, wl.k_scale,
+                        wl.v_scale, self.kc, self.vc, abort)
+        o.paged_decode_attn(self.q, self.kc, self.vc, wl.page_table, wl.seq_lens,
+                            wl.num_kv_heads, wl.page_size, wl.sm_scale, wl.k_scale, wl.v_scale,
+                            abort=abort, items=items, threads=self.threads)
+        return time.perf_counter() - t0, int(items.size)
+
+    def tokens_per_s(self, seconds, n_items):
+        step_s = seconds / n_items * (HEADLINE_BATCH * self.wl.num_kv_heads)
+        return HEADLINE_BATCH / step_s
+
+
+def oracle_sample(target_s: float = 10.0, seed: int = 2):
+    """cpu_baseline entry of the JSON line: the oracle timed for about
+    target_s seconds of wall time on all host cores."""
+    threads = os.cpu_count() or 1
+    probe = OracleSampler(requests=1, seed=seed)
+    t1, n1 = probe.step(n_items=min(threads, 8))
+    per_round = t1                      # one item per thread, all threads busy
+    rounds = max(1, int(target_s / max(per_round, 1e-6)))
+    n_items = min(threads * rounds, 8 * 16)
+    requests = max(1, (n_items + 7) // 8)
+    sampler = OracleSampler(requests=requests, seed=seed)
+    t, n = sampler.step(n_items=n_items)
+    return {"value": round(sampler.tokens_per_s(t, n), 4), "unit": UNIT, "cores": threads,
+            "kind": "oracle",
+            "sample": f"{n} (request, KV head) items of {requests} request(s) with the batch-64 "
+                      f"step's shape (8,192 tokens, P=64, 64/8 heads, D=128, FP8) plus their tag "
+                      f"check and append, {t:.1f} s wall on {threads} threads; scaled to the "
+                      f"512 items of the batch-64 step"}
+
+
+def reference_arm(args, rank, world):
+    """The oracle as the reference arm: each step is one oracle step over the
+    items of one request of the headline shape (a bounded sample), scaled to
+    the batch-64 step."""
+    if rank != 0:
+        return None
+    sampler = OracleSampler(requests=1)
+    for _ in range(args.warmup):
+        sampler.step()
+    secs, items = 0.0, 0
+    for _ in range(args.steps):
+        t, n = sampler.step()
+        secs += t
+        items += n
+    value = sampler.tokens_per_s(secs, items)
+    step_s = HEADLINE_BATCH / value
+    cpu = {"value": round(value, 4), "unit": UNIT, "cores": sampler.threads, "kind": "oracle",
+           "sample": f"per step: the 8 (request, KV head) items of one request of the batch-64 "
+                     f"step's shape plus its tag check and append, on {sampler.threads} "
+                     f"threads; scaled to the 512 items of the batch-64 step"}
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(step_s * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic (seeded)",
+            "config": {"workload": f"concurrency sweep, batch {HEADLINE_BATCH} x context {CONTEXT}, "
+                                   "page 64, 64 q heads / 8 kv heads, head_dim 128, FP8 E4M3 KV",
+                       "global_batch": HEADLINE_BATCH, "seq_len": CONTEXT,
+                       "parallelism": "host cores"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# --------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-only", choices=["fp8", "bf16"], default=None,
+                    help="profiling target: run only the attention call (warmup + steps "
+                         "times) on a --batch request concurrency-sweep batch; prints nothing")
+    ap.add_argument("--batch", type=int, default=16)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        line = reference_arm(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    if args.kernel_only:
+        import workloads
+        wl = workloads.concurrency_sweep(args.batch, device="cuda")
+        st = Step(wl, args.kernel_only)
+        for _ in range(args.warmup + args.steps):
+            st.check()
+            st.append(True)
+            st.attend(True)
+        torch.cuda.synchronize()
+        assert pkv_status_ok(st)
+        return
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        line = gpu_arm(args, rank, world)
+        if rank == 0 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = oracle_sample()
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

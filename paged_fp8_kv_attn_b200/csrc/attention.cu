@@ -685,9 +685,15 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
 }
 
 // ---------------------------------------------------------------------------
-// merge: one CTA per (request, KV head) item
+// merge: one CTA per (request, KV head) item.  For each query head h of the
+// item: M = max_s m_s, L = sum_s l_s 2^(m_s - M), out = sum_s O_s 2^(m_s - M) / L
+// over the item's segments s (one per CTA that worked on it).  Segment
+// weights are computed once into shared memory (in tiles of kMergeTile
+// segments, merged online), then every thread sums its (head, dim) outputs
+// with independent loads.
 // ---------------------------------------------------------------------------
-constexpr int kMergeThreads = 128;
+constexpr int kMergeThreads = 256;
+constexpr int kMergeTile = 256;
 
 __device__ __forceinline__ int64_t cta_of_unit(int64_t u, int64_t U, int N) {
     // largest c with floor(c * U / N) <= u
@@ -697,17 +703,21 @@ __device__ __forceinline__ int64_t cta_of_unit(int64_t u, int64_t U, int N) {
 template <int kD>
 __global__ void __launch_bounds__(kMergeThreads)
 attn_merge_kernel(const AttnArgs a) {
+    __shared__ float s_w[kMergeTile][16];   // weight of segment s for head h (this tile)
+    __shared__ float s_m[16], s_l[16], s_scale[16];
+    __shared__ int s_dead;
     launch_dependents();
     grid_dependency_wait();
     const int Hkv = a.num_kv_heads;
     const int item = blockIdx.x;
     const int b = item / Hkv, h = item % Hkv;
     const int G = a.group;
+    const int tid = threadIdx.x;
     const int64_t head0 = static_cast<int64_t>(b) * a.num_q_heads + h * G;
     const int32_t pre = a.ws_prefix[b];
     const int32_t n = a.ws_prefix[b + 1] - pre;
     if (n == 0) {
-        for (int e = threadIdx.x; e < G * kD; e += kMergeThreads) {
+        for (int e = tid; e < G * kD; e += kMergeThreads) {
             const int hq = e / kD, d = e % kD;
             a.out[(head0 + hq) * kD + d] = 0;
             if (d == 0) a.lse[head0 + hq] = kNegInf;
@@ -719,29 +729,90 @@ attn_merge_kernel(const AttnArgs a) {
     const int64_t c0 = cta_of_unit(u0, U, a.num_ctas);
     const int64_t c1 = cta_of_unit(u0 + n - 1, U, a.num_ctas);
     if (c0 == c1) return;   // finished by the partial kernel
-    for (int e = threadIdx.x; e < G * kD; e += kMergeThreads) {
-        const int hq = e / kD, d = e % kD;
-        float M = kNegInf;
-        bool dead = false;
-        for (int64_t cc = c0; cc <= c1; ++cc) {
-            const int64_t slot = cc + item;
-            M = fmaxf(M, a.ws_ml[(slot * G + hq) * 2 + 0]);
-            dead |= a.ws_ml[(slot * G + hq) * 2 + 1] < 0.f;
+    const int nseg = static_cast<int>(c1 - c0 + 1);
+    if (tid < 16) {
+        s_m[tid] = kNegInf;
+        s_l[tid] = 0.f;
+    }
+    if (tid == 0) s_dead = 0;
+    // every thread owns the same (head, dim) outputs across tiles
+    constexpr int kPer = (16 * kD + kMergeThreads - 1) / kMergeThreads;
+    float acc[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
+    __syncthreads();
+
+    for (int t0 = 0; t0 < nseg; t0 += kMergeTile) {
+        const int tn = min(kMergeTile, nseg - t0);
+        // (1) per head: tile max, rescale of the running state
+        for (int hq = tid >> 5; hq < G; hq += kMergeThreads / 32) {
+            float mx = kNegInf;
+            int dead = 0;
+            for (int s = (tid & 31); s < tn; s += 32) {
+                const int64_t slot = c0 + t0 + s + item;
+                mx = fmaxf(mx, a.ws_ml[(slot * G + hq) * 2 + 0]);
+                dead |= a.ws_ml[(slot * G + hq) * 2 + 1] < 0.f;
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                dead |= __shfl_xor_sync(0xffffffffu, dead, off);
+            }
+            if ((tid & 31) == 0) {
+                if (dead) s_dead = 1;
+                const float m_old = s_m[hq];
+                const float m_new = fmaxf(m_old, mx);
+                const float r = (m_old == kNegInf) ? 0.f : exp2f(m_old - m_new);
+                s_scale[hq] = r;          // factor for what was accumulated so far
+                s_l[hq] *= r;
+                s_m[hq] = m_new;
+            }
         }
-        float Lsum = 0.f, O = 0.f;
-        for (int64_t cc = c0; cc <= c1; ++cc) {
-            const int64_t slot = cc + item;
+        __syncthreads();
+        // (2) segment weights relative to the running max, and the sum
+        for (int e = tid; e < tn * G; e += kMergeThreads) {
+            const int s = e / G, hq = e % G;
+            const int64_t slot = c0 + t0 + s + item;
             const float ms = a.ws_ml[(slot * G + hq) * 2 + 0];
-            const float wt = (ms == kNegInf) ? 0.f : exp2f(ms - M);
-            Lsum += wt * a.ws_ml[(slot * G + hq) * 2 + 1];
-            O += wt * a.ws_o[(slot * G + hq) * kD + d];
+            s_w[s][hq] = (ms == kNegInf) ? 0.f : exp2f(ms - s_m[hq]);
         }
-        if (dead) {
+        __syncthreads();
+        for (int hq = tid >> 5; hq < G; hq += kMergeThreads / 32) {
+            float lsum = 0.f;
+            for (int s = (tid & 31); s < tn; s += 32) {
+                const int64_t slot = c0 + t0 + s + item;
+                lsum += s_w[s][hq] * a.ws_ml[(slot * G + hq) * 2 + 1];
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+            if ((tid & 31) == 0) s_l[hq] += lsum;
+        }
+        // (3) outputs: independent loads over the tile's segments
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            const int e = tid + k * kMergeThreads;
+            if (e >= G * kD) break;
+            const int hq = e / kD, d = e % kD;
+            float o = acc[k] * s_scale[hq];
+            const float* src = a.ws_o + ((c0 + t0 + item) * G + hq) * kD + d;
+            const int64_t stride = static_cast<int64_t>(G) * kD;
+#pragma unroll 8
+            for (int s = 0; s < tn; ++s) o += s_w[s][hq] * src[s * stride];
+            acc[k] = o;
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const int e = tid + k * kMergeThreads;
+        if (e >= G * kD) break;
+        const int hq = e / kD, d = e % kD;
+        if (s_dead) {
             a.out[(head0 + hq) * kD + d] = 0;
             if (d == 0) a.lse[head0 + hq] = kNegInf;
         } else {
-            a.out[(head0 + hq) * kD + d] = f32_to_bf16_bits(O / Lsum);
-            if (d == 0) a.lse[head0 + hq] = (M + log2f(Lsum)) * kLn2;
+            a.out[(head0 + hq) * kD + d] = f32_to_bf16_bits(acc[k] / s_l[hq]);
+            if (d == 0) a.lse[head0 + hq] = (s_m[hq] + log2f(s_l[hq])) * kLn2;
         }
     }
 }

@@ -23,8 +23,11 @@ tag_check_kernel(const uint32_t* __restrict__ page_tags, int32_t num_pages,
                  const uint32_t* __restrict__ expected_tags, int32_t max_pages,
                  const int32_t* __restrict__ seq_lens, int32_t page_size,
                  uint8_t* __restrict__ abort_out, int32_t* __restrict__ num_aborted) {
-    grid_dependency_wait();
+    // Let the next kernel on the stream launch at once (its own prologue
+    // overlaps this grid); it still waits for this grid to finish before it
+    // reads anything this grid writes.
     launch_dependents();
+    grid_dependency_wait();
     const int b = blockIdx.x;
     const int32_t L = seq_lens[b];
     int bad = (L < 1 || static_cast<int64_t>(L) > static_cast<int64_t>(max_pages) * page_size);
@@ -97,8 +100,11 @@ append_kernel(const uint16_t* __restrict__ k_new, const uint16_t* __restrict__ v
               const int32_t* __restrict__ seq_lens, int32_t num_kv_heads, int32_t head_dim,
               int32_t page_size, float k_scale, float v_scale, void* __restrict__ k_cache,
               void* __restrict__ v_cache, int32_t num_pages, const uint8_t* __restrict__ abort) {
-    grid_dependency_wait();
+    // Let the next kernel on the stream launch at once (its own prologue
+    // overlaps this grid); it still waits for this grid to finish before it
+    // reads anything this grid writes.
     launch_dependents();
+    grid_dependency_wait();
     const int b = blockIdx.x;
     const int32_t L = seq_lens[b];
     if (L < 1 || static_cast<int64_t>(L) > static_cast<int64_t>(max_pages) * page_size) return;
@@ -154,8 +160,11 @@ requant_kernel(const uint16_t* __restrict__ src_pool, int32_t src_num_pages,
                const int32_t* __restrict__ src_pages, uint8_t* __restrict__ dst_pool,
                int32_t dst_num_pages, const int32_t* __restrict__ dst_pages, int32_t num_pairs,
                int64_t page_elems, float scale) {
-    grid_dependency_wait();
+    // Let the next kernel on the stream launch at once (its own prologue
+    // overlaps this grid); it still waits for this grid to finish before it
+    // reads anything this grid writes.
     launch_dependents();
+    grid_dependency_wait();
     const int64_t groups = page_elems / 16;
     const int64_t total = static_cast<int64_t>(num_pairs) * groups;
     for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;

@@ -1,0 +1,83 @@
+"""Host-side logic of bench.py on the CPU: byte accounting, replica seeds and
+the max-over-ranks timing reduction with two gloo ranks."""
+import os
+import socket
+import sys
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def test_algorithmic_bytes_headline():
+    lens = [8192] * 64
+    kv = bench.kv_bytes_per_step(lens, 8, 128, 1)
+    assert kv == 64 * 8192 * 8 * 128 * 2 == 1_073_741_824
+    total = bench.attn_algorithmic_bytes(lens, 64, 64, 8, 128, 1)
+    assert total == kv + 64 * 64 * (2 * 128 * 2 + 4) + 64 * 128 * 4
+    assert bench.attn_algorithmic_bytes(lens, 64, 64, 8, 128, 2) - total == kv
+
+
+def test_replica_seeds_are_distinct():
+    seeds = {bench.replica_seed(2, r) for r in range(8)}
+    assert len(seeds) == 8
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    import datetime
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        out[rank] = bench.reduce_max_time(1.5 + rank, world)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo():
+    world = 2
+    port = _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    ctx = mp.get_context("spawn")
+    procs = [ctx.Process(target=_worker, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    assert dict(out) == {0: 2.5, 1: 2.5}
+
+
+def test_reference_arm_line_shape(monkeypatch):
+    class FakeSampler:
+        threads = 3
+
+        def __init__(self, requests, seed=2):
+            self.wl = type("W", (), {"num_kv_heads": 8})()
+
+        def step(self, n_items=None):
+            return 0.5, 8
+
+        def tokens_per_s(self, seconds, n):
+            return bench.HEADLINE_BATCH / (seconds / n * 512)
+
+    monkeypatch.setattr(bench, "OracleSampler", FakeSampler)
+    args = type("A", (), {"warmup": 3, "steps": 2})()
+    line = bench.reference_arm(args, 0, 1)
+    assert line["impl"] == "reference"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 3
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
+    assert bench.reference_arm(args, 1, 2) is None

@@ -128,7 +128,7 @@ def test_append_bit_exact(cuda_device, kv, P, D, Hkv):
     abort = np.zeros(wl.batch, dtype=np.uint8)
     abort[::5] = 1
     db.abort.copy_(torch.from_numpy(abort))
-    before_k = db.k_cache.cpu().numpy().copy()
+    before_k = db.k_cache.cpu().numpy().copy() if kv == "fp8" else None
     db.append(use_abort=True)
     torch.cuda.synchronize()
     if kv == "fp8":

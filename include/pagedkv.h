@@ -233,6 +233,44 @@ PKV_API pkv_status paged_decode_attn_bf16(const uint16_t* q, const uint16_t* k_c
                                   void* workspace, size_t workspace_bytes, int32_t num_ctas,
                                   void* stream);
 
+/*
+ * paged_decode_attn_fp8_noalloc -- paged_decode_attn_fp8 for callers that
+ * cannot allocate device memory.  The source pages have no counterpart to
+ * this call; it exists for integration only.
+ *
+ * Some callers cannot hand the attention call a workspace: a plugin whose
+ * host framework passes it only its inputs and outputs and owns every other
+ * allocation, or a latency-critical path where cudaMalloc / cudaFree would
+ * implicitly synchronise the device.  This call takes the same arguments as
+ * paged_decode_attn_fp8 without the workspace and runs the same kernels,
+ * using instead a scratch array compiled into the library:
+ *   - its size is paged_decode_attn_fp8_noalloc_scratch_bytes() (8 MiB); every
+ *     GPU that loads the library holds it until the process exits;
+ *   - sizes whose workspace (paged_decode_attn_workspace_size(PKV_KV_FP8, ...))
+ *     would exceed it are rejected with PKV_ERR_WORKSPACE and a message; with
+ *     the default grid on a B200 that is roughly batch * num_kv_heads > 1700
+ *     at head_dim 128 and a GQA group of 8;
+ *   - the first call on a device looks up the array's device address for that
+ *     device (make that first call before any stream capture);
+ *   - the call allocates and frees nothing; it clears the array's status word
+ *     on the stream and otherwise relies on the kernels writing every scratch
+ *     value before reading it (the array keeps the previous call's contents);
+ *   - all calls on a device share the one array, so two calls whose work
+ *     overlaps on the GPU (different streams, or different host threads
+ *     without ordering) race and corrupt each other's results.
+ */
+PKV_API pkv_status paged_decode_attn_fp8_noalloc(const uint16_t* q, const uint8_t* k_cache,
+                                         const uint8_t* v_cache, float k_scale, float v_scale,
+                                         const int32_t* page_table, int32_t max_pages,
+                                         const int32_t* seq_lens, int32_t batch,
+                                         int32_t num_q_heads, int32_t num_kv_heads,
+                                         int32_t head_dim, int32_t page_size, int32_t num_pages,
+                                         float sm_scale, const uint8_t* abort, uint16_t* out,
+                                         float* lse, int32_t num_ctas, void* stream);
+
+/* Bytes of the built-in scratch used by paged_decode_attn_fp8_noalloc. */
+PKV_API size_t paged_decode_attn_fp8_noalloc_scratch_bytes(void);
+
 /* Message describing the last non-OK status returned on this thread. */
 PKV_API const char* pkv_last_error(void);
 

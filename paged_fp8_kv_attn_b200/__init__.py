@@ -66,6 +66,11 @@ def _load():
             fn = getattr(lib, name)
             fn.argtypes = args
             fn.restype = i32
+        lib.paged_decode_attn_fp8_noalloc.argtypes = [P, P, P, f32, f32, P, i32, P, i32, i32,
+                                                      i32, i32, i32, i32, f32, P, P, P, i32, P]
+        lib.paged_decode_attn_fp8_noalloc.restype = i32
+        lib.paged_decode_attn_fp8_noalloc_scratch_bytes.argtypes = []
+        lib.paged_decode_attn_fp8_noalloc_scratch_bytes.restype = sz
         lib.paged_decode_attn_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
         lib.paged_decode_attn_workspace_size.restype = sz
         lib.pkv_last_error.argtypes = []
@@ -243,6 +248,33 @@ def paged_decode_attn_bf16(q, k_cache, v_cache, page_table, seq_lens, sm_scale, 
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(page_table), page_table.shape[1],
         _ptr(seq_lens), B, Hq, Hkv, D, P, NP, float(sm_scale), _ptr(abort), _ptr(out), _ptr(lse),
         _ptr(workspace), workspace.numel(), num_ctas, _stream(stream)))
+
+
+def paged_decode_attn_fp8_noalloc(q, k_cache, v_cache, k_scale, v_scale, page_table, seq_lens,
+                                  sm_scale, out, lse, abort=None, num_ctas=0, stream=None):
+    """paged_decode_attn_fp8 without a workspace argument, for callers that
+    cannot allocate device memory: the library uses its built-in scratch array
+    (see paged_decode_attn_fp8_noalloc_scratch_bytes()).  Calls that overlap
+    on the GPU share that array and must not run concurrently."""
+    _need(k_cache, torch.uint8, 4, "k_cache")
+    _need(v_cache, torch.uint8, 4, "v_cache")
+    _need(q, torch.bfloat16, 3, "q")
+    _need(page_table, torch.int32, 2, "page_table")
+    _need(seq_lens, torch.int32, 1, "seq_lens")
+    _need(out, torch.bfloat16, 3, "out")
+    _need(lse, torch.float32, 2, "lse")
+    if abort is not None:
+        _need(abort, torch.uint8, 1, "abort")
+    B, Hq, D = q.shape
+    NP, Hkv, P, _ = k_cache.shape
+    _check("paged_decode_attn_fp8_noalloc", _load().paged_decode_attn_fp8_noalloc(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), float(k_scale), float(v_scale), _ptr(page_table),
+        page_table.shape[1], _ptr(seq_lens), B, Hq, Hkv, D, P, NP, float(sm_scale), _ptr(abort),
+        _ptr(out), _ptr(lse), num_ctas, _stream(stream)))
+
+
+def noalloc_scratch_bytes() -> int:
+    return int(_load().paged_decode_attn_fp8_noalloc_scratch_bytes())
 
 
 def version() -> int:

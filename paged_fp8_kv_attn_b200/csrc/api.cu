@@ -238,6 +238,8 @@ pkv_status attn_impl(bool fp8, const uint16_t* q, const void* k_cache, const voi
 }  // namespace
 
 namespace pkv {
+void set_last_error(const char* message) { g_last_error = message; }
+
 WorkspaceLayout workspace_layout(int32_t batch, int32_t group, int32_t num_kv_heads,
                                  int32_t head_dim, int32_t num_ctas) {
     WorkspaceLayout l{};

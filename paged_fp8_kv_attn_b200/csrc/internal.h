@@ -36,6 +36,9 @@ struct AttnArgs {
     float v_scale;              // per-tensor V scale (1 for BF16)
 };
 
+// Sets the message pkv_last_error() returns on this thread.
+void set_last_error(const char* message);
+
 // Workspace layout for given sizes and grid.
 struct WorkspaceLayout {
     size_t prefix_off, ml_off, o_off, total;

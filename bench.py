@@ -308,7 +308,13 @@ def gpu_arm(args, rank, world):
         dist.barrier()
     clocks = ClockSampler(gpu_index)
     clocks.start()
-    torch.cuda.synchronize()
+    # keep the GPU busy for ~1 s before the timed steps so that the clock
+    # samples describe the same load the timed region runs under
+    soak_until = time.perf_counter() + 1.0
+    while time.perf_counter() < soak_until:
+        for _ in range(200):
+            g_full.replay()
+        torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()

@@ -40,9 +40,9 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_library_is_built_for_sm100a():
-    log = open(os.path.join(ROOT, "paged_fp8_kv_attn_b200", "build.log")).read()
-    assert "arch=compute_100a,code=sm_100a" in log
-    assert "sm_100a" in log
+    flags = " ".join(pkv_build.NVCC_FLAGS)
+    assert "arch=compute_100a,code=sm_100a" in flags
+    assert "compute_90" not in flags and "sm_90" not in flags
 
 
 def test_version_and_error_string(lib):

@@ -346,13 +346,36 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
     }
 
     // ================= consumer warps =================
+    // Per warp and chunk: the 16 token rows rb..rb+15.  S = K Q^T and
+    // O^T = V^T P^T run as m16n8k16 MMAs whose M dimension is 16 tokens (QK)
+    // or 16 head dimensions (PV) and whose N dimension is 8 query heads of
+    // the GQA group (kNB n-blocks of 8).  P is moved from the S accumulator
+    // layout into the PV B-operand layout with an in-register 8x8 transpose.
     grid_dependency_wait();
-    const int g = lane >> 2;   // MMA group id: head row g (and g + 8)
+    const int g = lane >> 2;   // MMA group id
     const int c = lane & 3;    // thread in group
     const int G = a.group;
     const int rb = warp * 16;  // this warp's rows of each chunk
-    constexpr int kNB = kD / 8;       // n-blocks of the output
+    constexpr int kNB = kGP / 8;      // n-blocks of query heads
+    constexpr int kMB = kD / 16;      // m-blocks of the head dimension (PV)
     constexpr int kKS = kD / 16;      // k-steps of the QK contraction
+
+    // Fixed shared-memory offsets of this thread's K and V reads.
+    uint32_t k_off[2][kD / 64];       // FP8: rows tau(g), 8+tau(g); chunks c, 4+c
+    uint32_t v_off[4];                // FP8: rows tau(2c), tau(2c+1), 8+.., 8+..; chunk g
+    if constexpr (kFp8) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half)
+#pragma unroll
+            for (int part = 0; part < kD / 64; ++part)
+                k_off[half][part] = swz<C::kRowBytes, C::kSwizzle>(rb + 8 * half + tau(g),
+                                                                   16 * (4 * part + c));
+        const int vr[4] = {rb + tau(2 * c), rb + tau(2 * c + 1), rb + 8 + tau(2 * c),
+                           rb + 8 + tau(2 * c + 1)};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            v_off[i] = swz<C::kRowBytes, C::kSwizzle>(vr[i], (kD == 128 ? 16 : 8) * g);
+    }
 
     uint32_t it = 0;
     Segment s;
@@ -379,16 +402,18 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
             continue;
         }
 
-        // ---- query fragments (A operand, rows = heads g and g + 8) -------
-        uint32_t qa[kKS][4];
-        float qk0 = 0.f, qk1 = 0.f;
+        // ---- Q^T as the B operand: column n = head g (+8 per n-block) -----
+        uint32_t qb[kNB][kKS][2];
+        float qs[kNB][2];   // score scale of S columns 2c and 2c+1
 #pragma unroll
-        for (int half = 0; half < (kGP == 16 ? 2 : 1); ++half) {
-            const int hh = g + 8 * half;
+        for (int nb = 0; nb < kNB; ++nb) {
+            const int hh = g + 8 * nb;
             const bool valid = hh < G;
             const uint16_t* qrow = a.q + (head0 + (valid ? hh : 0)) * kD;
+            float my_scale;
             if constexpr (kFp8) {
-                // this thread's dims: [16c, 16c+16) and, for D=128, [64+16c, 64+16c+16)
+                // this thread's dims: [16c, 16c+16) and, for D=128, [64+16c, 64+16c+16);
+                // word j of them holds dims D_c[4j..4j+3] of the permuted contraction
                 float v[kD / 4];
 #pragma unroll
                 for (int part = 0; part < kD / 64; ++part) {
@@ -414,31 +439,35 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 }
 #pragma unroll
                 for (int j = 0; j < kKS; ++j) {
-                    qa[j][half] = pack_f16x2(ldexpf(v[4 * j], shift), ldexpf(v[4 * j + 1], shift));
-                    qa[j][2 + half] =
-                        pack_f16x2(ldexpf(v[4 * j + 2], shift), ldexpf(v[4 * j + 3], shift));
+                    qb[nb][j][0] = pack_f16x2(ldexpf(v[4 * j], shift), ldexpf(v[4 * j + 1], shift));
+                    qb[nb][j][1] = pack_f16x2(ldexpf(v[4 * j + 2], shift), ldexpf(v[4 * j + 3], shift));
                 }
-                const float qs = a.qk_scale * ldexpf(1.f, -shift);
-                if (half == 0) qk0 = qs; else qk1 = qs;
+                my_scale = a.qk_scale * ldexpf(1.f, -shift);
             } else {
 #pragma unroll
                 for (int j = 0; j < kKS; ++j) {
                     const uint32_t* src = reinterpret_cast<const uint32_t*>(qrow + 16 * j + 2 * c);
-                    qa[j][half] = valid ? src[0] : 0u;
-                    qa[j][2 + half] = valid ? src[4] : 0u;
+                    qb[nb][j][0] = valid ? src[0] : 0u;
+                    qb[nb][j][1] = valid ? src[4] : 0u;
                 }
-                if (half == 0) qk0 = a.qk_scale; else qk1 = a.qk_scale;
+                my_scale = a.qk_scale;
             }
-        }
-        if constexpr (kGP == 8) {
-#pragma unroll
-            for (int j = 0; j < kKS; ++j) qa[j][1] = qa[j][3] = 0u;
+            // column 2c + col of this n-block is head 2c + col, owned by lanes 4(2c+col)+*
+            qs[nb][0] = __shfl_sync(0xffffffffu, my_scale, 4 * (2 * c));
+            qs[nb][1] = __shfl_sync(0xffffffffu, my_scale, 4 * (2 * c + 1));
         }
 
-        float o[kNB][4];
+        float o[kNB][kMB][4];
 #pragma unroll
-        for (int nb = 0; nb < kNB; ++nb) o[nb][0] = o[nb][1] = o[nb][2] = o[nb][3] = 0.f;
-        float m0 = kNegInf, m1 = kNegInf, l0 = 0.f, l1 = 0.f;
+        for (int nb = 0; nb < kNB; ++nb)
+#pragma unroll
+            for (int mb = 0; mb < kMB; ++mb) o[nb][mb][0] = o[nb][mb][1] = o[nb][mb][2] = o[nb][mb][3] = 0.f;
+        float m[kNB][2], l[kNB][2];
+#pragma unroll
+        for (int nb = 0; nb < kNB; ++nb) {
+            m[nb][0] = m[nb][1] = kNegInf;
+            l[nb][0] = l[nb][1] = 0.f;
+        }
         int poisoned = 0;
 
         for (int ch = s.c0; ch < s.c1; ++ch, ++it) {
@@ -450,164 +479,176 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const uint32_t kb = smem_addr(smem + stage * C::kStageBytes);
             const uint32_t vb = kb + C::kTileBytes;
 
-            // ---- S = Q K^T: two n-blocks of 8 tokens -------------------
-            float sc[2][4];
+            // ---- S[16 tokens][8 heads] = K Q^T, two accumulator chains ------
+            float acc[kNB][2][4];
 #pragma unroll
-            for (int nb = 0; nb < 2; ++nb) sc[nb][0] = sc[nb][1] = sc[nb][2] = sc[nb][3] = 0.f;
+            for (int nb = 0; nb < kNB; ++nb)
+#pragma unroll
+                for (int q = 0; q < 2; ++q) acc[nb][q][0] = acc[nb][q][1] = acc[nb][q][2] = acc[nb][q][3] = 0.f;
             if constexpr (kFp8) {
+                uint32_t wa[kKS], wb[kKS];
 #pragma unroll
-                for (int nb = 0; nb < 2; ++nb) {
-                    const int r = rb + 8 * nb + tau(g);
-                    uint32_t wk[kKS];
-                    const uint4 lo = lds128(kb + swz<C::kRowBytes, C::kSwizzle>(r, 16 * c));
-                    wk[0] = lo.x; wk[1] = lo.y; wk[2] = lo.z; wk[3] = lo.w;
-                    if constexpr (kD == 128) {
-                        const uint4 hi = lds128(kb + swz<C::kRowBytes, C::kSwizzle>(r, 16 * (4 + c)));
-                        wk[4] = hi.x; wk[5] = hi.y; wk[6] = hi.z; wk[7] = hi.w;
+                for (int part = 0; part < kD / 64; ++part) {
+                    const uint4 x = lds128(kb + k_off[0][part]);
+                    const uint4 y = lds128(kb + k_off[1][part]);
+                    wa[4 * part + 0] = x.x; wa[4 * part + 1] = x.y; wa[4 * part + 2] = x.z; wa[4 * part + 3] = x.w;
+                    wb[4 * part + 0] = y.x; wb[4 * part + 1] = y.y; wb[4 * part + 2] = y.z; wb[4 * part + 3] = y.w;
+                }
+#pragma unroll
+                for (int j = 0; j < kKS; ++j) {
+                    uint32_t a0, a2, a1, a3;
+                    e4m3x4_to_f16x2x2(wa[j], a0, a2);   // token row tau(g): k 2c.. / 2c+8..
+                    e4m3x4_to_f16x2x2(wb[j], a1, a3);   // token row 8+tau(g)
+#pragma unroll
+                    for (int nb = 0; nb < kNB; ++nb)
+                        mma_f16(acc[nb][j & 1], a0, a1, a2, a3, qb[nb][j][0], qb[nb][j][1]);
+                }
+            } else {
+                const int q8 = lane >> 3;
+                const int row = rb + 8 * (q8 & 1) + (lane & 7);
+#pragma unroll
+                for (int j = 0; j < kKS; ++j) {
+                    const int chunk16 = 2 * j + (q8 >> 1);
+                    const uint32_t addr = kb + (chunk16 >> 3) * C::kSubTileBytes +
+                                          swz<128, 128>(row, (chunk16 & 7) * 16);
+                    uint32_t a0, a1, a2, a3;
+                    ldsm_x4(addr, a0, a1, a2, a3);
+#pragma unroll
+                    for (int nb = 0; nb < kNB; ++nb)
+                        mma_bf16(acc[nb][j & 1], a0, a1, a2, a3, qb[nb][j][0], qb[nb][j][1]);
+                }
+            }
+
+            // ---- online softmax over the 16 tokens, per head (log2 units) ----
+            // p[nb][0..1]: token row g, heads 2c, 2c+1; p[nb][2..3]: row g + 8
+            float p[kNB][4];
+#pragma unroll
+            for (int nb = 0; nb < kNB; ++nb)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    p[nb][i] = (acc[nb][0][i] + acc[nb][1][i]) * qs[nb][i & 1];
+            if (tail) {
+                const int t_lo = kFp8 ? rb + tau(g) : rb + g;
+                const int t_hi = t_lo + 8;
+#pragma unroll
+                for (int nb = 0; nb < kNB; ++nb) {
+                    if (t_lo >= n_valid) p[nb][0] = p[nb][1] = kNegInf;
+                    if (t_hi >= n_valid) p[nb][2] = p[nb][3] = kNegInf;
+                }
+            }
+            float mx[kNB][2];
+            bool need = false;
+#pragma unroll
+            for (int nb = 0; nb < kNB; ++nb)
+#pragma unroll
+                for (int col = 0; col < 2; ++col) {
+                    float v = fmaxf(p[nb][col], p[nb][col + 2]);
+                    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+                    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+                    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+                    mx[nb][col] = v;
+                    need |= v > m[nb][col] + kRescaleThreshold;
+                }
+            if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+                for (int nb = 0; nb < kNB; ++nb) {
+                    float alpha[2];
+#pragma unroll
+                    for (int col = 0; col < 2; ++col) {
+                        const float nm = fmaxf(m[nb][col], mx[nb][col]);
+                        alpha[col] = (nm == kNegInf) ? 1.f : exp2f(m[nb][col] - nm);
+                        m[nb][col] = nm;
+                        l[nb][col] *= alpha[col];
                     }
 #pragma unroll
-                    for (int j = 0; j < kKS; ++j) {
-                        const uint32_t b0 = e4m3x2_to_f16x2(wk[j] & 0xFFFFu);
-                        const uint32_t b1 = e4m3x2_to_f16x2(wk[j] >> 16);
-                        mma_f16(sc[nb], qa[j][0], qa[j][1], qa[j][2], qa[j][3], b0, b1);
+                    for (int mb = 0; mb < kMB; ++mb) {
+                        o[nb][mb][0] *= alpha[0];
+                        o[nb][mb][1] *= alpha[1];
+                        o[nb][mb][2] *= alpha[0];
+                        o[nb][mb][3] *= alpha[1];
                     }
+                }
+            }
+            // P^T as the PV B operand: k = token row, n = head g
+            uint32_t pb[kNB][2];
+#pragma unroll
+            for (int nb = 0; nb < kNB; ++nb) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float ref = (m[nb][i & 1] == kNegInf) ? 0.f : m[nb][i & 1];
+                    p[nb][i] = exp2f(p[nb][i] - ref);
+                }
+                l[nb][0] += p[nb][0] + p[nb][2];
+                l[nb][1] += p[nb][1] + p[nb][3];
+                if constexpr (kFp8) {
+                    pb[nb][0] = movmatrix_trans(pack_f16x2(p[nb][0], p[nb][1]));
+                    pb[nb][1] = movmatrix_trans(pack_f16x2(p[nb][2], p[nb][3]));
+                } else {
+                    pb[nb][0] = movmatrix_trans(pack_bf16x2(p[nb][0], p[nb][1]));
+                    pb[nb][1] = movmatrix_trans(pack_bf16x2(p[nb][2], p[nb][3]));
+                }
+            }
+
+            // ---- O^T[16 dims][8 heads] += V^T P^T per m-block of dims --------
+            if constexpr (kFp8) {
+                constexpr int kW = kD / 32;   // 32-bit words per thread and row: 4 (D=128), 2 (D=64)
+                uint32_t x[4][kW];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    if constexpr (kW == 4) {
+                        const uint4 t = lds128(vb + v_off[r]);
+                        x[r][0] = t.x; x[r][1] = t.y; x[r][2] = t.z; x[r][3] = t.w;
+                    } else {
+                        const uint2 t = lds64(vb + v_off[r]);
+                        x[r][0] = t.x; x[r][1] = t.y;
+                    }
+                }
+                if (tail) {
+                    const int vr[4] = {rb + tau(2 * c), rb + tau(2 * c + 1), rb + 8 + tau(2 * c),
+                                       rb + 8 + tau(2 * c + 1)};
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+                        if (vr[r] >= n_valid)
+#pragma unroll
+                            for (int q = 0; q < kW; ++q) x[r][q] = 0u;
+                }
+#pragma unroll
+                for (int q = 0; q < kW; ++q) {
+                    // word q holds dims 4q..4q+3 of this thread's block: m-blocks 2q, 2q+1
+                    uint32_t a0, a1, a2, a3;
+                    e4m3x4_to_f16x2x2(prmt(x[0][q], x[1][q], 0x5140u), a0, a1);
+                    e4m3x4_to_f16x2x2(prmt(x[2][q], x[3][q], 0x5140u), a2, a3);
+#pragma unroll
+                    for (int nb = 0; nb < kNB; ++nb)
+                        mma_f16(o[nb][2 * q], a0, a1, a2, a3, pb[nb][0], pb[nb][1]);
+                    e4m3x4_to_f16x2x2(prmt(x[0][q], x[1][q], 0x7362u), a0, a1);
+                    e4m3x4_to_f16x2x2(prmt(x[2][q], x[3][q], 0x7362u), a2, a3);
+#pragma unroll
+                    for (int nb = 0; nb < kNB; ++nb)
+                        mma_f16(o[nb][2 * q + 1], a0, a1, a2, a3, pb[nb][0], pb[nb][1]);
                 }
             } else {
                 const int q8 = lane >> 3;
                 const int row = rb + 8 * (q8 >> 1) + (lane & 7);
-#pragma unroll
-                for (int j = 0; j < kKS; ++j) {
-                    const int chunk16 = 2 * j + (q8 & 1);
-                    const uint32_t addr = kb + (chunk16 >> 3) * C::kSubTileBytes +
-                                          swz<128, 128>(row, (chunk16 & 7) * 16);
-                    uint32_t r0, r1, r2, r3;
-                    ldsm_x4(addr, r0, r1, r2, r3);
-                    mma_bf16(sc[0], qa[j][0], qa[j][1], qa[j][2], qa[j][3], r0, r1);
-                    mma_bf16(sc[1], qa[j][0], qa[j][1], qa[j][2], qa[j][3], r2, r3);
-                }
-            }
-
-            // ---- online softmax (log2 domain) ---------------------------
-            float p[2][4];
-#pragma unroll
-            for (int nb = 0; nb < 2; ++nb) {
-                p[nb][0] = sc[nb][0] * qk0;
-                p[nb][1] = sc[nb][1] * qk0;
-                p[nb][2] = sc[nb][2] * qk1;
-                p[nb][3] = sc[nb][3] * qk1;
-            }
-            if (tail) {
-#pragma unroll
-                for (int nb = 0; nb < 2; ++nb) {
-#pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        const int tok = kFp8 ? (rb + 8 * nb + tau(2 * c + i)) : (rb + 8 * nb + 2 * c + i);
-                        if (tok >= n_valid) p[nb][i] = p[nb][i + 2] = kNegInf;
-                    }
-                }
-            }
-            float mx0 = fmaxf(fmaxf(p[0][0], p[0][1]), fmaxf(p[1][0], p[1][1]));
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-            float mx1 = kNegInf;
-            if constexpr (kGP == 16) {
-                mx1 = fmaxf(fmaxf(p[0][2], p[0][3]), fmaxf(p[1][2], p[1][3]));
-                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-            }
-            const bool need = (mx0 > m0 + kRescaleThreshold) || (mx1 > m1 + kRescaleThreshold);
-            if (__any_sync(0xffffffffu, need)) {
-                const float n0 = fmaxf(m0, mx0);
-                const float a0 = (n0 == kNegInf) ? 1.f : exp2f(m0 - n0);
-                m0 = n0;
-                l0 *= a0;
-                float a1 = 1.f;
-                if constexpr (kGP == 16) {
-                    const float n1 = fmaxf(m1, mx1);
-                    a1 = (n1 == kNegInf) ? 1.f : exp2f(m1 - n1);
-                    m1 = n1;
-                    l1 *= a1;
+                const int t0 = rb + 2 * c;    // tokens of a0/a1: t0, t0+1; of a2/a3: t0+8, t0+9
+                uint32_t keep01 = 0xFFFFFFFFu, keep23 = 0xFFFFFFFFu;
+                if (tail) {
+                    keep01 = (t0 < n_valid ? 0x0000FFFFu : 0u) | (t0 + 1 < n_valid ? 0xFFFF0000u : 0u);
+                    keep23 = (t0 + 8 < n_valid ? 0x0000FFFFu : 0u) | (t0 + 9 < n_valid ? 0xFFFF0000u : 0u);
                 }
 #pragma unroll
-                for (int nb = 0; nb < kNB; ++nb) {
-                    o[nb][0] *= a0;
-                    o[nb][1] *= a0;
-                    if constexpr (kGP == 16) {
-                        o[nb][2] *= a1;
-                        o[nb][3] *= a1;
-                    }
-                }
-            }
-            const float ref0 = (m0 == kNegInf) ? 0.f : m0;
-            const float ref1 = (m1 == kNegInf) ? 0.f : m1;
-#pragma unroll
-            for (int nb = 0; nb < 2; ++nb) {
-                p[nb][0] = exp2f(p[nb][0] - ref0);
-                p[nb][1] = exp2f(p[nb][1] - ref0);
-                l0 += p[nb][0] + p[nb][1];
-                if constexpr (kGP == 16) {
-                    p[nb][2] = exp2f(p[nb][2] - ref1);
-                    p[nb][3] = exp2f(p[nb][3] - ref1);
-                    l1 += p[nb][2] + p[nb][3];
-                }
-            }
-
-            // ---- O += P V ------------------------------------------------
-            if constexpr (kFp8) {
-                const uint32_t pa0 = pack_f16x2(p[0][0], p[0][1]);
-                const uint32_t pa2 = pack_f16x2(p[1][0], p[1][1]);
-                const uint32_t pa1 = (kGP == 16) ? pack_f16x2(p[0][2], p[0][3]) : 0u;
-                const uint32_t pa3 = (kGP == 16) ? pack_f16x2(p[1][2], p[1][3]) : 0u;
-                const int r0 = rb + tau(2 * c), r1 = rb + tau(2 * c + 1);
-                const int r2 = r0 + 8, r3 = r1 + 8;
-#pragma unroll
-                for (int blk = 0; blk < kD / 32; ++blk) {
-                    const int off = 32 * blk + 4 * g;
-                    uint32_t x0 = lds32(vb + swz<C::kRowBytes, C::kSwizzle>(r0, off));
-                    uint32_t x1 = lds32(vb + swz<C::kRowBytes, C::kSwizzle>(r1, off));
-                    uint32_t x2 = lds32(vb + swz<C::kRowBytes, C::kSwizzle>(r2, off));
-                    uint32_t x3 = lds32(vb + swz<C::kRowBytes, C::kSwizzle>(r3, off));
-                    if (tail) {
-                        x0 = r0 < n_valid ? x0 : 0u;
-                        x1 = r1 < n_valid ? x1 : 0u;
-                        x2 = r2 < n_valid ? x2 : 0u;
-                        x3 = r3 < n_valid ? x3 : 0u;
-                    }
-                    const uint32_t lo01 = prmt(x0, x1, 0x5140u), hi01 = prmt(x0, x1, 0x7362u);
-                    const uint32_t lo23 = prmt(x2, x3, 0x5140u), hi23 = prmt(x2, x3, 0x7362u);
-                    mma_f16(o[4 * blk + 0], pa0, pa1, pa2, pa3, e4m3x2_to_f16x2(lo01 & 0xFFFFu),
-                            e4m3x2_to_f16x2(lo23 & 0xFFFFu));
-                    mma_f16(o[4 * blk + 1], pa0, pa1, pa2, pa3, e4m3x2_to_f16x2(lo01 >> 16),
-                            e4m3x2_to_f16x2(lo23 >> 16));
-                    mma_f16(o[4 * blk + 2], pa0, pa1, pa2, pa3, e4m3x2_to_f16x2(hi01 & 0xFFFFu),
-                            e4m3x2_to_f16x2(hi23 & 0xFFFFu));
-                    mma_f16(o[4 * blk + 3], pa0, pa1, pa2, pa3, e4m3x2_to_f16x2(hi01 >> 16),
-                            e4m3x2_to_f16x2(hi23 >> 16));
-                }
-            } else {
-                const uint32_t pa0 = pack_bf16x2(p[0][0], p[0][1]);
-                const uint32_t pa2 = pack_bf16x2(p[1][0], p[1][1]);
-                const uint32_t pa1 = (kGP == 16) ? pack_bf16x2(p[0][2], p[0][3]) : 0u;
-                const uint32_t pa3 = (kGP == 16) ? pack_bf16x2(p[1][2], p[1][3]) : 0u;
-                const int q8 = lane >> 3;
-                const int row = rb + 8 * (q8 & 1) + (lane & 7);
-                // rows of this thread's B fragments, for masking the tail
-                const int t0 = rb + 2 * c, t1 = t0 + 1, t2 = t0 + 8, t3 = t0 + 9;
-#pragma unroll
-                for (int m = 0; m < kD / 16; ++m) {
-                    const int chunk16 = 2 * m + (q8 >> 1);
+                for (int mb = 0; mb < kMB; ++mb) {
+                    const int chunk16 = 2 * mb + (q8 & 1);
                     const uint32_t addr = vb + (chunk16 >> 3) * C::kSubTileBytes +
                                           swz<128, 128>(row, (chunk16 & 7) * 16);
-                    uint32_t v0, v1, v2, v3;
-                    ldsm_x4_trans(addr, v0, v1, v2, v3);
+                    uint32_t a0, a1, a2, a3;
+                    ldsm_x4_trans(addr, a0, a1, a2, a3);
                     if (tail) {
-                        const uint32_t m01 = (t0 < n_valid ? 0x0000FFFFu : 0u) | (t1 < n_valid ? 0xFFFF0000u : 0u);
-                        const uint32_t m23 = (t2 < n_valid ? 0x0000FFFFu : 0u) | (t3 < n_valid ? 0xFFFF0000u : 0u);
-                        v0 &= m01; v2 &= m01;
-                        v1 &= m23; v3 &= m23;
+                        a0 &= keep01; a1 &= keep01; a2 &= keep23; a3 &= keep23;
                     }
-                    mma_bf16(o[2 * m + 0], pa0, pa1, pa2, pa3, v0, v1);
-                    mma_bf16(o[2 * m + 1], pa0, pa1, pa2, pa3, v2, v3);
+#pragma unroll
+                    for (int nb = 0; nb < kNB; ++nb)
+                        mma_bf16(o[nb][mb], a0, a1, a2, a3, pb[nb][0], pb[nb][1]);
                 }
             }
             __syncwarp();
@@ -615,40 +656,45 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
 
         // ---- epilogue: combine the four warps, then write ---------------
-        l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-        l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-        if constexpr (kGP == 16) {
-            l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-            l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-        }
-        if (c == 0) {
-            red_m[warp * kGP + g] = m0;
-            red_l[warp * kGP + g] = l0;
-            if constexpr (kGP == 16) {
-                red_m[warp * kGP + g + 8] = m1;
-                red_l[warp * kGP + g + 8] = l1;
+#pragma unroll
+        for (int nb = 0; nb < kNB; ++nb)
+#pragma unroll
+            for (int col = 0; col < 2; ++col) {
+                float v = l[nb][col];
+                v += __shfl_xor_sync(0xffffffffu, v, 4);
+                v += __shfl_xor_sync(0xffffffffu, v, 8);
+                v += __shfl_xor_sync(0xffffffffu, v, 16);
+                l[nb][col] = v;
             }
+        if (g == 0) {
+#pragma unroll
+            for (int nb = 0; nb < kNB; ++nb)
+#pragma unroll
+                for (int col = 0; col < 2; ++col) {
+                    red_m[warp * kGP + 8 * nb + 2 * c + col] = m[nb][col];
+                    red_l[warp * kGP + 8 * nb + 2 * c + col] = l[nb][col];
+                }
         }
 #pragma unroll
-        for (int nb = 0; nb < kNB; ++nb) {
-            int d0, d1;
-            if constexpr (kFp8) {
-                // n-block 4*blk + i, column n  <->  dim 32*blk + 4*n + i
-                const int blk = nb >> 2, i = nb & 3;
-                d0 = 32 * blk + 8 * c + i;
-                d1 = d0 + 4;
-            } else {
-                d0 = 8 * nb + 2 * c;
-                d1 = d0 + 1;
+        for (int nb = 0; nb < kNB; ++nb)
+#pragma unroll
+            for (int mb = 0; mb < kMB; ++mb) {
+                // rows of the O^T accumulator: dims d_lo (i = 0, 1) and d_hi (i = 2, 3)
+                int d_lo, d_hi;
+                if constexpr (kFp8) {
+                    d_lo = (kD == 128 ? 16 : 8) * g + 2 * mb;
+                    d_hi = d_lo + 1;
+                } else {
+                    d_lo = 16 * mb + g;
+                    d_hi = d_lo + 8;
+                }
+                float* dst0 = red_o + (warp * kGP + 8 * nb + 2 * c) * kD;
+                float* dst1 = dst0 + kD;
+                dst0[d_lo] = o[nb][mb][0];
+                dst1[d_lo] = o[nb][mb][1];
+                dst0[d_hi] = o[nb][mb][2];
+                dst1[d_hi] = o[nb][mb][3];
             }
-            float* dst = red_o + (warp * kGP + g) * kD;
-            dst[d0] = o[nb][0];
-            dst[d1] = o[nb][1];
-            if constexpr (kGP == 16) {
-                dst[8 * kD + d0] = o[nb][2];
-                dst[8 * kD + d1] = o[nb][3];
-            }
-        }
         named_barrier_sync(1, kConsumerThreads);
         for (int e = tid; e < G * kD; e += kConsumerThreads) {
             const int hq = e / kD, d = e % kD;

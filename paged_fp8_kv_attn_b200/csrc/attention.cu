@@ -61,10 +61,19 @@ struct AttnCfg {
     static constexpr int kSubTileBytes = kChunkTokens * kBoxBytes;
     static constexpr int kTileBytes = kChunkTokens * kRowBytes;  // one of K or V per stage
     static constexpr int kStageBytes = 2 * kTileBytes;
-    static constexpr int kStages =
-        kFp8 ? (kD == 128 ? 5 : 8) : (kD == 128 ? (kGP == 8 ? 3 : 2) : 5);
+    // Pipeline depth and resident CTAs per SM, chosen by measurement on B200:
+    // resident warps matter more than depth (each CTA keeps up to kStages
+    // chunks in flight), so the depth is the largest that still lets
+    // kMinBlocks CTAs share an SM's 228 KB of shared memory.
+    static constexpr int kStages = kFp8 ? (kD == 128 ? 4 : 6) : (kD == 128 ? 2 : 4);
+    static constexpr int kMinBlocks = (kFp8 && kGP == 8) ? 3 : 2;
+    // The epilogue's cross-warp reduction of O (4 warps x kGP heads x kD fp32)
+    // reuses the stage of the segment's last chunk when it fits there (a
+    // group of 8: exactly one FP8 stage), which is released to the producer
+    // only after the epilogue; otherwise it has its own buffer.
+    static constexpr bool kRedInStage = kConsumerWarps * kGP * kD * 4 <= kStageBytes;
     static constexpr int kRedOff = kStages * kStageBytes;
-    static constexpr int kRedFloats = kConsumerWarps * kGP * (kD + 2);
+    static constexpr int kRedFloats = kConsumerWarps * kGP * ((kRedInStage ? 0 : kD) + 2);
     static constexpr int kBarOff = kRedOff + kRedFloats * 4;
     static constexpr int kFlagOff = kBarOff + 2 * kStages * 8;
     static constexpr int kScratchOff = kFlagOff + kStages * 4;
@@ -174,7 +183,7 @@ struct PageWindow {
 // the split-K partial kernel
 // ---------------------------------------------------------------------------
 template <bool kFp8, int kD, int kGP>
-__global__ void __launch_bounds__(kAttnThreads, 2)
+__global__ void __launch_bounds__(kAttnThreads, (AttnCfg<kFp8, kD, kGP>::kMinBlocks))
 attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v, const AttnArgs a) {
     using C = AttnCfg<kFp8, kD, kGP>;
@@ -182,9 +191,9 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    float* red_o = reinterpret_cast<float*>(smem + C::kRedOff);
-    float* red_m = red_o + kConsumerWarps * kGP * kD;
+    float* red_m = reinterpret_cast<float*>(smem + C::kRedOff);
     float* red_l = red_m + kConsumerWarps * kGP;
+    float* const red_o_own = red_l + kConsumerWarps * kGP;   // used when !kRedInStage
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
     uint64_t* empty_bar = full_bar + S;
     volatile int* stage_bad = reinterpret_cast<volatile int*>(smem + C::kFlagOff);
@@ -652,7 +661,14 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty_bar[stage]);
+            if (lane == 0 && !(C::kRedInStage && ch + 1 == s.c1)) mbar_arrive(&empty_bar[stage]);
+        }
+        const int last_stage = (it + S - 1) % S;   // stage of the segment's last chunk
+        float* red_o = C::kRedInStage ? reinterpret_cast<float*>(smem + last_stage * C::kStageBytes)
+                                      : red_o_own;
+        if constexpr (C::kRedInStage) {
+            // every warp has finished reading the last chunk before O overwrites it
+            named_barrier_sync(1, kConsumerThreads);
         }
 
         // ---- epilogue: combine the four warps, then write ---------------
@@ -726,7 +742,11 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 }
             }
         }
+        // the stage is about to be refilled by TMA (async proxy) after our
+        // generic-proxy writes to it: order them first
+        if constexpr (C::kRedInStage) fence_proxy_async_smem();
         named_barrier_sync(1, kConsumerThreads);
+        if (C::kRedInStage && lane == 0) mbar_arrive(&empty_bar[last_stage]);
     }
 }
 

@@ -236,9 +236,22 @@ class Step:
                                             self.seq_lens, wl.sm_scale, self.out, self.lse,
                                             self.ws, abort=ab)
 
+    def check_append(self):
+        wl = self.wl
+        if self.kv == "fp8":
+            self.pkv.kv_check_append_fp8(self.page_tags, self.page_table, self.expected,
+                                         self.seq_lens, wl.page_size, self.k_new, self.v_new,
+                                         wl.k_scale, wl.v_scale, self.k_cache, self.v_cache,
+                                         self.abort)
+        else:
+            self.pkv.kv_check_append_bf16(self.page_tags, self.page_table, self.expected,
+                                          self.seq_lens, wl.page_size, self.k_new, self.v_new,
+                                          self.k_cache, self.v_cache, self.abort)
+
     def full(self):
-        self.check()
-        self.append(True)
+        """The checked step: tag check and append (one fused kernel), then
+        attention with the abort mask."""
+        self.check_append()
         self.attend(True)
 
     def unchecked(self):
@@ -431,7 +444,8 @@ def gpu_arm(args, rank, world):
         "data": "synthetic (seeded; Q~N(0,1), K/V~N(0,1) with 1% x20 outliers, bf16 -> e4m3 at amax/448)",
         "config": {"workload": f"concurrency sweep, batch {HEADLINE_BATCH} x context {CONTEXT}, "
                                "page 64, 64 q heads / 8 kv heads, head_dim 128, FP8 E4M3 KV",
-                   "step": "tag check + FP8 append + paged attention (partial + merge), one layer",
+                   "step": "tag check + FP8 append (one fused kernel) + paged attention "
+                           "(partial + merge), one layer",
                    "global_batch": world * HEADLINE_BATCH, "seq_len": CONTEXT,
                    "kv_dtype": "fp8_e4m3", "parallelism": f"replicas x{world}",
                    "launch": "CUDA graph of the step (programmatic dependent launch)",
@@ -449,7 +463,7 @@ def gpu_arm(args, rank, world):
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "api": "python binding -> C ABI, eager calls, pinned host buffers"},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 3 * args.steps,
         "clocks": clk,
         "sweep": sweep,
     }
@@ -607,9 +621,7 @@ def main():
         wl = workloads.concurrency_sweep(args.batch, device="cuda")
         st = Step(wl, args.kernel_only)
         for _ in range(args.warmup + args.steps):
-            st.check()
-            st.append(True)
-            st.attend(True)
+            st.full()
         torch.cuda.synchronize()
         assert pkv_status_ok(st)
         return

@@ -147,6 +147,35 @@ PKV_API pkv_status kv_append_bf16(const uint16_t* k_new, const uint16_t* v_new,
                           const uint8_t* abort, void* stream);
 
 /*
+ * kv_check_append_fp8 -- kv_tag_check followed by kv_append_fp8 (with the
+ * abort mask just computed), as one kernel with one CTA per request.
+ * [T] "保护共享 KV cache" / [S] "共享 KV 快取的完整性檢查": the check stays a
+ * batched pass of its own, separate from the attention kernel; only the
+ * append, whose write of request b depends on nothing but request b's own
+ * check, rides along.  Outputs are exactly those of the two calls in
+ * sequence: abort_out[b] and num_aborted as kv_tag_check defines them, and
+ * the new token of every request that passed written as kv_append_fp8
+ * defines it.  Arguments: the union of the two calls' arguments, with the
+ * same meaning, layout and alignment rules.
+ */
+PKV_API pkv_status kv_check_append_fp8(const uint32_t* page_tags, int32_t num_pages,
+                               const int32_t* page_table, const uint32_t* expected_tags,
+                               int32_t max_pages, const int32_t* seq_lens, int32_t batch,
+                               int32_t page_size, const uint16_t* k_new, const uint16_t* v_new,
+                               int32_t num_kv_heads, int32_t head_dim, float k_scale,
+                               float v_scale, uint8_t* k_cache, uint8_t* v_cache,
+                               uint8_t* abort_out, int32_t* num_aborted, void* stream);
+
+/* kv_check_append_bf16 -- the same for a BF16 cache (kv_append_bf16). */
+PKV_API pkv_status kv_check_append_bf16(const uint32_t* page_tags, int32_t num_pages,
+                                const int32_t* page_table, const uint32_t* expected_tags,
+                                int32_t max_pages, const int32_t* seq_lens, int32_t batch,
+                                int32_t page_size, const uint16_t* k_new, const uint16_t* v_new,
+                                int32_t num_kv_heads, int32_t head_dim, uint16_t* k_cache,
+                                uint16_t* v_cache, uint8_t* abort_out, int32_t* num_aborted,
+                                void* stream);
+
+/*
  * kv_requant_pages_fp8 -- BF16 -> FP8 page handoff.  [S] "KV 快取量化" and
  * [T] "量化 KV cache": the prefill pool keeps a BF16 cache while the decode
  * pool stores FP8.  Page src_pages[i] of the BF16 pool is re-quantised into

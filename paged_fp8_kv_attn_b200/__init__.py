@@ -57,6 +57,10 @@ def _load():
             "kv_append_fp8": [P, P, P, i32, P, i32, i32, i32, i32, f32, f32, P, P, i32, P, P],
             "kv_append_bf16": [P, P, P, i32, P, i32, i32, i32, i32, P, P, i32, P, P],
             "kv_requant_pages_fp8": [P, i32, P, P, i32, P, i32, i32, i32, i32, f32, P],
+            "kv_check_append_fp8": [P, i32, P, P, i32, P, i32, i32, P, P, i32, i32, f32, f32, P, P,
+                                    P, P, P],
+            "kv_check_append_bf16": [P, i32, P, P, i32, P, i32, i32, P, P, i32, i32, P, P, P, P,
+                                     P],
             "paged_decode_attn_fp8": [P, P, P, f32, f32, P, i32, P, i32, i32, i32, i32, i32, i32,
                                       f32, P, P, P, P, sz, i32, P],
             "paged_decode_attn_bf16": [P, P, P, P, i32, P, i32, i32, i32, i32, i32, i32, f32, P,
@@ -167,6 +171,52 @@ def kv_append_bf16(k_new, v_new, page_table, seq_lens, page_size, k_cache, v_cac
         _ptr(k_new), _ptr(v_new), _ptr(page_table), page_table.shape[1], _ptr(seq_lens), B, Hkv,
         D, page_size, _ptr(k_cache), _ptr(v_cache), k_cache.shape[0], _ptr(abort),
         _stream(stream)))
+
+
+def kv_check_append_fp8(page_tags, page_table, expected_tags, seq_lens, page_size, k_new, v_new,
+                        k_scale, v_scale, k_cache, v_cache, abort_out, num_aborted=None,
+                        stream=None):
+    """kv_tag_check then kv_append_fp8 (with that abort mask) in one kernel."""
+    _need(page_tags, _TAG_DTYPES, 1, "page_tags")
+    _need(page_table, torch.int32, 2, "page_table")
+    _need(expected_tags, _TAG_DTYPES, 2, "expected_tags")
+    _need(seq_lens, torch.int32, 1, "seq_lens")
+    _need(k_new, torch.bfloat16, 3, "k_new")
+    _need(v_new, torch.bfloat16, 3, "v_new")
+    _need(k_cache, torch.uint8, 4, "k_cache")
+    _need(v_cache, torch.uint8, 4, "v_cache")
+    _need(abort_out, torch.uint8, 1, "abort_out")
+    if num_aborted is not None:
+        _need(num_aborted, torch.int32, 1, "num_aborted")
+    B, MP = page_table.shape
+    _, Hkv, D = k_new.shape
+    _check("kv_check_append_fp8", _load().kv_check_append_fp8(
+        _ptr(page_tags), k_cache.shape[0], _ptr(page_table), _ptr(expected_tags), MP,
+        _ptr(seq_lens), B, page_size, _ptr(k_new), _ptr(v_new), Hkv, D, float(k_scale),
+        float(v_scale), _ptr(k_cache), _ptr(v_cache), _ptr(abort_out), _ptr(num_aborted),
+        _stream(stream)))
+
+
+def kv_check_append_bf16(page_tags, page_table, expected_tags, seq_lens, page_size, k_new, v_new,
+                         k_cache, v_cache, abort_out, num_aborted=None, stream=None):
+    """kv_tag_check then kv_append_bf16 (with that abort mask) in one kernel."""
+    _need(page_tags, _TAG_DTYPES, 1, "page_tags")
+    _need(page_table, torch.int32, 2, "page_table")
+    _need(expected_tags, _TAG_DTYPES, 2, "expected_tags")
+    _need(seq_lens, torch.int32, 1, "seq_lens")
+    _need(k_new, torch.bfloat16, 3, "k_new")
+    _need(v_new, torch.bfloat16, 3, "v_new")
+    _need(k_cache, torch.bfloat16, 4, "k_cache")
+    _need(v_cache, torch.bfloat16, 4, "v_cache")
+    _need(abort_out, torch.uint8, 1, "abort_out")
+    if num_aborted is not None:
+        _need(num_aborted, torch.int32, 1, "num_aborted")
+    B, MP = page_table.shape
+    _, Hkv, D = k_new.shape
+    _check("kv_check_append_bf16", _load().kv_check_append_bf16(
+        _ptr(page_tags), k_cache.shape[0], _ptr(page_table), _ptr(expected_tags), MP,
+        _ptr(seq_lens), B, page_size, _ptr(k_new), _ptr(v_new), Hkv, D, _ptr(k_cache),
+        _ptr(v_cache), _ptr(abort_out), _ptr(num_aborted), _stream(stream)))
 
 
 def kv_requant_pages_fp8(src_pool, src_pages, dst_pool, dst_pages, scale, stream=None):

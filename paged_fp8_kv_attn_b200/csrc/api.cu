@@ -322,6 +322,62 @@ pkv_status kv_append_bf16(const uint16_t* k_new, const uint16_t* v_new,
                        head_dim, page_size, 1.f, 1.f, k_cache, v_cache, num_pages, abort, stream);
 }
 
+static pkv_status check_append_impl(bool fp8, const uint32_t* page_tags, int32_t num_pages,
+                                    const int32_t* page_table, const uint32_t* expected_tags,
+                                    int32_t max_pages, const int32_t* seq_lens, int32_t batch,
+                                    int32_t page_size, const uint16_t* k_new,
+                                    const uint16_t* v_new, int32_t num_kv_heads,
+                                    int32_t head_dim, float k_scale, float v_scale, void* k_cache,
+                                    void* v_cache, uint8_t* abort_out, int32_t* num_aborted,
+                                    void* stream) {
+    pkv_status st = check_common_kv(batch, num_kv_heads, head_dim, page_size, num_pages, max_pages);
+    if (st != PKV_OK) return st;
+    if (fp8 && (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) ||
+                !std::isfinite(v_scale)))
+        return fail(PKV_ERR_INVALID_ARG, "k_scale and v_scale must be finite and > 0");
+    if (num_aborted) {
+        cudaError_t e = cudaMemsetAsync(num_aborted, 0, sizeof(int32_t), as_stream(stream));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(num_aborted)");
+    }
+    if (batch == 0) return PKV_OK;
+    if (!page_tags || !page_table || !expected_tags || !seq_lens || !k_new || !v_new ||
+        !k_cache || !v_cache || !abort_out)
+        return fail(PKV_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) ||
+        !aligned(v_cache, 16))
+        return fail(PKV_ERR_INVALID_ARG, "k_new, v_new and the caches must be 16-byte aligned");
+    cudaError_t e = pkv::launch_check_append(fp8, page_tags, num_pages, page_table, expected_tags,
+                                             max_pages, seq_lens, batch, page_size, k_new, v_new,
+                                             num_kv_heads, head_dim, k_scale, v_scale, k_cache,
+                                             v_cache, abort_out, num_aborted, as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "check+append launch");
+    return PKV_OK;
+}
+
+pkv_status kv_check_append_fp8(const uint32_t* page_tags, int32_t num_pages,
+                               const int32_t* page_table, const uint32_t* expected_tags,
+                               int32_t max_pages, const int32_t* seq_lens, int32_t batch,
+                               int32_t page_size, const uint16_t* k_new, const uint16_t* v_new,
+                               int32_t num_kv_heads, int32_t head_dim, float k_scale,
+                               float v_scale, uint8_t* k_cache, uint8_t* v_cache,
+                               uint8_t* abort_out, int32_t* num_aborted, void* stream) {
+    return check_append_impl(true, page_tags, num_pages, page_table, expected_tags, max_pages,
+                             seq_lens, batch, page_size, k_new, v_new, num_kv_heads, head_dim,
+                             k_scale, v_scale, k_cache, v_cache, abort_out, num_aborted, stream);
+}
+
+pkv_status kv_check_append_bf16(const uint32_t* page_tags, int32_t num_pages,
+                                const int32_t* page_table, const uint32_t* expected_tags,
+                                int32_t max_pages, const int32_t* seq_lens, int32_t batch,
+                                int32_t page_size, const uint16_t* k_new, const uint16_t* v_new,
+                                int32_t num_kv_heads, int32_t head_dim, uint16_t* k_cache,
+                                uint16_t* v_cache, uint8_t* abort_out, int32_t* num_aborted,
+                                void* stream) {
+    return check_append_impl(false, page_tags, num_pages, page_table, expected_tags, max_pages,
+                             seq_lens, batch, page_size, k_new, v_new, num_kv_heads, head_dim,
+                             1.f, 1.f, k_cache, v_cache, abort_out, num_aborted, stream);
+}
+
 pkv_status kv_requant_pages_fp8(const uint16_t* src_pool, int32_t src_num_pages,
                                 const int32_t* src_pages, uint8_t* dst_pool,
                                 int32_t dst_num_pages, const int32_t* dst_pages,

@@ -71,6 +71,14 @@ cudaError_t launch_append(bool fp8, const uint16_t* k_new, const uint16_t* v_new
                           void* v_cache, int32_t num_pages, const uint8_t* abort,
                           cudaStream_t stream);
 
+cudaError_t launch_check_append(bool fp8, const uint32_t* page_tags, int32_t num_pages,
+                                const int32_t* page_table, const uint32_t* expected_tags,
+                                int32_t max_pages, const int32_t* seq_lens, int32_t batch,
+                                int32_t page_size, const uint16_t* k_new, const uint16_t* v_new,
+                                int32_t num_kv_heads, int32_t head_dim, float k_scale,
+                                float v_scale, void* k_cache, void* v_cache, uint8_t* abort_out,
+                                int32_t* num_aborted, cudaStream_t stream);
+
 cudaError_t launch_requant(const uint16_t* src_pool, int32_t src_num_pages,
                            const int32_t* src_pages, uint8_t* dst_pool, int32_t dst_num_pages,
                            const int32_t* dst_pages, int32_t num_pairs, int64_t page_elems,

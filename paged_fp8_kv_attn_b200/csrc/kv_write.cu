@@ -151,6 +151,114 @@ cudaError_t launch_append(bool fp8, const uint16_t* k_new, const uint16_t* v_new
 }
 
 // ---------------------------------------------------------------------------
+// fused check + append: one CTA per request.  The request's tag check and its
+// append depend on nothing but the request itself, so one CTA checks the used
+// entries while the new token's K/V are already being loaded, and writes the
+// token only if the request passed.  Results are those of kv_tag_check
+// followed by kv_append_* with its abort mask.
+// ---------------------------------------------------------------------------
+constexpr int kFusedThreads = 256;
+
+template <bool kFp8>
+__global__ void __launch_bounds__(kFusedThreads)
+check_append_kernel(const uint32_t* __restrict__ page_tags, int32_t num_pages,
+                    const int32_t* __restrict__ page_table,
+                    const uint32_t* __restrict__ expected_tags, int32_t max_pages,
+                    const int32_t* __restrict__ seq_lens, int32_t page_size,
+                    const uint16_t* __restrict__ k_new, const uint16_t* __restrict__ v_new,
+                    int32_t num_kv_heads, int32_t head_dim, float k_scale, float v_scale,
+                    void* __restrict__ k_cache, void* __restrict__ v_cache,
+                    uint8_t* __restrict__ abort_out, int32_t* __restrict__ num_aborted) {
+    launch_dependents();
+    grid_dependency_wait();
+    const int b = blockIdx.x;
+    const int32_t L = seq_lens[b];
+    int bad = (L < 1 || static_cast<int64_t>(L) > static_cast<int64_t>(max_pages) * page_size);
+    const int per_tensor = num_kv_heads * (head_dim / 8);
+    // the new token's values for this thread's first two 8-element groups,
+    // loaded before the check finishes (they are inputs, not cache contents)
+    uint4 raw[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+    int32_t pid = -1, slot = 0;
+    if (!bad) {
+        const int32_t pos = L - 1;
+        slot = pos % page_size;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int e = threadIdx.x + k * kFusedThreads;
+            if (e < 2 * per_tensor) {
+                const bool is_v = e >= per_tensor;
+                const int r = is_v ? e - per_tensor : e;
+                const int h = r / (head_dim / 8), d8 = r % (head_dim / 8);
+                raw[k] = *reinterpret_cast<const uint4*>(
+                    (is_v ? v_new : k_new) + (static_cast<int64_t>(b) * num_kv_heads + h) * head_dim +
+                    d8 * 8);
+            }
+        }
+        const int32_t used = (L + page_size - 1) / page_size;
+        const int32_t* row = page_table + static_cast<int64_t>(b) * max_pages;
+        const uint32_t* exp = expected_tags + static_cast<int64_t>(b) * max_pages;
+        pid = row[pos / page_size];
+        for (int j = threadIdx.x; j < used; j += kFusedThreads) {
+            const int32_t p = row[j];
+            const uint32_t want = exp[j];
+            if (p < 0 || p >= num_pages)
+                bad = 1;
+            else if (__ldg(page_tags + p) != want)
+                bad = 1;
+        }
+    }
+    bad = __syncthreads_or(bad);
+    if (threadIdx.x == 0) {
+        abort_out[b] = static_cast<uint8_t>(bad != 0);
+        if (bad && num_aborted) atomicAdd(num_aborted, 1);
+    }
+    if (bad) return;   // an aborted request writes nothing (its last page id was checked too)
+    int k = 0;
+    for (int e = threadIdx.x; e < 2 * per_tensor; e += kFusedThreads, ++k) {
+        const bool is_v = e >= per_tensor;
+        const int r = is_v ? e - per_tensor : e;
+        const int h = r / (head_dim / 8), d8 = r % (head_dim / 8);
+        uint4 val;
+        if (k == 0)
+            val = raw[0];
+        else if (k == 1)
+            val = raw[1];
+        else
+            val = *reinterpret_cast<const uint4*>(
+                (is_v ? v_new : k_new) + (static_cast<int64_t>(b) * num_kv_heads + h) * head_dim +
+                d8 * 8);
+        const int64_t dst =
+            ((static_cast<int64_t>(pid) * num_kv_heads + h) * page_size + slot) * head_dim + d8 * 8;
+        if constexpr (kFp8) {
+            uint8_t* cache = static_cast<uint8_t*>(is_v ? v_cache : k_cache);
+            *reinterpret_cast<uint2*>(cache + dst) = quantize8(val, is_v ? v_scale : k_scale);
+        } else {
+            uint16_t* cache = static_cast<uint16_t*>(is_v ? v_cache : k_cache);
+            *reinterpret_cast<uint4*>(cache + dst) = val;
+        }
+    }
+}
+
+cudaError_t launch_check_append(bool fp8, const uint32_t* page_tags, int32_t num_pages,
+                                const int32_t* page_table, const uint32_t* expected_tags,
+                                int32_t max_pages, const int32_t* seq_lens, int32_t batch,
+                                int32_t page_size, const uint16_t* k_new, const uint16_t* v_new,
+                                int32_t num_kv_heads, int32_t head_dim, float k_scale,
+                                float v_scale, void* k_cache, void* v_cache, uint8_t* abort_out,
+                                int32_t* num_aborted, cudaStream_t stream) {
+    PdlLaunch l(dim3(batch), dim3(kFusedThreads), 0, stream);
+    if (fp8)
+        return cudaLaunchKernelEx(&l.cfg, check_append_kernel<true>, page_tags, num_pages,
+                                  page_table, expected_tags, max_pages, seq_lens, page_size, k_new,
+                                  v_new, num_kv_heads, head_dim, k_scale, v_scale, k_cache, v_cache,
+                                  abort_out, num_aborted);
+    return cudaLaunchKernelEx(&l.cfg, check_append_kernel<false>, page_tags, num_pages, page_table,
+                              expected_tags, max_pages, seq_lens, page_size, k_new, v_new,
+                              num_kv_heads, head_dim, k_scale, v_scale, k_cache, v_cache,
+                              abort_out, num_aborted);
+}
+
+// ---------------------------------------------------------------------------
 // BF16 -> FP8 page handoff: grid-stride over 16-element groups
 // ---------------------------------------------------------------------------
 constexpr int kRequantThreads = 256;

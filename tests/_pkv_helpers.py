@@ -94,11 +94,28 @@ class DeviceBatch:
                                        self.seq_lens, wl.sm_scale, self.out, self.lse, ws,
                                        abort=ab, num_ctas=num_ctas)
 
-    def step(self, check=True, append=True, num_ctas=0):
-        if check:
-            self.tag_check()
-        if append:
-            self.append(use_abort=check)
+    def check_append(self):
+        wl = self.wl
+        if self.kv_dtype == "fp8":
+            pkv.kv_check_append_fp8(self.page_tags, self.page_table, self.expected, self.seq_lens,
+                                    wl.page_size, self.k_new, self.v_new, wl.k_scale, wl.v_scale,
+                                    self.k_cache, self.v_cache, self.abort, self.num_aborted)
+        else:
+            pkv.kv_check_append_bf16(self.page_tags, self.page_table, self.expected,
+                                     self.seq_lens, wl.page_size, self.k_new, self.v_new,
+                                     self.k_cache, self.v_cache, self.abort, self.num_aborted)
+
+    def step(self, check=True, append=True, num_ctas=0, fused=True):
+        """One decode step.  With check and append, fused=True uses the fused
+        check+append call (the benchmark's configuration); fused=False the two
+        separate calls."""
+        if check and append and fused:
+            self.check_append()
+        else:
+            if check:
+                self.tag_check()
+            if append:
+                self.append(use_abort=check)
         self.attend(use_abort=check, num_ctas=num_ctas)
         torch.cuda.synchronize()
 

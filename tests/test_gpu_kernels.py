@@ -170,6 +170,50 @@ def test_append_special_values_bit_exact(cuda_device):
     assert np.array_equal(db.v_cache.cpu().numpy(), want_v)
 
 
+@pytest.mark.parametrize("kv", ["fp8", "bf16"])
+@pytest.mark.parametrize("seed", range(4))
+def test_check_append_fused_bit_exact(cuda_device, kv, seed):
+    """The fused call equals the oracle's tag check followed by its append with
+    that mask: abort bytes, count and every cache byte."""
+    rng = np.random.Generator(np.random.PCG64(900 + seed))
+    P = int(rng.choice([16, 64]))
+    lens = rng.integers(1, 9 * P, 45).astype(np.int32)
+    wl = workloads.custom(lens, page_size=P, num_q_heads=16, num_kv_heads=int(rng.choice([1, 8])),
+                          head_dim=int(rng.choice([64, 128])), seed=77 + seed, spare_pages=5)
+    table, expected, lens2 = wl.page_table.copy(), wl.expected_tags.copy(), wl.seq_lens.copy()
+    expected[3, 0] += np.uint32(1)                       # stale first page
+    expected[7, wl.used_pages(7) - 1] += np.uint32(1)    # stale page holding the new token
+    table[11, 0] = wl.num_pages + 3                      # page id out of range
+    lens2[13] = 0                                        # invalid length
+    wl.page_table, wl.expected_tags, wl.seq_lens = table, expected, lens2
+    db = DeviceBatch(wl, kv_dtype=kv)
+    before_k = (db.k_cache.cpu().numpy() if kv == "fp8" else bf16_bits(db.k_cache)).copy()
+    before_v = (db.v_cache.cpu().numpy() if kv == "fp8" else bf16_bits(db.v_cache)).copy()
+    if kv == "fp8":
+        pkv.kv_check_append_fp8(db.page_tags, db.page_table, db.expected, db.seq_lens, P,
+                                db.k_new, db.v_new, wl.k_scale, wl.v_scale, db.k_cache,
+                                db.v_cache, db.abort, db.num_aborted)
+    else:
+        pkv.kv_check_append_bf16(db.page_tags, db.page_table, db.expected, db.seq_lens, P,
+                                 db.k_new, db.v_new, db.k_cache, db.v_cache, db.abort,
+                                 db.num_aborted)
+    torch.cuda.synchronize()
+    want_abort, n_want = oracle.kv_tag_check(wl.page_tags, table, expected, lens2, P)
+    assert want_abort[[3, 7, 11, 13]].all()
+    assert np.array_equal(db.abort.cpu().numpy(), want_abort)
+    assert int(db.num_aborted.item()) == n_want
+    if kv == "fp8":
+        oracle.kv_append_fp8(bf16_bits(wl.k_new), bf16_bits(wl.v_new), table, lens2, P,
+                             wl.k_scale, wl.v_scale, before_k, before_v, want_abort)
+        got_k, got_v = db.k_cache.cpu().numpy(), db.v_cache.cpu().numpy()
+    else:
+        oracle.kv_append_bf16(bf16_bits(wl.k_new), bf16_bits(wl.v_new), table, lens2, P,
+                              before_k, before_v, want_abort)
+        got_k, got_v = bf16_bits(db.k_cache), bf16_bits(db.v_cache)
+    assert np.array_equal(got_k, before_k)
+    assert np.array_equal(got_v, before_v)
+
+
 # --------------------------------------------------------------------------
 # attention: small cases, every item compared
 # --------------------------------------------------------------------------
@@ -198,7 +242,7 @@ def test_attention_small_all_items(cuda_device, case, kv):
     ref_o, ref_l, _ = oracle_step(wl, items, kv_dtype=kv, check=True, append=True)
     for ctas in (0, 1, 3, 37):
         db2 = DeviceBatch(wl, kv_dtype=kv)
-        db2.step(check=True, append=True, num_ctas=ctas)
+        db2.step(check=True, append=True, num_ctas=ctas, fused=ctas in (0, 3))
         out, lse = db2.outputs()
         compare(wl, items, out, lse, ref_o, ref_l, label=f"{kv} ctas={ctas}")
         assert pkv.workspace_status(db2.ws) == 0
@@ -207,13 +251,14 @@ def test_attention_small_all_items(cuda_device, case, kv):
 @pytest.mark.parametrize("kv", ["fp8", "bf16"])
 def test_attention_tiny_decode_with_check(cuda_device, kv):
     wl = workloads.tiny_decode()
-    db = DeviceBatch(wl, kv_dtype=kv)
-    db.step(check=True, append=True)
-    out, lse = db.outputs()
     ref_o, ref_l, ref_abort = oracle_step(wl, [0, 1], kv_dtype=kv)
     assert ref_abort.tolist() == [0, 1]
-    assert db.abort.cpu().tolist() == [0, 1]
-    compare(wl, [0, 1], out, lse, ref_o, ref_l, label=kv)
+    for fused in (True, False):
+        db = DeviceBatch(wl, kv_dtype=kv)
+        db.step(check=True, append=True, fused=fused)
+        out, lse = db.outputs()
+        assert db.abort.cpu().tolist() == [0, 1]
+        compare(wl, [0, 1], out, lse, ref_o, ref_l, label=f"{kv} fused={fused}")
     assert np.all(np.isneginf(lse[1])) and not out[1].any()
     # with the check switched off (abort = NULL) both requests are computed
     db = DeviceBatch(wl, kv_dtype=kv)

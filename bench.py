@@ -183,17 +183,24 @@ class Step:
         self.wl = wl
         self.kv = kv
         dev = torch.device("cuda")
-        self.q = wl.q.to(dev).contiguous()
-        self.k_new = wl.k_new.to(dev).contiguous()
-        self.v_new = wl.v_new.to(dev).contiguous()
-        self.page_table = torch.from_numpy(wl.page_table).to(dev)
-        self.seq_lens = torch.from_numpy(wl.seq_lens).to(dev)
-        self.page_tags = torch.from_numpy(wl.page_tags.view(np.int32)).to(dev)
-        self.expected = torch.from_numpy(wl.expected_tags.view(np.int32)).to(dev)
         B, Hq, D = wl.q.shape
-        self.out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=dev)
-        self.lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
-        self.abort = torch.zeros(B, dtype=torch.uint8, device=dev)
+        # The per-step inputs and outputs live in one packed device buffer each,
+        # so that an end-to-end step moves them with one copy in and one out.
+        ins = [("q", wl.q.contiguous()), ("k_new", wl.k_new.contiguous()),
+               ("v_new", wl.v_new.contiguous()),
+               ("seq_lens", torch.from_numpy(wl.seq_lens)),
+               ("page_table", torch.from_numpy(wl.page_table)),
+               ("expected", torch.from_numpy(wl.expected_tags.view(np.int32)))]
+        outs = [("out", torch.empty((B, Hq, D), dtype=torch.bfloat16)),
+                ("lse", torch.empty((B, Hq), dtype=torch.float32)),
+                ("abort", torch.zeros(B, dtype=torch.uint8))]
+        self.dev_in, self.in_views = self._pack(ins, dev)
+        self.dev_out, self.out_views = self._pack(outs, dev)
+        for name, t in {**self.in_views, **self.out_views}.items():
+            setattr(self, name, t)
+        for name, src in ins:
+            getattr(self, name).copy_(src.to(dev))
+        self.page_tags = torch.from_numpy(wl.page_tags.view(np.int32)).to(dev)
         if kv == "fp8":
             self.k_cache = torch.empty(wl.k_pool.shape, dtype=torch.uint8, device=dev)
             self.v_cache = torch.empty(wl.v_pool.shape, dtype=torch.uint8, device=dev)
@@ -207,6 +214,22 @@ class Step:
             code = pkv.PKV_KV_BF16
         self.ws = pkv.alloc_workspace(code, B, Hq, wl.num_kv_heads, D, device=dev)
         torch.cuda.synchronize()
+
+    @staticmethod
+    def _pack(named, dev):
+        """One uint8 device buffer holding every tensor (256-byte aligned
+        slots) and typed views into it."""
+        import torch
+        offs, total = [], 0
+        for _, t in named:
+            offs.append(total)
+            total += (t.numel() * t.element_size() + 255) // 256 * 256
+        buf = torch.zeros(total, dtype=torch.uint8, device=dev)
+        views = {}
+        for (name, t), off in zip(named, offs):
+            n = t.numel() * t.element_size()
+            views[name] = buf[off: off + n].view(t.dtype).view(t.shape)
+        return buf, views
 
     def check(self):
         wl = self.wl
@@ -294,6 +317,28 @@ def time_per_call(fn, steps, warmup, flush=None):
     return statistics.median(ts), sum(ts) / len(ts)
 
 
+def time_pair(fn_a, fn_b, steps, warmup, flush=None):
+    """Median device times (us) of two calls measured alternately (a, b, a, b,
+    ...) so that clock and thermal drift affect both alike."""
+    import torch
+    for _ in range(warmup):
+        fn_a()
+        fn_b()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for i in range(steps):
+        for j, fn in enumerate((fn_a, fn_b)):
+            if flush is not None:
+                flush.add_(1)
+            ev[i][2 * j].record()
+            fn()
+            ev[i][2 * j + 1].record()
+    torch.cuda.synchronize()
+    ta = [e[0].elapsed_time(e[1]) * 1e3 for e in ev]
+    tb = [e[2].elapsed_time(e[3]) * 1e3 for e in ev]
+    return statistics.median(ta), statistics.median(tb)
+
+
 def gpu_arm(args, rank, world):
     import numpy as np
     import torch
@@ -352,33 +397,24 @@ def gpu_arm(args, rank, world):
     traffic = ncu_traffic_per_launch(wl.logical_tokens() * wl.num_kv_heads)
 
     # ---- tag-check overhead: full step vs step without the check ---------
-    t_full, _ = time_per_call(g_full.replay, args.steps, args.warmup)
-    t_unch, _ = time_per_call(g_unchecked.replay, args.steps, args.warmup)
+    t_full, t_unch = time_pair(g_full.replay, g_unchecked.replay, max(args.steps, 100),
+                               args.warmup)
     overhead_pct = 100.0 * (t_full - t_unch) / t_unch
 
     # ---- end to end through the public API with host buffers -------------
     B = HEADLINE_BATCH
-    pin = lambda t: t.detach().cpu().pin_memory()
-    h_in = {"q": pin(st.q), "k_new": pin(st.k_new), "v_new": pin(st.v_new),
-            "seq_lens": pin(st.seq_lens), "page_table": pin(st.page_table),
-            "expected": pin(st.expected)}
-    h_out = {"out": torch.empty_like(st.out, device="cpu").pin_memory(),
-             "lse": torch.empty_like(st.lse, device="cpu").pin_memory(),
-             "abort": torch.empty_like(st.abort, device="cpu").pin_memory()}
-    h2d = sum(t.numel() * t.element_size() for t in h_in.values())
-    d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+    # pinned host staging with the device buffers' packed layout: the step's
+    # inputs (q, new K/V, lengths, page table, expected tags) go in with one
+    # copy; its results (out, lse, abort mask) come back with one copy
+    h_in = st.dev_in.cpu().pin_memory()
+    h_out = torch.empty_like(st.dev_out, device="cpu").pin_memory()
+    h2d = h_in.numel()       # bytes copied in per step (packed, 256-byte aligned slots)
+    d2h = h_out.numel()      # bytes copied out per step
 
     def e2e_step():
-        st.q.copy_(h_in["q"], non_blocking=True)
-        st.k_new.copy_(h_in["k_new"], non_blocking=True)
-        st.v_new.copy_(h_in["v_new"], non_blocking=True)
-        st.seq_lens.copy_(h_in["seq_lens"], non_blocking=True)
-        st.page_table.copy_(h_in["page_table"], non_blocking=True)
-        st.expected.copy_(h_in["expected"], non_blocking=True)
+        st.dev_in.copy_(h_in, non_blocking=True)
         st.full()
-        h_out["out"].copy_(st.out, non_blocking=True)
-        h_out["lse"].copy_(st.lse, non_blocking=True)
-        h_out["abort"].copy_(st.abort, non_blocking=True)
+        h_out.copy_(st.dev_out, non_blocking=True)
 
     for _ in range(args.warmup):
         e2e_step()
@@ -413,8 +449,7 @@ def gpu_arm(args, rank, world):
                 ga = _graph(lambda: sb.attend(True))
                 steps = max(args.steps, 20)
                 fl = flush if small else None
-                t_step, _ = time_per_call(gf.replay, steps, args.warmup, fl)
-                t_u, _ = time_per_call(gu.replay, steps, args.warmup, fl)
+                t_step, t_u = time_pair(gf.replay, gu.replay, max(steps, 60), args.warmup, fl)
                 t_a, _ = time_per_call(ga.replay, steps, args.warmup, fl)
                 row[kv] = {"step_us": round(t_step, 2), "tokens_per_s": round(b / (t_step * 1e-6), 1),
                            "attn_us": round(t_a, 2),
@@ -462,7 +497,8 @@ def gpu_arm(args, rank, world):
                      "launch_us_mean": round(attn_mean, 2)},
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
-                "api": "python binding -> C ABI, eager calls, pinned host buffers"},
+                "api": "python binding -> C ABI, eager calls; one pinned H2D copy of the "
+                       "packed inputs and one D2H copy of the packed results per step"},
         "gpu_launches": 3 * args.steps,
         "clocks": clk,
         "sweep": sweep,

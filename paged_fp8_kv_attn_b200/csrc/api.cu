@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -182,8 +183,19 @@ pkv_status attn_impl(bool fp8, const uint16_t* q, const void* k_cache, const voi
 
     int grid = num_ctas;
     if (grid == 0) {
+        // one wave of resident CTAs, but no more than leaves each CTA about
+        // eight 64-token chunks of the largest batch the page table allows
+        // (small batches gain from fewer, longer segments and a lighter merge)
         st = default_ctas(fp8, head_dim, group, &grid);
         if (st != PKV_OK) return st;
+        const DeviceInfo* info = nullptr;
+        st = device_info(&info);
+        if (st != PKV_OK) return st;
+        const int64_t chunks_per_seq =
+            (static_cast<int64_t>(max_pages) * page_size + pkv::kChunkTokens - 1) / pkv::kChunkTokens;
+        const int64_t max_units = static_cast<int64_t>(batch) * num_kv_heads * chunks_per_seq;
+        const int64_t cap = std::max<int64_t>(info->sms, (max_units + 7) / 8);
+        if (cap < grid) grid = static_cast<int>(cap);
     } else {
         const DeviceInfo* info = nullptr;
         st = device_info(&info);  // sets the shared-memory attribute

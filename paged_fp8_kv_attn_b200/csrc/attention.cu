@@ -156,6 +156,7 @@ __device__ __forceinline__ void record_timeout(const AttnArgs& a, volatile int* 
 // status word reports the failure.
 __device__ __forceinline__ void wait_or_give_up(uint64_t* bar, uint32_t parity, const AttnArgs& a,
                                                 volatile int* cta_failed) {
+    if (mbar_try_wait(bar, parity)) return;   // the common case: already complete
     if (*cta_failed) return;
     if (!mbar_wait(bar, parity)) record_timeout(a, cta_failed);
 }
@@ -197,6 +198,8 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
     uint64_t* empty_bar = full_bar + S;
     volatile int* stage_bad = reinterpret_cast<volatile int*>(smem + C::kFlagOff);
+    // read after the stage's full barrier, whose wait orders it after the write
+    const int* stage_bad_rd = reinterpret_cast<const int*>(smem + C::kFlagOff);
     int* scratch = reinterpret_cast<int*>(smem + C::kScratchOff);
     volatile int* cta_failed = scratch + 10;
 
@@ -482,7 +485,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
         for (int ch = s.c0; ch < s.c1; ++ch, ++it) {
             const int stage = it % S;
             wait_or_give_up(&full_bar[stage], (it / S) & 1, a, cta_failed);
-            poisoned |= stage_bad[stage];
+            poisoned |= stage_bad_rd[stage];
             const int n_valid = min(kChunkTokens, s.L - ch * kChunkTokens);
             const bool tail = n_valid < kChunkTokens;
             const uint32_t kb = smem_addr(smem + stage * C::kStageBytes);
@@ -545,26 +548,26 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     if (t_hi >= n_valid) p[nb][2] = p[nb][3] = kNegInf;
                 }
             }
-            float mx[kNB][2];
+            // Lazy rescaling: the running max m (uniform over the warp, per head)
+            // only moves when some score exceeds it by more than the threshold;
+            // until then p = 2^(s - m) <= 2^8 and no cross-lane max is needed.
             bool need = false;
 #pragma unroll
             for (int nb = 0; nb < kNB; ++nb)
 #pragma unroll
-                for (int col = 0; col < 2; ++col) {
-                    float v = fmaxf(p[nb][col], p[nb][col + 2]);
-                    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-                    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-                    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-                    mx[nb][col] = v;
-                    need |= v > m[nb][col] + kRescaleThreshold;
-                }
+                for (int col = 0; col < 2; ++col)
+                    need |= fmaxf(p[nb][col], p[nb][col + 2]) > m[nb][col] + kRescaleThreshold;
             if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
                 for (int nb = 0; nb < kNB; ++nb) {
                     float alpha[2];
 #pragma unroll
                     for (int col = 0; col < 2; ++col) {
-                        const float nm = fmaxf(m[nb][col], mx[nb][col]);
+                        float v = fmaxf(p[nb][col], p[nb][col + 2]);
+                        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+                        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+                        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+                        const float nm = fmaxf(m[nb][col], v);
                         alpha[col] = (nm == kNegInf) ? 1.f : exp2f(m[nb][col] - nm);
                         m[nb][col] = nm;
                         l[nb][col] *= alpha[col];
@@ -758,7 +761,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
 // segments, merged online), then every thread sums its (head, dim) outputs
 // with independent loads.
 // ---------------------------------------------------------------------------
-constexpr int kMergeThreads = 256;
+constexpr int kMergeThreads = 512;
 constexpr int kMergeTile = 256;
 
 __device__ __forceinline__ int64_t cta_of_unit(int64_t u, int64_t U, int N) {
@@ -853,18 +856,22 @@ attn_merge_kernel(const AttnArgs a) {
             for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
             if ((tid & 31) == 0) s_l[hq] += lsum;
         }
-        // (3) outputs: independent loads over the tile's segments
+        // (3) outputs: segment-major, so each thread keeps kPer x 8 independent
+        // loads in flight
+        const int64_t stride = static_cast<int64_t>(G) * kD;
+        const float* base = a.ws_o + (c0 + t0 + item) * stride;
 #pragma unroll
         for (int k = 0; k < kPer; ++k) {
             const int e = tid + k * kMergeThreads;
-            if (e >= G * kD) break;
-            const int hq = e / kD, d = e % kD;
-            float o = acc[k] * s_scale[hq];
-            const float* src = a.ws_o + ((c0 + t0 + item) * G + hq) * kD + d;
-            const int64_t stride = static_cast<int64_t>(G) * kD;
+            if (e < G * kD) acc[k] *= s_scale[e / kD];
+        }
 #pragma unroll 8
-            for (int s = 0; s < tn; ++s) o += s_w[s][hq] * src[s * stride];
-            acc[k] = o;
+        for (int s = 0; s < tn; ++s) {
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) {
+                const int e = tid + k * kMergeThreads;
+                if (e < G * kD) acc[k] += s_w[s][e / kD] * base[s * stride + e];
+            }
         }
         __syncthreads();
     }

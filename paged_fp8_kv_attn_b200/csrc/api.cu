@@ -46,7 +46,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
     bool ready = false;
     int sms = 0;
-    int occupancy[2][2][2] = {};   // [fp8][d128][gp16]
+    int occupancy[2][2][2][2] = {};   // [fp8][d128][gp16][two KV heads per item]
 };
 std::mutex g_dev_mutex;
 DeviceInfo g_dev[kMaxDevices];
@@ -63,16 +63,18 @@ pkv_status device_info(const DeviceInfo** out) {
         if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
         for (int f = 0; f < 2; ++f)
             for (int d = 0; d < 2; ++d)
-                for (int gp = 0; gp < 2; ++gp) {
-                    const bool fp8 = f == 1;
-                    const int hd = d ? 128 : 64, gpad = gp ? 16 : 8;
-                    e = pkv::attn_set_smem_attr(fp8, hd, gpad);
-                    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-                    int blocks = 0;
-                    e = pkv::attn_occupancy(fp8, hd, gpad, &blocks);
-                    if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
-                    info.occupancy[f][d][gp] = blocks < 1 ? 1 : blocks;
-                }
+                for (int gp = 0; gp < 2; ++gp)
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const bool fp8 = f == 1;
+                        const int hd = d ? 128 : 64, gpad = gp ? 16 : 8, kvh = h2 ? 2 : 1;
+                        if (pkv::attn_partial_smem_bytes(fp8, hd, gpad, kvh) == 0) continue;
+                        e = pkv::attn_set_smem_attr(fp8, hd, gpad, kvh);
+                        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+                        int blocks = 0;
+                        e = pkv::attn_occupancy(fp8, hd, gpad, kvh, &blocks);
+                        if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
+                        info.occupancy[f][d][gp][h2] = blocks < 1 ? 1 : blocks;
+                    }
         info.ready = true;
     }
     *out = &info;
@@ -81,11 +83,11 @@ pkv_status device_info(const DeviceInfo** out) {
 
 int group_pad_of(int group) { return group <= 8 ? 8 : 16; }
 
-pkv_status default_ctas(bool fp8, int head_dim, int group, int* ctas) {
+pkv_status default_ctas(bool fp8, int head_dim, int group, int kv_per_item, int* ctas) {
     const DeviceInfo* info = nullptr;
     pkv_status st = device_info(&info);
     if (st != PKV_OK) return st;
-    *ctas = info->sms * info->occupancy[fp8 ? 1 : 0][head_dim == 128][group > 8];
+    *ctas = info->sms * info->occupancy[fp8 ? 1 : 0][head_dim == 128][group > 8][kv_per_item == 2];
     return PKV_OK;
 }
 
@@ -181,19 +183,21 @@ pkv_status attn_impl(bool fp8, const uint16_t* q, const void* k_cache, const voi
     if (!workspace || !aligned(workspace, 256))
         return fail(PKV_ERR_WORKSPACE, "workspace must be non-null and 256-byte aligned");
 
+    const int kv_per_item = pkv::kv_heads_per_item(fp8, num_kv_heads, group);
     int grid = num_ctas;
     if (grid == 0) {
         // one wave of resident CTAs, but no more than leaves each CTA about
         // eight 64-token chunks of the largest batch the page table allows
         // (small batches gain from fewer, longer segments and a lighter merge)
-        st = default_ctas(fp8, head_dim, group, &grid);
+        st = default_ctas(fp8, head_dim, group, kv_per_item, &grid);
         if (st != PKV_OK) return st;
         const DeviceInfo* info = nullptr;
         st = device_info(&info);
         if (st != PKV_OK) return st;
         const int64_t chunks_per_seq =
             (static_cast<int64_t>(max_pages) * page_size + pkv::kChunkTokens - 1) / pkv::kChunkTokens;
-        const int64_t max_units = static_cast<int64_t>(batch) * num_kv_heads * chunks_per_seq;
+        const int64_t max_units =
+            static_cast<int64_t>(batch) * (num_kv_heads / kv_per_item) * chunks_per_seq;
         const int64_t cap = std::max<int64_t>(info->sms, (max_units + 7) / 8);
         if (cap < grid) grid = static_cast<int>(cap);
     } else {
@@ -202,12 +206,17 @@ pkv_status attn_impl(bool fp8, const uint16_t* q, const void* k_cache, const voi
         if (st != PKV_OK) return st;
     }
     const pkv::WorkspaceLayout wl =
-        pkv::workspace_layout(batch, group, num_kv_heads, head_dim, grid);
+        pkv::workspace_layout(batch, group, num_kv_heads, kv_per_item, head_dim, grid);
     if (workspace_bytes < wl.total)
         return fail(PKV_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes,
                     wl.total);
 
-    const int box_rows = page_size < pkv::kChunkTokens ? page_size : pkv::kChunkTokens;
+    // rows of one TMA box: a 64-token chunk of a page (a whole page when
+    // smaller); with two KV heads per item and 64-token pages, both heads' rows
+    // of the page at once (they are adjacent in the pool)
+    const int box_rows = (kv_per_item == 2 && page_size == pkv::kChunkTokens)
+                             ? 2 * pkv::kChunkTokens
+                             : (page_size < pkv::kChunkTokens ? page_size : pkv::kChunkTokens);
     const int64_t rows = static_cast<int64_t>(num_pages) * num_kv_heads * page_size;
     CUtensorMap tk, tv;
     st = encode_pool_map(&tk, k_cache, fp8, head_dim, rows, box_rows);
@@ -231,6 +240,8 @@ pkv_status attn_impl(bool fp8, const uint16_t* q, const void* k_cache, const voi
     a.max_pages = max_pages;
     a.num_q_heads = num_q_heads;
     a.num_kv_heads = num_kv_heads;
+    a.kv_per_item = kv_per_item;
+    a.items_per_req = num_kv_heads / kv_per_item;
     a.group = group;
     a.page_size = page_size;
     a.num_pages = num_pages;
@@ -239,7 +250,7 @@ pkv_status attn_impl(bool fp8, const uint16_t* q, const void* k_cache, const voi
     a.qk_scale = sm_scale * (fp8 ? k_scale : 1.f) * 1.4426950408889634f;
     a.v_scale = fp8 ? v_scale : 1.f;
 
-    cudaError_t e = pkv::launch_attn_partial(fp8, head_dim, group_pad_of(group), grid,
+    cudaError_t e = pkv::launch_attn_partial(fp8, head_dim, group_pad_of(group), kv_per_item, grid,
                                              as_stream(stream), tk, tv, a);
     if (e != cudaSuccess) return cuda_fail(e, "attention partial launch");
     e = pkv::launch_attn_merge(head_dim, as_stream(stream), a);
@@ -253,13 +264,15 @@ namespace pkv {
 void set_last_error(const char* message) { g_last_error = message; }
 
 WorkspaceLayout workspace_layout(int32_t batch, int32_t group, int32_t num_kv_heads,
-                                 int32_t head_dim, int32_t num_ctas) {
+                                 int32_t kv_per_item, int32_t head_dim, int32_t num_ctas) {
     WorkspaceLayout l{};
     l.prefix_off = 256;
-    const size_t slots = static_cast<size_t>(num_ctas) + static_cast<size_t>(batch) * num_kv_heads;
+    const size_t items = static_cast<size_t>(batch) * (num_kv_heads / kv_per_item);
+    const size_t heads_per_slot = static_cast<size_t>(group) * kv_per_item;
+    const size_t slots = static_cast<size_t>(num_ctas) + items;
     l.ml_off = round_up(l.prefix_off + (static_cast<size_t>(batch) + 1) * 4, 256);
-    l.o_off = round_up(l.ml_off + slots * group * 2 * 4, 256);
-    l.total = round_up(l.o_off + slots * group * head_dim * 4, 256);
+    l.o_off = round_up(l.ml_off + slots * heads_per_slot * 2 * 4, 256);
+    l.total = round_up(l.o_off + slots * heads_per_slot * head_dim * 4, 256);
     return l;
 }
 }  // namespace pkv
@@ -435,9 +448,10 @@ size_t paged_decode_attn_workspace_size(int32_t kv_dtype, int32_t batch, int32_t
         return 0;
     }
     int grid = num_ctas;
-    if (grid == 0 && default_ctas(kv_dtype == PKV_KV_FP8, head_dim, group, &grid) != PKV_OK)
-        return 0;
-    return pkv::workspace_layout(batch, group, num_kv_heads, head_dim, grid).total;
+    const bool fp8 = kv_dtype == PKV_KV_FP8;
+    const int kv_per_item = pkv::kv_heads_per_item(fp8, num_kv_heads, group);
+    if (grid == 0 && default_ctas(fp8, head_dim, group, kv_per_item, &grid) != PKV_OK) return 0;
+    return pkv::workspace_layout(batch, group, num_kv_heads, kv_per_item, head_dim, grid).total;
 }
 
 pkv_status paged_decode_attn_fp8(const uint16_t* q, const uint8_t* k_cache,

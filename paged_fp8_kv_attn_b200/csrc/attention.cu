@@ -51,7 +51,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr float kNegInf = -__builtin_huge_valf();
 
-template <bool kFp8, int kD, int kGP>
+template <bool kFp8, int kD, int kGP, int kH>
 struct AttnCfg {
     static constexpr int kElem = kFp8 ? 1 : 2;
     static constexpr int kRowBytes = kD * kElem;                 // 64, 128 or 256
@@ -59,14 +59,16 @@ struct AttnCfg {
     static constexpr int kSubTiles = kRowBytes / kBoxBytes;      // 2 for BF16 D=128
     static constexpr int kSwizzle = kBoxBytes;                   // 128 or 64
     static constexpr int kSubTileBytes = kChunkTokens * kBoxBytes;
-    static constexpr int kTileBytes = kChunkTokens * kRowBytes;  // one of K or V per stage
+    static constexpr int kHeadTileBytes = kChunkTokens * kRowBytes;  // one KV head of a chunk
+    static constexpr int kTileBytes = kH * kHeadTileBytes;           // K (or V) of a stage
     static constexpr int kStageBytes = 2 * kTileBytes;
     // Pipeline depth and resident CTAs per SM, chosen by measurement on B200:
     // resident warps matter more than depth (each CTA keeps up to kStages
     // chunks in flight), so the depth is the largest that still lets
     // kMinBlocks CTAs share an SM's 228 KB of shared memory.
-    static constexpr int kStages = kFp8 ? (kD == 128 ? 4 : 6) : (kD == 128 ? 2 : 4);
-    static constexpr int kMinBlocks = (kFp8 && kGP == 8) ? 3 : 2;
+    static constexpr int kStages = kFp8 ? (kD == 128 ? (kH == 2 ? 3 : 4) : (kH == 2 ? 3 : 6))
+                                        : (kD == 128 ? 2 : 4);
+    static constexpr int kMinBlocks = (kFp8 && kGP == 8 && kH == 1) ? 3 : 2;
     // The epilogue's cross-warp reduction of O (4 warps x kGP heads x kD fp32)
     // reuses the stage of the segment's last chunk when it fits there (a
     // group of 8: exactly one FP8 stage), which is released to the producer
@@ -80,6 +82,7 @@ struct AttnCfg {
     static constexpr int kSmemBytes = kScratchOff + 16 * 4 + 1024;  // + alignment slack
     static_assert(kD == 64 || kD == 128, "head_dim");
     static_assert(kGP == 8 || kGP == 16, "group pad");
+    static_assert(kH == 1 || (kH == 2 && kGP == 8), "two KV heads per item need a group <= 8");
 };
 
 // Token permutation inside an 8-row group: row tau(n) feeds MMA column n.
@@ -183,11 +186,11 @@ struct PageWindow {
 // ---------------------------------------------------------------------------
 // the split-K partial kernel
 // ---------------------------------------------------------------------------
-template <bool kFp8, int kD, int kGP>
-__global__ void __launch_bounds__(kAttnThreads, (AttnCfg<kFp8, kD, kGP>::kMinBlocks))
+template <bool kFp8, int kD, int kGP, int kH>
+__global__ void __launch_bounds__(kAttnThreads, (AttnCfg<kFp8, kD, kGP, kH>::kMinBlocks))
 attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v, const AttnArgs a) {
-    using C = AttnCfg<kFp8, kD, kGP>;
+    using C = AttnCfg<kFp8, kD, kGP, kH>;
     constexpr int S = C::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -207,7 +210,8 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int warp = tid >> 5;
     const int lane = tid & 31;
     const int B = a.batch;
-    const int Hkv = a.num_kv_heads;
+    const int Hkv = a.num_kv_heads;        // KV heads of the pool
+    const int IPR = a.items_per_req;       // work items per request (Hkv / kH)
     const int64_t max_tokens = static_cast<int64_t>(a.max_pages) * a.page_size;
 
     launch_dependents();
@@ -224,7 +228,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
     Walker walk;
     walk.seq_lens = a.seq_lens;
     walk.max_tokens = max_tokens;
-    walk.num_kv_heads = Hkv;
+    walk.num_kv_heads = IPR;
     walk.batch = B;
     const int per = (B + kAttnThreads - 1) / kAttnThreads;
     const int b_lo = min(B, tid * per);
@@ -246,7 +250,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
         if (w < warp) warp_base += t;
         total += t;
     }
-    const int64_t U = static_cast<int64_t>(Hkv) * total;
+    const int64_t U = static_cast<int64_t>(IPR) * total;
     const int64_t u_lo = static_cast<int64_t>(blockIdx.x) * U / a.num_ctas;
     const int64_t u_hi = static_cast<int64_t>(blockIdx.x + 1) * U / a.num_ctas;
     {
@@ -254,8 +258,8 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
         for (int b = b_lo; b < b_hi; ++b) {
             const int n = walk.chunks_of(a.seq_lens[b]);
             if (blockIdx.x == 0) a.ws_prefix[b] = run;
-            if (n > 0 && u_lo < u_hi && static_cast<int64_t>(Hkv) * run <= u_lo &&
-                u_lo < static_cast<int64_t>(Hkv) * (run + n)) {
+            if (n > 0 && u_lo < u_hi && static_cast<int64_t>(IPR) * run <= u_lo &&
+                u_lo < static_cast<int64_t>(IPR) * (run + n)) {
                 scratch[8] = b;
                 scratch[9] = run;
             }
@@ -269,7 +273,11 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
     const int P = a.page_size;
     const int box_rows = a.box_rows;
-    const int boxes = kChunkTokens / box_rows;
+    // With two KV heads per item and 64-token pages, the item's K (or V) rows
+    // of a page are one contiguous 128-row box; otherwise one box per KV head
+    // and page (per 64 rows for 128-token pages).
+    const bool joint = (kH == 2) && (box_rows == 2 * kChunkTokens);
+    const int boxes = joint ? 1 : kChunkTokens / box_rows;
 
     if (warp == kConsumerWarps) {
         // ================= producer warp =================
@@ -291,10 +299,12 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         if (j >= npages) break;
                         const int32_t pid = win.get(j, npages, lane);
                         if (lane == 0 && pid >= 0 && pid < a.num_pages) {
-                            const int32_t y = (pid * Hkv + s.h) * P + (tok0 % P);
-                            for (int st = 0; st < C::kSubTiles; ++st) {
-                                tma_prefetch_l2_2d(&tmap_k, st * 64, y);
-                                tma_prefetch_l2_2d(&tmap_v, st * 64, y);
+                            for (int kv = 0; kv < (joint ? 1 : kH); ++kv) {
+                                const int32_t y = (pid * Hkv + s.h * kH + kv) * P + (tok0 % P);
+                                for (int st = 0; st < C::kSubTiles; ++st) {
+                                    tma_prefetch_l2_2d(&tmap_k, st * 64, y);
+                                    tma_prefetch_l2_2d(&tmap_v, st * 64, y);
+                                }
                             }
                         }
                     }
@@ -331,7 +341,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
                                 bad = 1;
                                 pids[i] = -1;
                             } else {
-                                bytes += 2u * C::kSubTiles * box_rows * C::kBoxBytes;
+                                bytes += 2u * C::kSubTiles * box_rows * C::kBoxBytes * (joint ? 1 : kH);
                             }
                         }
                     }
@@ -343,11 +353,14 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     for (int i = 0; i < 4; ++i) {
                         if (pids[i] < 0) continue;
                         const int tok0 = ch * kChunkTokens + i * box_rows;
-                        const int32_t y = (pids[i] * Hkv + s.h) * P + (tok0 % P);
-                        for (int st = 0; st < C::kSubTiles; ++st) {
-                            const uint32_t off = st * C::kSubTileBytes + i * box_rows * C::kBoxBytes;
-                            tma_load_2d(kdst + off, &tmap_k, st * 64, y, &full_bar[stage]);
-                            tma_load_2d(vdst + off, &tmap_v, st * 64, y, &full_bar[stage]);
+                        for (int kv = 0; kv < (joint ? 1 : kH); ++kv) {
+                            const int32_t y = (pids[i] * Hkv + s.h * kH + kv) * P + (tok0 % P);
+                            for (int st = 0; st < C::kSubTiles; ++st) {
+                                const uint32_t off = kv * C::kHeadTileBytes + st * C::kSubTileBytes +
+                                                     i * box_rows * C::kBoxBytes;
+                                tma_load_2d(kdst + off, &tmap_k, st * 64, y, &full_bar[stage]);
+                                tma_load_2d(vdst + off, &tmap_v, st * 64, y, &full_bar[stage]);
+                            }
                         }
                     }
                 }
@@ -367,7 +380,13 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int g = lane >> 2;   // MMA group id
     const int c = lane & 3;    // thread in group
     const int G = a.group;
-    const int rb = warp * 16;  // this warp's rows of each chunk
+    const int IQ = kH * G;                 // query heads of one item
+    // Warp -> (KV head of the item, rows of each chunk): with one KV head per
+    // item each warp owns 16 rows; with two, two warps share a head and each
+    // owns 32 rows (two 16-row MMA tiles).
+    constexpr int kWarpsPerHead = kConsumerWarps / kH;
+    const int kvh_w = warp / kWarpsPerHead;
+    const int row0 = (warp % kWarpsPerHead) * 16 * kH;
     constexpr int kNB = kGP / 8;      // n-blocks of query heads
     constexpr int kMB = kD / 16;      // m-blocks of the head dimension (PV)
     constexpr int kKS = kD / 16;      // k-steps of the QK contraction
@@ -380,10 +399,10 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
         for (int half = 0; half < 2; ++half)
 #pragma unroll
             for (int part = 0; part < kD / 64; ++part)
-                k_off[half][part] = swz<C::kRowBytes, C::kSwizzle>(rb + 8 * half + tau(g),
+                k_off[half][part] = swz<C::kRowBytes, C::kSwizzle>(row0 + 8 * half + tau(g),
                                                                    16 * (4 * part + c));
-        const int vr[4] = {rb + tau(2 * c), rb + tau(2 * c + 1), rb + 8 + tau(2 * c),
-                           rb + 8 + tau(2 * c + 1)};
+        const int vr[4] = {row0 + tau(2 * c), row0 + tau(2 * c + 1), row0 + 8 + tau(2 * c),
+                           row0 + 8 + tau(2 * c + 1)};
 #pragma unroll
         for (int i = 0; i < 4; ++i)
             v_off[i] = swz<C::kRowBytes, C::kSwizzle>(vr[i], (kD == 128 ? 16 : 8) * g);
@@ -392,22 +411,23 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
     uint32_t it = 0;
     Segment s;
     while (walk.next(s)) {
-        const int item = s.b * Hkv + s.h;
+        const int item = s.b * IPR + s.h;
         const bool whole = (s.c0 == 0 && s.c1 == s.n);
         const int64_t slot = static_cast<int64_t>(blockIdx.x) + item;
-        const int64_t head0 = static_cast<int64_t>(s.b) * a.num_q_heads + s.h * G;
+        const int64_t head0 = static_cast<int64_t>(s.b) * a.num_q_heads + s.h * IQ;  // item
+        const int64_t head0_w = head0 + kvh_w * G;                                    // this warp
 
         if (a.abort != nullptr && a.abort[s.b] != 0) {
-            for (int e = tid; e < G * kD; e += kConsumerThreads) {
+            for (int e = tid; e < IQ * kD; e += kConsumerThreads) {
                 const int hq = e / kD, d = e % kD;
                 if (whole) {
                     a.out[(head0 + hq) * kD + d] = 0;
                     if (d == 0) a.lse[head0 + hq] = kNegInf;
                 } else {
-                    a.ws_o[(slot * G + hq) * kD + d] = 0.f;
+                    a.ws_o[(slot * IQ + hq) * kD + d] = 0.f;
                     if (d == 0) {
-                        a.ws_ml[(slot * G + hq) * 2 + 0] = kNegInf;
-                        a.ws_ml[(slot * G + hq) * 2 + 1] = -1.f;
+                        a.ws_ml[(slot * IQ + hq) * 2 + 0] = kNegInf;
+                        a.ws_ml[(slot * IQ + hq) * 2 + 1] = -1.f;
                     }
                 }
             }
@@ -421,7 +441,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
         for (int nb = 0; nb < kNB; ++nb) {
             const int hh = g + 8 * nb;
             const bool valid = hh < G;
-            const uint16_t* qrow = a.q + (head0 + (valid ? hh : 0)) * kD;
+            const uint16_t* qrow = a.q + (head0_w + (valid ? hh : 0)) * kD;
             float my_scale;
             if constexpr (kFp8) {
                 // this thread's dims: [16c, 16c+16) and, for D=128, [64+16c, 64+16c+16);
@@ -488,8 +508,15 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
             poisoned |= stage_bad_rd[stage];
             const int n_valid = min(kChunkTokens, s.L - ch * kChunkTokens);
             const bool tail = n_valid < kChunkTokens;
-            const uint32_t kb = smem_addr(smem + stage * C::kStageBytes);
-            const uint32_t vb = kb + C::kTileBytes;
+            const uint32_t kb_head = smem_addr(smem + stage * C::kStageBytes) + kvh_w * C::kHeadTileBytes;
+            const uint32_t vb_head = kb_head + C::kTileBytes;
+#pragma unroll
+            for (int t = 0; t < kH; ++t) {
+            const int rb = row0 + 16 * t;
+            // FP8 offsets are relative to the warp's first tile; 16 rows on, the
+            // swizzle pattern repeats, so the next tile is a plain offset
+            const uint32_t kb = kb_head + (kFp8 ? t * 16 * C::kRowBytes : 0);
+            const uint32_t vb = vb_head + (kFp8 ? t * 16 * C::kRowBytes : 0);
 
             // ---- S[16 tokens][8 heads] = K Q^T, two accumulator chains ------
             float acc[kNB][2][4];
@@ -663,6 +690,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         mma_bf16(o[nb][mb], a0, a1, a2, a3, pb[nb][0], pb[nb][1]);
                 }
             }
+            }   // tiles
             __syncwarp();
             if (lane == 0 && !(C::kRedInStage && ch + 1 == s.c1)) mbar_arrive(&empty_bar[stage]);
         }
@@ -715,18 +743,20 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 dst1[d_hi] = o[nb][mb][3];
             }
         named_barrier_sync(1, kConsumerThreads);
-        for (int e = tid; e < G * kD; e += kConsumerThreads) {
+        for (int e = tid; e < IQ * kD; e += kConsumerThreads) {
             const int hq = e / kD, d = e % kD;
+            const int hl = hq % G;                          // head within its KV head's group
+            const int w0 = (hq / G) * kWarpsPerHead;        // the warps that worked on it
             float M = kNegInf;
 #pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red_m[w * kGP + hq]);
+            for (int w = 0; w < kWarpsPerHead; ++w) M = fmaxf(M, red_m[(w0 + w) * kGP + hl]);
             float Lsum = 0.f, O = 0.f;
 #pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) {
-                const float mw = red_m[w * kGP + hq];
+            for (int w = 0; w < kWarpsPerHead; ++w) {
+                const float mw = red_m[(w0 + w) * kGP + hl];
                 const float wt = (mw == kNegInf) ? 0.f : exp2f(mw - M);
-                Lsum += wt * red_l[w * kGP + hq];
-                O += wt * red_o[(w * kGP + hq) * kD + d];
+                Lsum += wt * red_l[(w0 + w) * kGP + hl];
+                O += wt * red_o[((w0 + w) * kGP + hl) * kD + d];
             }
             if (whole) {
                 if (poisoned) {
@@ -738,10 +768,10 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     if (d == 0) a.lse[head0 + hq] = (M + log2f(Lsum)) * kLn2;
                 }
             } else {
-                a.ws_o[(slot * G + hq) * kD + d] = poisoned ? 0.f : O * a.v_scale;
+                a.ws_o[(slot * IQ + hq) * kD + d] = poisoned ? 0.f : O * a.v_scale;
                 if (d == 0) {
-                    a.ws_ml[(slot * G + hq) * 2 + 0] = poisoned ? kNegInf : M;
-                    a.ws_ml[(slot * G + hq) * 2 + 1] = poisoned ? -1.f : Lsum;
+                    a.ws_ml[(slot * IQ + hq) * 2 + 0] = poisoned ? kNegInf : M;
+                    a.ws_ml[(slot * IQ + hq) * 2 + 1] = poisoned ? -1.f : Lsum;
                 }
             }
         }
@@ -772,19 +802,22 @@ __device__ __forceinline__ int64_t cta_of_unit(int64_t u, int64_t U, int N) {
 template <int kD>
 __global__ void __launch_bounds__(kMergeThreads)
 attn_merge_kernel(const AttnArgs a) {
-    __shared__ float s_w[kMergeTile][16];   // weight of segment s for head h (this tile)
-    __shared__ float s_m[16], s_l[16], s_scale[16];
+    __shared__ float s_w[kMergeTile][16];   // m_s, then weight 2^(m_s - M), of segment s, head h
+    __shared__ float s_l[kMergeTile][16];   // l_s
+    __shared__ float s_m[16], s_sum[16], s_scale[16];
     __shared__ int s_dead;
     launch_dependents();
     grid_dependency_wait();
-    const int Hkv = a.num_kv_heads;
+    const int IPR = a.items_per_req;
     const int item = blockIdx.x;
-    const int b = item / Hkv, h = item % Hkv;
-    const int G = a.group;
+    const int b = item / IPR, h = item % IPR;
+    const int G = a.group * a.kv_per_item;   // query heads of one item
     const int tid = threadIdx.x;
     const int64_t head0 = static_cast<int64_t>(b) * a.num_q_heads + h * G;
     const int32_t pre = a.ws_prefix[b];
-    const int32_t n = a.ws_prefix[b + 1] - pre;
+    const int32_t nxt = a.ws_prefix[b + 1];
+    const int32_t tot = a.ws_prefix[a.batch];
+    const int32_t n = nxt - pre;
     if (n == 0) {
         for (int e = tid; e < G * kD; e += kMergeThreads) {
             const int hq = e / kD, d = e % kD;
@@ -793,72 +826,68 @@ attn_merge_kernel(const AttnArgs a) {
         }
         return;
     }
-    const int64_t U = static_cast<int64_t>(Hkv) * a.ws_prefix[a.batch];
-    const int64_t u0 = static_cast<int64_t>(Hkv) * pre + static_cast<int64_t>(h) * n;
+    const int64_t U = static_cast<int64_t>(IPR) * tot;
+    const int64_t u0 = static_cast<int64_t>(IPR) * pre + static_cast<int64_t>(h) * n;
     const int64_t c0 = cta_of_unit(u0, U, a.num_ctas);
     const int64_t c1 = cta_of_unit(u0 + n - 1, U, a.num_ctas);
     if (c0 == c1) return;   // finished by the partial kernel
     const int nseg = static_cast<int>(c1 - c0 + 1);
     if (tid < 16) {
         s_m[tid] = kNegInf;
-        s_l[tid] = 0.f;
+        s_sum[tid] = 0.f;
     }
     if (tid == 0) s_dead = 0;
-    // every thread owns the same (head, dim) outputs across tiles
     constexpr int kPer = (16 * kD + kMergeThreads - 1) / kMergeThreads;
     float acc[kPer];
 #pragma unroll
     for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
-    __syncthreads();
+    const int64_t stride = static_cast<int64_t>(G) * kD;
 
     for (int t0 = 0; t0 < nseg; t0 += kMergeTile) {
         const int tn = min(kMergeTile, nseg - t0);
-        // (1) per head: tile max, rescale of the running state
+        // (1) the tile's (m, l) pairs into shared memory: one round trip
+        for (int e = tid; e < tn * G; e += kMergeThreads) {
+            const int sg = e / G, hq = e % G;
+            const int64_t slot = c0 + t0 + sg + item;
+            const float2 ml = *reinterpret_cast<const float2*>(a.ws_ml + (slot * G + hq) * 2);
+            s_w[sg][hq] = ml.x;
+            s_l[sg][hq] = ml.y;
+        }
+        __syncthreads();
+        // (2) per head, in shared memory: new running max, weights, sum
         for (int hq = tid >> 5; hq < G; hq += kMergeThreads / 32) {
             float mx = kNegInf;
             int dead = 0;
-            for (int s = (tid & 31); s < tn; s += 32) {
-                const int64_t slot = c0 + t0 + s + item;
-                mx = fmaxf(mx, a.ws_ml[(slot * G + hq) * 2 + 0]);
-                dead |= a.ws_ml[(slot * G + hq) * 2 + 1] < 0.f;
+            for (int sg = (tid & 31); sg < tn; sg += 32) {
+                mx = fmaxf(mx, s_w[sg][hq]);
+                dead |= s_l[sg][hq] < 0.f;
             }
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) {
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
                 dead |= __shfl_xor_sync(0xffffffffu, dead, off);
             }
+            const float m_old = s_m[hq];
+            const float m_new = fmaxf(m_old, mx);
+            float lsum = 0.f;
+            for (int sg = (tid & 31); sg < tn; sg += 32) {
+                const float ms = s_w[sg][hq];
+                const float wt = (ms == kNegInf) ? 0.f : exp2f(ms - m_new);
+                s_w[sg][hq] = wt;
+                lsum += wt * s_l[sg][hq];
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
             if ((tid & 31) == 0) {
-                if (dead) s_dead = 1;
-                const float m_old = s_m[hq];
-                const float m_new = fmaxf(m_old, mx);
                 const float r = (m_old == kNegInf) ? 0.f : exp2f(m_old - m_new);
-                s_scale[hq] = r;          // factor for what was accumulated so far
-                s_l[hq] *= r;
+                if (dead) s_dead = 1;
+                s_scale[hq] = r;
+                s_sum[hq] = s_sum[hq] * r + lsum;
                 s_m[hq] = m_new;
             }
         }
         __syncthreads();
-        // (2) segment weights relative to the running max, and the sum
-        for (int e = tid; e < tn * G; e += kMergeThreads) {
-            const int s = e / G, hq = e % G;
-            const int64_t slot = c0 + t0 + s + item;
-            const float ms = a.ws_ml[(slot * G + hq) * 2 + 0];
-            s_w[s][hq] = (ms == kNegInf) ? 0.f : exp2f(ms - s_m[hq]);
-        }
-        __syncthreads();
-        for (int hq = tid >> 5; hq < G; hq += kMergeThreads / 32) {
-            float lsum = 0.f;
-            for (int s = (tid & 31); s < tn; s += 32) {
-                const int64_t slot = c0 + t0 + s + item;
-                lsum += s_w[s][hq] * a.ws_ml[(slot * G + hq) * 2 + 1];
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
-            if ((tid & 31) == 0) s_l[hq] += lsum;
-        }
-        // (3) outputs: segment-major, so each thread keeps kPer x 8 independent
-        // loads in flight
-        const int64_t stride = static_cast<int64_t>(G) * kD;
+        // (3) outputs: segment-major, kPer x 8 independent loads in flight
         const float* base = a.ws_o + (c0 + t0 + item) * stride;
 #pragma unroll
         for (int k = 0; k < kPer; ++k) {
@@ -866,11 +895,11 @@ attn_merge_kernel(const AttnArgs a) {
             if (e < G * kD) acc[k] *= s_scale[e / kD];
         }
 #pragma unroll 8
-        for (int s = 0; s < tn; ++s) {
+        for (int sg = 0; sg < tn; ++sg) {
 #pragma unroll
             for (int k = 0; k < kPer; ++k) {
                 const int e = tid + k * kMergeThreads;
-                if (e < G * kD) acc[k] += s_w[s][e / kD] * base[s * stride + e];
+                if (e < G * kD) acc[k] += s_w[sg][e / kD] * base[sg * stride + e];
             }
         }
         __syncthreads();
@@ -884,8 +913,8 @@ attn_merge_kernel(const AttnArgs a) {
             a.out[(head0 + hq) * kD + d] = 0;
             if (d == 0) a.lse[head0 + hq] = kNegInf;
         } else {
-            a.out[(head0 + hq) * kD + d] = f32_to_bf16_bits(acc[k] / s_l[hq]);
-            if (d == 0) a.lse[head0 + hq] = (s_m[hq] + log2f(s_l[hq])) * kLn2;
+            a.out[(head0 + hq) * kD + d] = f32_to_bf16_bits(acc[k] / s_sum[hq]);
+            if (d == 0) a.lse[head0 + hq] = (s_m[hq] + log2f(s_sum[hq])) * kLn2;
         }
     }
 }
@@ -893,61 +922,66 @@ attn_merge_kernel(const AttnArgs a) {
 // ---------------------------------------------------------------------------
 // host-side dispatch
 // ---------------------------------------------------------------------------
-template <bool kFp8, int kD, int kGP>
+template <bool kFp8, int kD, int kGP, int kH>
 static cudaError_t launch_variant(int grid, cudaStream_t stream, const CUtensorMap& tk,
                                   const CUtensorMap& tv, const AttnArgs& args) {
-    using C = AttnCfg<kFp8, kD, kGP>;
+    using C = AttnCfg<kFp8, kD, kGP, kH>;
     PdlLaunch l(dim3(grid), dim3(kAttnThreads), C::kSmemBytes, stream);
-    return cudaLaunchKernelEx(&l.cfg, attn_partial_kernel<kFp8, kD, kGP>, tk, tv, args);
+    return cudaLaunchKernelEx(&l.cfg, attn_partial_kernel<kFp8, kD, kGP, kH>, tk, tv, args);
 }
 
-#define PKV_FOR_EACH_VARIANT(X) \
-    X(true, 64, 8) X(true, 64, 16) X(true, 128, 8) X(true, 128, 16) \
-    X(false, 64, 8) X(false, 64, 16) X(false, 128, 8) X(false, 128, 16)
+// (fp8, head_dim, group pad, KV heads per item)
+#define PKV_FOR_EACH_VARIANT(X)                                                    \
+    X(true, 64, 8, 1) X(true, 64, 16, 1) X(true, 128, 8, 1) X(true, 128, 16, 1)    \
+    X(false, 64, 8, 1) X(false, 64, 16, 1) X(false, 128, 8, 1) X(false, 128, 16, 1) \
+    X(true, 64, 8, 2) X(true, 128, 8, 2)
 
-size_t attn_partial_smem_bytes(bool fp8, int head_dim, int group_pad) {
-#define X(F, D, GP) \
-    if (fp8 == F && head_dim == D && group_pad == GP) return AttnCfg<F, D, GP>::kSmemBytes;
+#define PKV_MATCH(F, D, GP, H) \
+    (fp8 == F && head_dim == D && group_pad == GP && kv_per_item == H)
+
+size_t attn_partial_smem_bytes(bool fp8, int head_dim, int group_pad, int kv_per_item) {
+#define X(F, D, GP, H) \
+    if (PKV_MATCH(F, D, GP, H)) return AttnCfg<F, D, GP, H>::kSmemBytes;
     PKV_FOR_EACH_VARIANT(X)
 #undef X
     return 0;
 }
 
-cudaError_t attn_set_smem_attr(bool fp8, int head_dim, int group_pad) {
-#define X(F, D, GP)                                                                        \
-    if (fp8 == F && head_dim == D && group_pad == GP)                                       \
-        return cudaFuncSetAttribute(attn_partial_kernel<F, D, GP>,                          \
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,            \
-                                    AttnCfg<F, D, GP>::kSmemBytes);
+cudaError_t attn_set_smem_attr(bool fp8, int head_dim, int group_pad, int kv_per_item) {
+#define X(F, D, GP, H)                                                              \
+    if (PKV_MATCH(F, D, GP, H))                                                      \
+        return cudaFuncSetAttribute(attn_partial_kernel<F, D, GP, H>,                \
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,     \
+                                    AttnCfg<F, D, GP, H>::kSmemBytes);
     PKV_FOR_EACH_VARIANT(X)
 #undef X
     return cudaErrorInvalidValue;
 }
 
-cudaError_t attn_occupancy(bool fp8, int head_dim, int group_pad, int* blocks_per_sm) {
-#define X(F, D, GP)                                                                         \
-    if (fp8 == F && head_dim == D && group_pad == GP)                                        \
-        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(                                \
-            blocks_per_sm, attn_partial_kernel<F, D, GP>, kAttnThreads,                      \
-            AttnCfg<F, D, GP>::kSmemBytes);
+cudaError_t attn_occupancy(bool fp8, int head_dim, int group_pad, int kv_per_item,
+                           int* blocks_per_sm) {
+#define X(F, D, GP, H)                                                               \
+    if (PKV_MATCH(F, D, GP, H))                                                       \
+        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(                         \
+            blocks_per_sm, attn_partial_kernel<F, D, GP, H>, kAttnThreads,            \
+            AttnCfg<F, D, GP, H>::kSmemBytes);
     PKV_FOR_EACH_VARIANT(X)
 #undef X
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_attn_partial(bool fp8, int head_dim, int group_pad, int grid,
+cudaError_t launch_attn_partial(bool fp8, int head_dim, int group_pad, int kv_per_item, int grid,
                                 cudaStream_t stream, const CUtensorMap& tmap_k,
                                 const CUtensorMap& tmap_v, const AttnArgs& args) {
-#define X(F, D, GP) \
-    if (fp8 == F && head_dim == D && group_pad == GP) \
-        return launch_variant<F, D, GP>(grid, stream, tmap_k, tmap_v, args);
+#define X(F, D, GP, H) \
+    if (PKV_MATCH(F, D, GP, H)) return launch_variant<F, D, GP, H>(grid, stream, tmap_k, tmap_v, args);
     PKV_FOR_EACH_VARIANT(X)
 #undef X
     return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_attn_merge(int head_dim, cudaStream_t stream, const AttnArgs& args) {
-    PdlLaunch l(dim3(args.batch * args.num_kv_heads), dim3(kMergeThreads), 0, stream);
+    PdlLaunch l(dim3(args.batch * args.items_per_req), dim3(kMergeThreads), 0, stream);
     if (head_dim == 64) return cudaLaunchKernelEx(&l.cfg, attn_merge_kernel<64>, args);
     return cudaLaunchKernelEx(&l.cfg, attn_merge_kernel<128>, args);
 }

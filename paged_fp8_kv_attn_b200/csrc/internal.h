@@ -26,8 +26,10 @@ struct AttnArgs {
     int32_t batch;
     int32_t max_pages;
     int32_t num_q_heads;
-    int32_t num_kv_heads;
-    int32_t group;
+    int32_t num_kv_heads;       // KV heads of the pool
+    int32_t kv_per_item;        // KV heads one work item covers (1 or 2)
+    int32_t items_per_req;      // num_kv_heads / kv_per_item
+    int32_t group;              // query heads per KV head
     int32_t page_size;
     int32_t num_pages;
     int32_t num_ctas;
@@ -39,21 +41,29 @@ struct AttnArgs {
 // Sets the message pkv_last_error() returns on this thread.
 void set_last_error(const char* message);
 
-// Workspace layout for given sizes and grid.
+// KV heads one attention work item covers: two adjacent heads (one
+// contiguous 16 KiB K or V block per 64-token page) for FP8 caches with an
+// even number of KV heads and a GQA group of at most 8; otherwise one.
+inline int kv_heads_per_item(bool fp8, int num_kv_heads, int group) {
+    return (fp8 && num_kv_heads % 2 == 0 && group <= 8) ? 2 : 1;
+}
+
+// Workspace layout for given sizes and grid (slots = grid + work items).
 struct WorkspaceLayout {
     size_t prefix_off, ml_off, o_off, total;
 };
 WorkspaceLayout workspace_layout(int32_t batch, int32_t group, int32_t num_kv_heads,
-                                 int32_t head_dim, int32_t num_ctas);
+                                 int32_t kv_per_item, int32_t head_dim, int32_t num_ctas);
 
 // Attention variant properties: dynamic shared memory bytes.  Returns 0 if
 // the combination is not compiled.
-size_t attn_partial_smem_bytes(bool fp8, int head_dim, int group_pad);
-cudaError_t attn_set_smem_attr(bool fp8, int head_dim, int group_pad);
-cudaError_t attn_occupancy(bool fp8, int head_dim, int group_pad, int* blocks_per_sm);
+size_t attn_partial_smem_bytes(bool fp8, int head_dim, int group_pad, int kv_per_item);
+cudaError_t attn_set_smem_attr(bool fp8, int head_dim, int group_pad, int kv_per_item);
+cudaError_t attn_occupancy(bool fp8, int head_dim, int group_pad, int kv_per_item,
+                           int* blocks_per_sm);
 constexpr int kAttnThreads = 160;   // 4 consumer warps + 1 producer warp
 
-cudaError_t launch_attn_partial(bool fp8, int head_dim, int group_pad, int grid,
+cudaError_t launch_attn_partial(bool fp8, int head_dim, int group_pad, int kv_per_item, int grid,
                                 cudaStream_t stream, const CUtensorMap& tmap_k,
                                 const CUtensorMap& tmap_v, const AttnArgs& args);
 cudaError_t launch_attn_merge(int head_dim, cudaStream_t stream, const AttnArgs& args);

@@ -172,35 +172,39 @@ check_append_kernel(const uint32_t* __restrict__ page_tags, int32_t num_pages,
     launch_dependents();
     grid_dependency_wait();
     const int b = blockIdx.x;
-    const int32_t L = seq_lens[b];
-    int bad = (L < 1 || static_cast<int64_t>(L) > static_cast<int64_t>(max_pages) * page_size);
     const int per_tensor = num_kv_heads * (head_dim / 8);
-    // the new token's values for this thread's first two 8-element groups,
-    // loaded before the check finishes (they are inputs, not cache contents)
+    const int32_t* row = page_table + static_cast<int64_t>(b) * max_pages;
+    const uint32_t* exp = expected_tags + static_cast<int64_t>(b) * max_pages;
+    // One round trip for everything that does not depend on the length: the
+    // length itself, this thread's first page-table entry and expected tag,
+    // and the new token's values for this thread's first two 8-element groups.
+    const int32_t L = seq_lens[b];
+    const int j0 = threadIdx.x;
+    const int32_t p_first = j0 < max_pages ? row[j0] : -1;
+    const uint32_t e_first = j0 < max_pages ? exp[j0] : 0u;
     uint4 raw[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int e = threadIdx.x + k * kFusedThreads;
+        if (e < 2 * per_tensor) {
+            const bool is_v = e >= per_tensor;
+            const int r = is_v ? e - per_tensor : e;
+            const int h = r / (head_dim / 8), d8 = r % (head_dim / 8);
+            raw[k] = *reinterpret_cast<const uint4*>(
+                (is_v ? v_new : k_new) + (static_cast<int64_t>(b) * num_kv_heads + h) * head_dim +
+                d8 * 8);
+        }
+    }
+    int bad = (L < 1 || static_cast<int64_t>(L) > static_cast<int64_t>(max_pages) * page_size);
     int32_t pid = -1, slot = 0;
     if (!bad) {
         const int32_t pos = L - 1;
         slot = pos % page_size;
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-            const int e = threadIdx.x + k * kFusedThreads;
-            if (e < 2 * per_tensor) {
-                const bool is_v = e >= per_tensor;
-                const int r = is_v ? e - per_tensor : e;
-                const int h = r / (head_dim / 8), d8 = r % (head_dim / 8);
-                raw[k] = *reinterpret_cast<const uint4*>(
-                    (is_v ? v_new : k_new) + (static_cast<int64_t>(b) * num_kv_heads + h) * head_dim +
-                    d8 * 8);
-            }
-        }
         const int32_t used = (L + page_size - 1) / page_size;
-        const int32_t* row = page_table + static_cast<int64_t>(b) * max_pages;
-        const uint32_t* exp = expected_tags + static_cast<int64_t>(b) * max_pages;
         pid = row[pos / page_size];
-        for (int j = threadIdx.x; j < used; j += kFusedThreads) {
-            const int32_t p = row[j];
-            const uint32_t want = exp[j];
+        for (int j = j0; j < used; j += kFusedThreads) {
+            const int32_t p = (j == j0) ? p_first : row[j];
+            const uint32_t want = (j == j0) ? e_first : exp[j];
             if (p < 0 || p >= num_pages)
                 bad = 1;
             else if (__ldg(page_tags + p) != want)

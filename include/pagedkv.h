@@ -176,6 +176,32 @@ PKV_API pkv_status kv_check_append_bf16(const uint32_t* page_tags, int32_t num_p
                                 void* stream);
 
 /*
+ * kv_retag_pages -- device-side tag bump for reallocated pages.
+ * [T] "保护共享 KV cache": a physical page gets a tag that changes whenever the
+ * page is reallocated; [R] "共享 KV 缓存安全性成为生产问题" likens it to a
+ * generation counter.  For every i < num_ids with pages[i] inside
+ * [0, num_pages): page_tags[pages[i]] += 1 (mod 2^32), once per occurrence in
+ * the list (atomically, so duplicates are counted).  Other ids are ignored.
+ * page_tags [num_pages] uint32 (updated in place); pages [num_ids] int32.
+ */
+PKV_API pkv_status kv_retag_pages(uint32_t* page_tags, int32_t num_pages, const int32_t* pages,
+                                  int32_t num_ids, void* stream);
+
+/*
+ * kv_expected_tags -- rebuild each request's expected tags from the current
+ * page tags ([T] "保护共享 KV cache": the server records the pages and tags each
+ * request expects).  For every request b with seq_lens[b] inside
+ * [1, max_pages * page_size] and every used entry j < ceil(seq_lens[b] /
+ * page_size) naming a page inside [0, num_pages):
+ *   expected_tags[b][j] = page_tags[page_table[b][j]].
+ * Every other entry is left unchanged.  Layouts as for kv_tag_check.
+ */
+PKV_API pkv_status kv_expected_tags(const uint32_t* page_tags, int32_t num_pages,
+                                    const int32_t* page_table, int32_t max_pages,
+                                    const int32_t* seq_lens, int32_t batch, int32_t page_size,
+                                    uint32_t* expected_tags, void* stream);
+
+/*
  * kv_requant_pages_fp8 -- BF16 -> FP8 page handoff.  [S] "KV 快取量化" and
  * [T] "量化 KV cache": the prefill pool keeps a BF16 cache while the decode
  * pool stores FP8.  Page src_pages[i] of the BF16 pool is re-quantised into

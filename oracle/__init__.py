@@ -68,6 +68,8 @@ def _load():
                                                P, P, i32, P]
             lib.orc_kv_requant_pages_fp8.argtypes = [P, i32, P, P, i32, P, i32, i32,
                                                      i32, i32, f32]
+            lib.orc_kv_retag_pages.argtypes = [P, i32, P, i32]
+            lib.orc_kv_expected_tags.argtypes = [P, i32, P, i32, P, i32, i32, P]
             lib.orc_paged_decode_attn.argtypes = [i32, P, P, P, f32, f32, P, i32, P, i32,
                                                   i32, i32, i32, i32, i32, f32, P, P, i32,
                                                   P, P]
@@ -149,6 +151,28 @@ def kv_tag_check(page_tags, page_table, expected_tags, seq_lens, page_size):
                              _ptr(expected_tags), MP, _ptr(seq_lens), B, page_size,
                              _ptr(abort))
     return abort, int(n)
+
+
+def kv_retag_pages(page_tags, pages):
+    """Bump (mod 2^32) the tag of every listed page id inside the pool, in place."""
+    lib = _load()
+    if page_tags.dtype != np.uint32 or not page_tags.flags.c_contiguous:
+        raise TypeError("page_tags must be a C-contiguous uint32 array")
+    pages = _c(pages, np.int32)
+    lib.orc_kv_retag_pages(_ptr(page_tags), page_tags.size, _ptr(pages), pages.size)
+
+
+def kv_expected_tags(page_tags, page_table, seq_lens, page_size, expected_tags):
+    """Rebuild each request's expected tags from the current page tags, in place."""
+    lib = _load()
+    page_tags = _c(page_tags, np.uint32)
+    page_table = _c(page_table, np.int32)
+    seq_lens = _c(seq_lens, np.int32)
+    if expected_tags.dtype != np.uint32 or not expected_tags.flags.c_contiguous:
+        raise TypeError("expected_tags must be a C-contiguous uint32 array")
+    B, MP = page_table.shape
+    lib.orc_kv_expected_tags(_ptr(page_tags), page_tags.size, _ptr(page_table), MP,
+                             _ptr(seq_lens), B, page_size, _ptr(expected_tags))
 
 
 def kv_append_fp8(k_new_bits, v_new_bits, page_table, seq_lens, page_size,

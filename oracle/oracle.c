@@ -211,6 +211,42 @@ int32_t orc_kv_tag_check(const uint32_t* page_tags, int32_t num_pages,
     return aborted;
 }
 
+/* [T] "保护共享 KV cache" and [R] "共享 KV 缓存安全性成为生产问题": a page's tag
+ * changes whenever the page is reallocated (like a generation counter).
+ * Every listed page id inside [0, NP) has its tag increased by one, modulo
+ * 2^32, once per occurrence in the list; other ids are ignored. */
+void orc_kv_retag_pages(uint32_t* page_tags, int32_t num_pages, const int32_t* pages, int32_t n)
+{
+    for (int32_t i = 0; i < n; ++i) {
+        int32_t p = pages[i];
+        if (p >= 0 && p < num_pages)
+            page_tags[p] = page_tags[p] + 1u;
+    }
+}
+
+/* The server records, per request, the tags it expects for its pages: for
+ * every used entry j < ceil(L_b / P) that names a page inside [0, NP),
+ * expected_tags[b][j] = page_tags[page_table[b][j]].  Entries naming a page
+ * outside the pool, entries past the used ones and requests whose length is
+ * outside [1, MP*P] are left unchanged. */
+void orc_kv_expected_tags(const uint32_t* page_tags, int32_t num_pages,
+                          const int32_t* page_table, int32_t max_pages,
+                          const int32_t* seq_lens, int32_t batch, int32_t page_size,
+                          uint32_t* expected_tags)
+{
+    for (int32_t b = 0; b < batch; ++b) {
+        int32_t L = seq_lens[b];
+        if (L < 1 || (int64_t)L > (int64_t)max_pages * page_size)
+            continue;
+        int32_t used = (L + page_size - 1) / page_size;
+        for (int32_t j = 0; j < used; ++j) {
+            int32_t pid = page_table[(int64_t)b * max_pages + j];
+            if (pid >= 0 && pid < num_pages)
+                expected_tags[(int64_t)b * max_pages + j] = page_tags[pid];
+        }
+    }
+}
+
 /* ------------------------------------------------------------------------ */
 /* Quantise-and-append of the new token                                     */
 /* ------------------------------------------------------------------------ */

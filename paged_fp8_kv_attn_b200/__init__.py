@@ -57,6 +57,8 @@ def _load():
             "kv_append_fp8": [P, P, P, i32, P, i32, i32, i32, i32, f32, f32, P, P, i32, P, P],
             "kv_append_bf16": [P, P, P, i32, P, i32, i32, i32, i32, P, P, i32, P, P],
             "kv_requant_pages_fp8": [P, i32, P, P, i32, P, i32, i32, i32, i32, f32, P],
+            "kv_retag_pages": [P, i32, P, i32, P],
+            "kv_expected_tags": [P, i32, P, i32, P, i32, i32, P, P],
             "kv_check_append_fp8": [P, i32, P, P, i32, P, i32, i32, P, P, i32, i32, f32, f32, P, P,
                                     P, P, P],
             "kv_check_append_bf16": [P, i32, P, P, i32, P, i32, i32, P, P, i32, i32, P, P, P, P,
@@ -135,6 +137,26 @@ def kv_tag_check(page_tags, page_table, expected_tags, seq_lens, page_size, abor
     _check("kv_tag_check", _load().kv_tag_check(
         _ptr(page_tags), page_tags.shape[0], _ptr(page_table), _ptr(expected_tags), MP,
         _ptr(seq_lens), B, page_size, _ptr(abort_out), _ptr(num_aborted), _stream(stream)))
+
+
+def kv_retag_pages(page_tags, pages, stream=None):
+    """Bump (mod 2^32) the tag of every listed page id inside the pool, in place."""
+    _need(page_tags, _TAG_DTYPES, 1, "page_tags")
+    _need(pages, torch.int32, 1, "pages")
+    _check("kv_retag_pages", _load().kv_retag_pages(
+        _ptr(page_tags), page_tags.shape[0], _ptr(pages), pages.shape[0], _stream(stream)))
+
+
+def kv_expected_tags(page_tags, page_table, seq_lens, page_size, expected_tags, stream=None):
+    """Rebuild each request's expected tags from the current page tags, in place."""
+    _need(page_tags, _TAG_DTYPES, 1, "page_tags")
+    _need(page_table, torch.int32, 2, "page_table")
+    _need(seq_lens, torch.int32, 1, "seq_lens")
+    _need(expected_tags, _TAG_DTYPES, 2, "expected_tags")
+    B, MP = page_table.shape
+    _check("kv_expected_tags", _load().kv_expected_tags(
+        _ptr(page_tags), page_tags.shape[0], _ptr(page_table), MP, _ptr(seq_lens), B, page_size,
+        _ptr(expected_tags), _stream(stream)))
 
 
 def kv_append_fp8(k_new, v_new, page_table, seq_lens, page_size, k_scale, v_scale,

@@ -403,6 +403,35 @@ pkv_status kv_check_append_bf16(const uint32_t* page_tags, int32_t num_pages,
                              1.f, 1.f, k_cache, v_cache, abort_out, num_aborted, stream);
 }
 
+pkv_status kv_retag_pages(uint32_t* page_tags, int32_t num_pages, const int32_t* pages,
+                          int32_t num_ids, void* stream) {
+    if (num_pages < 1 || num_ids < 0)
+        return fail(PKV_ERR_INVALID_ARG, "num_pages must be >= 1 and num_ids >= 0");
+    if (num_ids == 0) return PKV_OK;
+    if (!page_tags || !pages) return fail(PKV_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned(page_tags, 4) || !aligned(pages, 4))
+        return fail(PKV_ERR_INVALID_ARG, "misaligned pointer");
+    cudaError_t e = pkv::launch_retag(page_tags, num_pages, pages, num_ids, as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "retag launch");
+    return PKV_OK;
+}
+
+pkv_status kv_expected_tags(const uint32_t* page_tags, int32_t num_pages,
+                            const int32_t* page_table, int32_t max_pages,
+                            const int32_t* seq_lens, int32_t batch, int32_t page_size,
+                            uint32_t* expected_tags, void* stream) {
+    if (batch < 0 || num_pages < 1 || max_pages < 1 || page_size < 1)
+        return fail(PKV_ERR_INVALID_ARG, "invalid sizes");
+    if (batch == 0) return PKV_OK;
+    if (!page_tags || !page_table || !seq_lens || !expected_tags)
+        return fail(PKV_ERR_INVALID_ARG, "null pointer argument");
+    cudaError_t e = pkv::launch_expected_tags(page_tags, num_pages, page_table, max_pages,
+                                              seq_lens, batch, page_size, expected_tags,
+                                              as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "expected-tags launch");
+    return PKV_OK;
+}
+
 pkv_status kv_requant_pages_fp8(const uint16_t* src_pool, int32_t src_num_pages,
                                 const int32_t* src_pages, uint8_t* dst_pool,
                                 int32_t dst_num_pages, const int32_t* dst_pages,

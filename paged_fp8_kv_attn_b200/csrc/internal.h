@@ -89,6 +89,13 @@ cudaError_t launch_check_append(bool fp8, const uint32_t* page_tags, int32_t num
                                 float v_scale, void* k_cache, void* v_cache, uint8_t* abort_out,
                                 int32_t* num_aborted, cudaStream_t stream);
 
+cudaError_t launch_retag(uint32_t* page_tags, int32_t num_pages, const int32_t* pages, int32_t n,
+                         cudaStream_t stream);
+cudaError_t launch_expected_tags(const uint32_t* page_tags, int32_t num_pages,
+                                 const int32_t* page_table, int32_t max_pages,
+                                 const int32_t* seq_lens, int32_t batch, int32_t page_size,
+                                 uint32_t* expected_tags, cudaStream_t stream);
+
 cudaError_t launch_requant(const uint16_t* src_pool, int32_t src_num_pages,
                            const int32_t* src_pages, uint8_t* dst_pool, int32_t dst_num_pages,
                            const int32_t* dst_pages, int32_t num_pairs, int64_t page_elems,

@@ -263,6 +263,59 @@ cudaError_t launch_check_append(bool fp8, const uint32_t* page_tags, int32_t num
 }
 
 // ---------------------------------------------------------------------------
+// page reallocation bookkeeping: tag bumps and expected-tag rebuilds
+// ("保护共享 KV cache": a page's tag changes whenever it is reallocated; the
+// server records each request's expected tags)
+// ---------------------------------------------------------------------------
+constexpr int kTagOpThreads = 256;
+
+__global__ void __launch_bounds__(kTagOpThreads)
+retag_kernel(uint32_t* __restrict__ page_tags, int32_t num_pages,
+             const int32_t* __restrict__ pages, int32_t n) {
+    launch_dependents();
+    grid_dependency_wait();
+    for (int i = blockIdx.x * kTagOpThreads + threadIdx.x; i < n; i += gridDim.x * kTagOpThreads) {
+        const int32_t p = pages[i];
+        if (p >= 0 && p < num_pages) atomicAdd(page_tags + p, 1u);   // wraps mod 2^32
+    }
+}
+
+__global__ void __launch_bounds__(kTagOpThreads)
+expected_tags_kernel(const uint32_t* __restrict__ page_tags, int32_t num_pages,
+                     const int32_t* __restrict__ page_table, int32_t max_pages,
+                     const int32_t* __restrict__ seq_lens, int32_t page_size,
+                     uint32_t* __restrict__ expected_tags) {
+    launch_dependents();
+    grid_dependency_wait();
+    const int b = blockIdx.x;
+    const int32_t L = seq_lens[b];
+    if (L < 1 || static_cast<int64_t>(L) > static_cast<int64_t>(max_pages) * page_size) return;
+    const int32_t used = (L + page_size - 1) / page_size;
+    const int64_t row = static_cast<int64_t>(b) * max_pages;
+    for (int j = threadIdx.x; j < used; j += kTagOpThreads) {
+        const int32_t p = page_table[row + j];
+        if (p >= 0 && p < num_pages) expected_tags[row + j] = page_tags[p];
+    }
+}
+
+cudaError_t launch_retag(uint32_t* page_tags, int32_t num_pages, const int32_t* pages, int32_t n,
+                         cudaStream_t stream) {
+    int blocks = (n + kTagOpThreads - 1) / kTagOpThreads;
+    if (blocks > 1024) blocks = 1024;
+    PdlLaunch l(dim3(blocks), dim3(kTagOpThreads), 0, stream);
+    return cudaLaunchKernelEx(&l.cfg, retag_kernel, page_tags, num_pages, pages, n);
+}
+
+cudaError_t launch_expected_tags(const uint32_t* page_tags, int32_t num_pages,
+                                 const int32_t* page_table, int32_t max_pages,
+                                 const int32_t* seq_lens, int32_t batch, int32_t page_size,
+                                 uint32_t* expected_tags, cudaStream_t stream) {
+    PdlLaunch l(dim3(batch), dim3(kTagOpThreads), 0, stream);
+    return cudaLaunchKernelEx(&l.cfg, expected_tags_kernel, page_tags, num_pages, page_table,
+                              max_pages, seq_lens, page_size, expected_tags);
+}
+
+// ---------------------------------------------------------------------------
 // BF16 -> FP8 page handoff: grid-stride over 16-element groups
 // ---------------------------------------------------------------------------
 constexpr int kRequantThreads = 256;

@@ -333,3 +333,31 @@ def test_attention_rejects_bad_arguments(cuda_device):
         pkv.paged_decode_attn_fp8(db.q, db.k_cache, db.v_cache, wl.k_scale, wl.v_scale,
                                   db.page_table, db.seq_lens, wl.sm_scale, db.out, db.lse,
                                   ws[:64])
+
+
+# --------------------------------------------------------------------------
+# page reallocation bookkeeping: bit-exact
+# --------------------------------------------------------------------------
+
+def test_retag_and_expected_tags_bit_exact(cuda_device):
+    wl = workloads.integrity_stress(batch=64, lo=64, hi=4000, stale_fraction=0.01)
+    rng = np.random.Generator(np.random.PCG64(3))
+    moved = rng.choice(wl.num_pages, size=500, replace=True).astype(np.int32)   # duplicates
+    moved[:5] = [-1, wl.num_pages, wl.num_pages + 100, -50, 0]
+    tags = wl.page_tags.copy()
+    tags[0] = np.uint32(0xFFFFFFFF)
+    d_tags = _cuda_u32(tags)
+    pkv.kv_retag_pages(d_tags, torch.from_numpy(moved).cuda())
+    want_tags = tags.copy()
+    oracle.kv_retag_pages(want_tags, moved)
+    torch.cuda.synchronize()
+    assert np.array_equal(d_tags.cpu().numpy().view(np.uint32), want_tags)
+    exp = np.full_like(wl.expected_tags, 0x5A5A5A5A)
+    d_exp = _cuda_u32(exp)
+    lens = wl.seq_lens.copy()
+    lens[3] = 0
+    pkv.kv_expected_tags(d_tags, torch.from_numpy(wl.page_table).cuda(),
+                         torch.from_numpy(lens).cuda(), 64, d_exp)
+    oracle.kv_expected_tags(want_tags, wl.page_table, lens, 64, exp)
+    torch.cuda.synchronize()
+    assert np.array_equal(d_exp.cpu().numpy().view(np.uint32), exp)

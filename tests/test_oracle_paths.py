@@ -303,3 +303,50 @@ def test_attention_nan_code_propagates():
                                         16, wl.sm_scale, wl.k_scale, wl.v_scale)
     assert np.isnan(out[0, 2:4]).all() and np.isnan(lse[0, 2:4]).all()
     assert np.isfinite(out[0, 0:2]).all() and np.isfinite(out[1]).all()
+
+
+# --------------------------------------------------------------------------
+# page reallocation bookkeeping
+# --------------------------------------------------------------------------
+
+def test_retag_pages_brute_force():
+    rng = _rng(41)
+    tags = rng.integers(0, 2**32, 50, dtype=np.uint64).astype(np.uint32)
+    tags[7] = np.uint32(0xFFFFFFFF)                   # wraps to 0
+    pages = np.array([7, 3, 3, -1, 50, 12, 7, 0], dtype=np.int32)
+    want = [int(t) for t in tags]
+    for p in pages:                                   # written out independently
+        if 0 <= p < 50:
+            want[p] = (want[p] + 1) % 2**32
+    got = tags.copy()
+    oracle.kv_retag_pages(got, pages)
+    assert [int(t) for t in got] == want
+    assert got[7] == 1 and got[3] == tags[3] + 2
+
+
+def test_expected_tags_rebuild_then_check_passes():
+    wl = workloads.integrity_stress(batch=30, lo=64, hi=3000, stale_fraction=0.02)
+    a, _ = oracle.kv_tag_check(wl.page_tags, wl.page_table, wl.expected_tags, wl.seq_lens, 64)
+    assert a.any()
+    exp = np.full_like(wl.expected_tags, 0xDEADBEEF)
+    oracle.kv_expected_tags(wl.page_tags, wl.page_table, wl.seq_lens, 64, exp)
+    a2, n2 = oracle.kv_tag_check(wl.page_tags, wl.page_table, exp, wl.seq_lens, 64)
+    assert n2 == 0 and not a2.any()
+    for b in range(wl.batch):                         # untouched past the used entries
+        assert (exp[b, wl.used_pages(b):] == 0xDEADBEEF).all()
+
+
+def test_reallocation_round_trip():
+    """Reassigning pages bumps their tags: requests still holding them fail the
+    check until their expected tags are rebuilt."""
+    wl = workloads.custom([100, 200, 50], page_size=16, num_q_heads=4, num_kv_heads=1,
+                          head_dim=64, seed=8)
+    tags = wl.page_tags.copy()
+    moved = wl.page_table[1, :3].copy()
+    oracle.kv_retag_pages(tags, moved)
+    a, _ = oracle.kv_tag_check(tags, wl.page_table, wl.expected_tags, wl.seq_lens, 16)
+    assert a.tolist() == [0, 1, 0]
+    exp = wl.expected_tags.copy()
+    oracle.kv_expected_tags(tags, wl.page_table, wl.seq_lens, 16, exp)
+    a, _ = oracle.kv_tag_check(tags, wl.page_table, exp, wl.seq_lens, 16)
+    assert a.tolist() == [0, 0, 0]

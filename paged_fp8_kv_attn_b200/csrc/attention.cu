@@ -791,8 +791,11 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
 // segments, merged online), then every thread sums its (head, dim) outputs
 // with independent loads.
 // ---------------------------------------------------------------------------
-constexpr int kMergeThreads = 512;
-constexpr int kMergeTile = 256;
+// Small enough (threads, registers, shared memory) to be resident next to two
+// partial-kernel CTAs per SM, so the merge grid is launched early and starts
+// the moment the partial kernel completes.
+constexpr int kMergeThreads = 128;
+constexpr int kMergeTile = 64;
 
 __device__ __forceinline__ int64_t cta_of_unit(int64_t u, int64_t U, int N) {
     // largest c with floor(c * U / N) <= u
@@ -907,7 +910,7 @@ attn_merge_kernel(const AttnArgs a) {
 #pragma unroll
     for (int k = 0; k < kPer; ++k) {
         const int e = tid + k * kMergeThreads;
-        if (e >= G * kD) break;
+        if (e >= G * kD) continue;
         const int hq = e / kD, d = e % kD;
         if (s_dead) {
             a.out[(head0 + hq) * kD + d] = 0;

@@ -791,11 +791,8 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
 // segments, merged online), then every thread sums its (head, dim) outputs
 // with independent loads.
 // ---------------------------------------------------------------------------
-// Small enough (threads, registers, shared memory) to be resident next to two
-// partial-kernel CTAs per SM, so the merge grid is launched early and starts
-// the moment the partial kernel completes.
-constexpr int kMergeThreads = 128;
-constexpr int kMergeTile = 64;
+constexpr int kMergeThreads = 512;
+constexpr int kMergeTile = 256;
 
 __device__ __forceinline__ int64_t cta_of_unit(int64_t u, int64_t U, int N) {
     // largest c with floor(c * U / N) <= u
@@ -910,7 +907,7 @@ attn_merge_kernel(const AttnArgs a) {
 #pragma unroll
     for (int k = 0; k < kPer; ++k) {
         const int e = tid + k * kMergeThreads;
-        if (e >= G * kD) continue;
+        if (e >= G * kD) break;
         const int hq = e / kD, d = e % kD;
         if (s_dead) {
             a.out[(head0 + hq) * kD + d] = 0;

@@ -80,10 +80,29 @@ struct AttnCfg {
     static constexpr int kFlagOff = kBarOff + 2 * kStages * 8;
     static constexpr int kScratchOff = kFlagOff + kStages * 4;
     static constexpr int kSmemBytes = kScratchOff + 16 * 4 + 1024;  // + alignment slack
+    // Registers per thread holding a segment's raw query words.  They are
+    // loaded before the previous segment's epilogue when that adds at most
+    // 16 live registers to a variant with the 2-CTA register budget (168);
+    // otherwise (more words, or the tighter 3-CTA budget) at the segment's
+    // start.
+    static constexpr int kQWords = kFp8 ? (kGP / 8) * (kD / 64) * 8 : (kGP / 8) * (kD / 16) * 2;
+    static constexpr bool kEarlyQ = kQWords <= 16 && kMinBlocks == 2;
     static_assert(kD == 64 || kD == 128, "head_dim");
     static_assert(kGP == 8 || kGP == 16, "group pad");
     static_assert(kH == 1 || (kH == 2 && kGP == 8), "two KV heads per item need a group <= 8");
 };
+
+// XOR applied to the 16-byte unit index of the epilogue's O rows written by
+// lanes with thread-in-group c (rows 2c, 2c+1 of each 8-head block).  Chosen
+// per accumulator layout so that one store instruction's lanes (and each
+// 8-lane phase of a 16-byte store) reach distinct banks: FP8 D=128 stores
+// units 4g+k, FP8 D=64 units 2g+k, BF16 single words of units 4mb+g/4 (+2).
+template <bool kFp8, int kD>
+__device__ __forceinline__ uint32_t red_swizzle(int c) {
+    if constexpr (!kFp8) return 2u * c;
+    else if constexpr (kD == 128) return static_cast<uint32_t>(c);
+    else return static_cast<uint32_t>((c & 1) | ((c & 2) << 1));
+}
 
 // Token permutation inside an 8-row group: row tau(n) feeds MMA column n.
 __device__ __forceinline__ int tau(int n) { return n ^ ((n & 1) << 2); }
@@ -173,6 +192,11 @@ struct PageWindow {
     __device__ __forceinline__ void reset(const int32_t* r) {
         row = r;
         base = -(1 << 30);
+    }
+    // Issues the load of the window starting at entry j ahead of its use.
+    __device__ __forceinline__ void preload(int j, int limit, int lane) {
+        base = j;
+        mine = (j + lane < limit) ? row[j + lane] : -1;
     }
     __device__ __forceinline__ int32_t get(int j, int limit, int lane) {
         if (j < base || j >= base + 32) {
@@ -312,11 +336,36 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
         }
         grid_dependency_wait();
+        // A segment's abort flag and first page-table window are loaded one
+        // segment ahead, so the first TMA of a segment waits on no load.
+        auto load_meta = [&](const Segment& sg, PageWindow& w) {
+            w.reset(a.page_table + static_cast<int64_t>(sg.b) * a.max_pages);
+            w.preload(sg.c0 * kChunkTokens / P, (sg.L + P - 1) / P, lane);
+            return (a.abort != nullptr) ? static_cast<int>(a.abort[sg.b]) : 0;
+        };
         uint32_t it = 0;
         Segment s;
-        while (walk.next(s)) {
-            if (a.abort != nullptr && a.abort[s.b] != 0) continue;
-            win.reset(a.page_table + static_cast<int64_t>(s.b) * a.max_pages);
+        bool have = walk.next(s);
+        int aborted = have ? load_meta(s, win) : 0;
+        while (have) {
+            Segment sn;
+            const bool have_next = walk.next(sn);
+            PageWindow next_win;
+            const int next_aborted = have_next ? load_meta(sn, next_win) : 0;
+            if (aborted) {
+                win = next_win;
+                aborted = next_aborted;
+                s = sn;
+                have = have_next;
+                continue;
+            }
+            // the consumers load this segment's query rows at the end of the
+            // previous one: start bringing them into L2 now
+            {
+                const int64_t q0 = (static_cast<int64_t>(s.b) * a.num_q_heads +
+                                    static_cast<int64_t>(s.h) * kH * a.group) * kD;
+                if (lane * 64 < kH * a.group * kD) prefetch_l2(a.q + q0 + lane * 64);
+            }
             const int npages = (s.L + P - 1) / P;
             for (int ch = s.c0; ch < s.c1; ++ch, ++it) {
                 const int stage = it % S;
@@ -366,6 +415,10 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 }
                 __syncwarp();
             }
+            win = next_win;
+            aborted = next_aborted;
+            s = sn;
+            have = have_next;
         }
         return;
     }
@@ -408,16 +461,59 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
             v_off[i] = swz<C::kRowBytes, C::kSwizzle>(vr[i], (kD == 128 ? 16 : 8) * g);
     }
 
+    // This warp's query rows of a segment as raw words: FP8, per n-block and
+    // 64-dim part the 16 bf16 dims [16c, 16c+16) (8 words); BF16, the two
+    // B-operand words of each k-step.  Heads past the group read as zero.
+    constexpr int kQWords = C::kQWords;
+    auto load_q = [&](const Segment& sg, uint32_t (&w)[kQWords]) {
+        const int64_t hw0 = static_cast<int64_t>(sg.b) * a.num_q_heads + sg.h * IQ + kvh_w * G;
+#pragma unroll
+        for (int nb = 0; nb < kNB; ++nb) {
+            const int hh = g + 8 * nb;
+            const bool valid = hh < G;
+            const uint16_t* qrow = a.q + (hw0 + (valid ? hh : 0)) * kD;
+            if constexpr (kFp8) {
+#pragma unroll
+                for (int part = 0; part < kD / 64; ++part) {
+                    const uint4* src = reinterpret_cast<const uint4*>(qrow + part * 64 + 16 * c);
+                    const uint4 w0 = src[0], w1 = src[1];
+                    uint32_t* d = &w[(nb * (kD / 64) + part) * 8];
+                    d[0] = valid ? w0.x : 0u; d[1] = valid ? w0.y : 0u;
+                    d[2] = valid ? w0.z : 0u; d[3] = valid ? w0.w : 0u;
+                    d[4] = valid ? w1.x : 0u; d[5] = valid ? w1.y : 0u;
+                    d[6] = valid ? w1.z : 0u; d[7] = valid ? w1.w : 0u;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < kKS; ++j) {
+                    const uint32_t* src = reinterpret_cast<const uint32_t*>(qrow + 16 * j + 2 * c);
+                    w[(nb * kKS + j) * 2 + 0] = valid ? src[0] : 0u;
+                    w[(nb * kKS + j) * 2 + 1] = valid ? src[4] : 0u;
+                }
+            }
+        }
+        return (a.abort != nullptr) ? static_cast<int>(a.abort[sg.b]) : 0;
+    };
+
+    // A segment's query words and abort flag are loaded before the previous
+    // segment's epilogue (C::kEarlyQ), which hides their latency behind it.
     uint32_t it = 0;
+    uint32_t qw[kQWords];
     Segment s;
-    while (walk.next(s)) {
+    bool have = walk.next(s);
+    int aborted = 0;
+    if constexpr (C::kEarlyQ) aborted = have ? load_q(s, qw) : 0;
+    while (have) {
+        Segment sn;
+        const bool have_next = walk.next(sn);
+        if constexpr (!C::kEarlyQ) aborted = load_q(s, qw);
         const int item = s.b * IPR + s.h;
         const bool whole = (s.c0 == 0 && s.c1 == s.n);
         const int64_t slot = static_cast<int64_t>(blockIdx.x) + item;
         const int64_t head0 = static_cast<int64_t>(s.b) * a.num_q_heads + s.h * IQ;  // item
         const int64_t head0_w = head0 + kvh_w * G;                                    // this warp
 
-        if (a.abort != nullptr && a.abort[s.b] != 0) {
+        if (aborted) {
             for (int e = tid; e < IQ * kD; e += kConsumerThreads) {
                 const int hq = e / kD, d = e % kD;
                 if (whole) {
@@ -431,6 +527,9 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     }
                 }
             }
+            if constexpr (C::kEarlyQ) aborted = have_next ? load_q(sn, qw) : 0;
+            s = sn;
+            have = have_next;
             continue;
         }
 
@@ -439,48 +538,44 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
         float qs[kNB][2];   // score scale of S columns 2c and 2c+1
 #pragma unroll
         for (int nb = 0; nb < kNB; ++nb) {
-            const int hh = g + 8 * nb;
-            const bool valid = hh < G;
-            const uint16_t* qrow = a.q + (head0_w + (valid ? hh : 0)) * kD;
             float my_scale;
             if constexpr (kFp8) {
-                // this thread's dims: [16c, 16c+16) and, for D=128, [64+16c, 64+16c+16);
-                // word j of them holds dims D_c[4j..4j+3] of the permuted contraction
+                // word j of the B operand holds dims D_c[4j..4j+3] of the
+                // permuted contraction: this thread's dims in order
                 float v[kD / 4];
 #pragma unroll
-                for (int part = 0; part < kD / 64; ++part) {
-                    const uint4* src = reinterpret_cast<const uint4*>(qrow + part * 64 + 16 * c);
-                    const uint4 w0 = src[0], w1 = src[1];
-                    const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        v[part * 16 + 2 * k] = valid ? bf16_bits_to_f32(ws[k] & 0xFFFFu) : 0.f;
-                        v[part * 16 + 2 * k + 1] = valid ? bf16_bits_to_f32(ws[k] >> 16) : 0.f;
-                    }
+                for (int k = 0; k < kD / 8; ++k) {
+                    const uint32_t w = qw[nb * (kD / 8) + k];
+                    v[2 * k] = bf16_bits_to_f32(w & 0xFFFFu);
+                    v[2 * k + 1] = bf16_bits_to_f32(w >> 16);
                 }
                 float amax = 0.f;
 #pragma unroll
                 for (int k = 0; k < kD / 4; ++k) amax = fmaxf(amax, fabsf(v[k]));
                 amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
                 amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-                int e = 0;
+                // 2^shift brings amax into [128, 256): with amax = f 2^e,
+                // f in [0.5, 1), shift = 8 - e, where e comes from the
+                // exponent field (a subnormal amax reads as e = -126, which
+                // the clamp maps to the same shift as its true exponent)
                 int shift = 0;
                 if (amax > 0.f && isfinite(amax)) {
-                    frexpf(amax, &e);
+                    const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu) - 126;
                     shift = min(60, max(-126, 8 - e));
                 }
+                // scaling by an exact power of two rounds like ldexp
+                const float up = __uint_as_float(static_cast<uint32_t>(shift + 127) << 23);
 #pragma unroll
                 for (int j = 0; j < kKS; ++j) {
-                    qb[nb][j][0] = pack_f16x2(ldexpf(v[4 * j], shift), ldexpf(v[4 * j + 1], shift));
-                    qb[nb][j][1] = pack_f16x2(ldexpf(v[4 * j + 2], shift), ldexpf(v[4 * j + 3], shift));
+                    qb[nb][j][0] = pack_f16x2(v[4 * j] * up, v[4 * j + 1] * up);
+                    qb[nb][j][1] = pack_f16x2(v[4 * j + 2] * up, v[4 * j + 3] * up);
                 }
-                my_scale = a.qk_scale * ldexpf(1.f, -shift);
+                my_scale = a.qk_scale * __uint_as_float(static_cast<uint32_t>(127 - shift) << 23);
             } else {
 #pragma unroll
                 for (int j = 0; j < kKS; ++j) {
-                    const uint32_t* src = reinterpret_cast<const uint32_t*>(qrow + 16 * j + 2 * c);
-                    qb[nb][j][0] = valid ? src[0] : 0u;
-                    qb[nb][j][1] = valid ? src[4] : 0u;
+                    qb[nb][j][0] = qw[(nb * kKS + j) * 2 + 0];
+                    qb[nb][j][1] = qw[(nb * kKS + j) * 2 + 1];
                 }
                 my_scale = a.qk_scale;
             }
@@ -694,6 +789,10 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
             __syncwarp();
             if (lane == 0 && !(C::kRedInStage && ch + 1 == s.c1)) mbar_arrive(&empty_bar[stage]);
         }
+        // the next segment's query words and abort flag, consumed after the epilogue
+        int next_aborted = 0;
+        if constexpr (C::kEarlyQ) next_aborted = have_next ? load_q(sn, qw) : 0;
+
         const int last_stage = (it + S - 1) % S;   // stage of the segment's last chunk
         float* red_o = C::kRedInStage ? reinterpret_cast<float*>(smem + last_stage * C::kStageBytes)
                                       : red_o_own;
@@ -702,7 +801,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
             named_barrier_sync(1, kConsumerThreads);
         }
 
-        // ---- epilogue: combine the four warps, then write ---------------
+        // ---- epilogue: combine the warps of each KV head, then write ------
 #pragma unroll
         for (int nb = 0; nb < kNB; ++nb)
 #pragma unroll
@@ -722,56 +821,86 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     red_l[warp * kGP + 8 * nb + 2 * c + col] = l[nb][col];
                 }
         }
+        // O into red_o[warp][head][kD] (fp32); the 16-byte units of a row are
+        // XOR-swizzled by red_swizzle of the row's head pair, which makes
+        // these writes and the row-contiguous reads below conflict-free.
+        {
+            const uint32_t sw = red_swizzle<kFp8, kD>(c);
 #pragma unroll
-        for (int nb = 0; nb < kNB; ++nb)
+            for (int nb = 0; nb < kNB; ++nb)
 #pragma unroll
-            for (int mb = 0; mb < kMB; ++mb) {
-                // rows of the O^T accumulator: dims d_lo (i = 0, 1) and d_hi (i = 2, 3)
-                int d_lo, d_hi;
-                if constexpr (kFp8) {
-                    d_lo = (kD == 128 ? 16 : 8) * g + 2 * mb;
-                    d_hi = d_lo + 1;
-                } else {
-                    d_lo = 16 * mb + g;
-                    d_hi = d_lo + 8;
+                for (int col = 0; col < 2; ++col) {
+                    float* row = red_o + (warp * kGP + 8 * nb + 2 * c + col) * kD;
+                    if constexpr (kFp8) {
+                        // dims [kD/8 g, kD/8 (g+1)): m-block mb holds dims
+                        // 2mb (accumulator col) and 2mb + 1 (col + 2)
+#pragma unroll
+                        for (int k = 0; k < kD / 32; ++k) {
+                            const uint32_t u = (kD / 32) * g + k;
+                            *reinterpret_cast<float4*>(row + 4 * (u ^ sw)) =
+                                make_float4(o[nb][2 * k][col], o[nb][2 * k][col + 2],
+                                            o[nb][2 * k + 1][col], o[nb][2 * k + 1][col + 2]);
+                        }
+                    } else {
+                        // m-block mb holds dims 16mb + g (col) and 16mb + g + 8 (col + 2)
+#pragma unroll
+                        for (int mb = 0; mb < kMB; ++mb) {
+                            const uint32_t d_lo = 16 * mb + g, d_hi = d_lo + 8;
+                            row[4 * ((d_lo >> 2) ^ sw) + (d_lo & 3)] = o[nb][mb][col];
+                            row[4 * ((d_hi >> 2) ^ sw) + (d_hi & 3)] = o[nb][mb][col + 2];
+                        }
+                    }
                 }
-                float* dst0 = red_o + (warp * kGP + 8 * nb + 2 * c) * kD;
-                float* dst1 = dst0 + kD;
-                dst0[d_lo] = o[nb][mb][0];
-                dst1[d_lo] = o[nb][mb][1];
-                dst0[d_hi] = o[nb][mb][2];
-                dst1[d_hi] = o[nb][mb][3];
-            }
+        }
         named_barrier_sync(1, kConsumerThreads);
-        for (int e = tid; e < IQ * kD; e += kConsumerThreads) {
-            const int hq = e / kD, d = e % kD;
-            const int hl = hq % G;                          // head within its KV head's group
-            const int w0 = (hq / G) * kWarpsPerHead;        // the warps that worked on it
-            float M = kNegInf;
+        // Thread -> (head, 16-byte unit of dims): per pass the consumer
+        // threads cover kConsumerThreads / (kD/4) heads.
+        {
+            constexpr int kUnits = kD / 4;
+            constexpr int kHeadsPerPass = kConsumerThreads / kUnits;
+            const int u = tid % kUnits;
+            for (int hq = tid / kUnits; hq < IQ; hq += kHeadsPerPass) {
+                const int kvh = hq / G;
+                const int hl = hq - kvh * G;                 // head within its KV head's group
+                const int r0 = kvh * kWarpsPerHead * kGP + hl;   // its row in the first warp
+                const uint32_t su = u ^ red_swizzle<kFp8, kD>((hl & 7) >> 1);
+                float M = kNegInf;
 #pragma unroll
-            for (int w = 0; w < kWarpsPerHead; ++w) M = fmaxf(M, red_m[(w0 + w) * kGP + hl]);
-            float Lsum = 0.f, O = 0.f;
+                for (int w = 0; w < kWarpsPerHead; ++w) M = fmaxf(M, red_m[r0 + w * kGP]);
+                float Lsum = 0.f;
+                float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int w = 0; w < kWarpsPerHead; ++w) {
-                const float mw = red_m[(w0 + w) * kGP + hl];
-                const float wt = (mw == kNegInf) ? 0.f : exp2f(mw - M);
-                Lsum += wt * red_l[(w0 + w) * kGP + hl];
-                O += wt * red_o[((w0 + w) * kGP + hl) * kD + d];
-            }
-            if (whole) {
-                if (poisoned) {
-                    a.out[(head0 + hq) * kD + d] = 0;
-                    if (d == 0) a.lse[head0 + hq] = kNegInf;
-                } else {
-                    const float val = O * a.v_scale / Lsum;
-                    a.out[(head0 + hq) * kD + d] = f32_to_bf16_bits(val);
-                    if (d == 0) a.lse[head0 + hq] = (M + log2f(Lsum)) * kLn2;
+                for (int w = 0; w < kWarpsPerHead; ++w) {
+                    const float mw = red_m[r0 + w * kGP];
+                    const float wt = (mw == kNegInf) ? 0.f : exp2f(mw - M);
+                    Lsum += wt * red_l[r0 + w * kGP];
+                    const float4 x = *reinterpret_cast<const float4*>(red_o + (r0 + w * kGP) * kD + 4 * su);
+                    O.x += wt * x.x;
+                    O.y += wt * x.y;
+                    O.z += wt * x.z;
+                    O.w += wt * x.w;
                 }
-            } else {
-                a.ws_o[(slot * IQ + hq) * kD + d] = poisoned ? 0.f : O * a.v_scale;
-                if (d == 0) {
-                    a.ws_ml[(slot * IQ + hq) * 2 + 0] = poisoned ? kNegInf : M;
-                    a.ws_ml[(slot * IQ + hq) * 2 + 1] = poisoned ? -1.f : Lsum;
+                const int64_t hrow = head0 + hq;
+                if (whole) {
+                    uint32_t* dst = reinterpret_cast<uint32_t*>(a.out + hrow * kD + 4 * u);
+                    if (poisoned) {
+                        dst[0] = 0u;
+                        dst[1] = 0u;
+                        if (u == 0) a.lse[hrow] = kNegInf;
+                    } else {
+                        dst[0] = pack_bf16x2(O.x * a.v_scale / Lsum, O.y * a.v_scale / Lsum);
+                        dst[1] = pack_bf16x2(O.z * a.v_scale / Lsum, O.w * a.v_scale / Lsum);
+                        if (u == 0) a.lse[hrow] = (M + log2f(Lsum)) * kLn2;
+                    }
+                } else {
+                    const int64_t r = slot * IQ + hq;
+                    const float4 val = poisoned ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                                : make_float4(O.x * a.v_scale, O.y * a.v_scale,
+                                                              O.z * a.v_scale, O.w * a.v_scale);
+                    *reinterpret_cast<float4*>(a.ws_o + r * kD + 4 * u) = val;
+                    if (u == 0)
+                        *reinterpret_cast<float2*>(a.ws_ml + r * 2) =
+                            poisoned ? make_float2(kNegInf, -1.f) : make_float2(M, Lsum);
                 }
             }
         }
@@ -780,6 +909,9 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
         if constexpr (C::kRedInStage) fence_proxy_async_smem();
         named_barrier_sync(1, kConsumerThreads);
         if (C::kRedInStage && lane == 0) mbar_arrive(&empty_bar[last_stage]);
+        if constexpr (C::kEarlyQ) aborted = next_aborted;
+        s = sn;
+        have = have_next;
     }
 }
 

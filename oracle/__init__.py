@@ -1,9 +1,10 @@
 """CPU oracle for paged FP8-KV decode attention (test infrastructure).
 
-This package wraps ``oracle.c``, a plain fp64 C implementation of the four
+This package wraps ``oracle.c``, a plain fp64 C implementation of the
 operations of the decode hot path: the page-tag integrity check, the FP8
-quantise-and-append of a new token, the BF16 -> FP8 page handoff and paged
-decode attention over an FP8 or BF16 cache.
+quantise-and-append of a new token, the BF16 -> FP8 page handoff, paged
+decode attention over an FP8 or BF16 cache, the page re-tagging helpers and
+the INT4 weight dequantisation GEMV.
 
 Only the test suite, the smoke check in ``__graft_entry__`` and the CPU
 baseline / reference arm of ``bench.py`` may import this package.  The CUDA
@@ -73,6 +74,10 @@ def _load():
             lib.orc_paged_decode_attn.argtypes = [i32, P, P, P, f32, f32, P, i32, P, i32,
                                                   i32, i32, i32, i32, i32, f32, P, P, i32,
                                                   P, P]
+            lib.orc_int4_code.argtypes = [P, i32, i32, i32]
+            lib.orc_int4_code.restype = i32
+            lib.orc_int4_unpack.argtypes = [P, i32, i32, P]
+            lib.orc_int4_gemv.argtypes = [P, P, P, i32, i32, i32, i32, P, i32, P, P]
             _lib = lib
     return _lib
 
@@ -275,3 +280,55 @@ def paged_decode_attn(q_bits, k_cache, v_cache, page_table, seq_lens, num_kv_hea
         with ThreadPoolExecutor(max_workers=len(chunks)) as ex:
             list(ex.map(run, chunks))
     return out, lse
+
+
+# --------------------------------------------------------------------------
+# INT4 weight dequantisation GEMV
+# --------------------------------------------------------------------------
+
+def int4_unpack(w_packed) -> np.ndarray:
+    """Signed codes [n][k] (int8) of a packed INT4 matrix [n][k/2]."""
+    lib = _load()
+    w_packed = _c(w_packed, np.uint8)
+    n, half = w_packed.shape
+    codes = np.empty((n, 2 * half), dtype=np.int8)
+    lib.orc_int4_unpack(_ptr(w_packed), n, 2 * half, _ptr(codes))
+    return codes
+
+
+def int4_gemv(x_bits, w_packed, scale_bits, group: int, rows=None, threads: int = 1):
+    """y = x W^T with W expanded from INT4 codes and group scales.
+
+    ``x_bits`` [B][k] bf16 bits, ``w_packed`` [n][k/2] uint8, ``scale_bits``
+    [k/group][n] bf16 bits.  Returns (y_exact fp64 [B][r], y bf16 bits
+    [B][r]) for the listed ``rows`` (default: all n, in order); ``threads``
+    > 1 splits the rows over host threads (the C call releases the GIL).
+    """
+    lib = _load()
+    x_bits = _c(x_bits, np.uint16)
+    w_packed = _c(w_packed, np.uint8)
+    scale_bits = _c(scale_bits, np.uint16)
+    B, k = x_bits.shape
+    n = w_packed.shape[0]
+    if w_packed.shape[1] * 2 != k or scale_bits.shape != (k // group, n) or k % group:
+        raise ValueError("inconsistent INT4 GEMV shapes")
+    rows = np.arange(n, dtype=np.int32) if rows is None else _c(np.asarray(rows, dtype=np.int32), np.int32)
+    y_exact = np.empty((B, rows.size), dtype=np.float64)
+    y = np.empty((B, rows.size), dtype=np.uint16)
+
+    def run(lo, hi):
+        sub = np.ascontiguousarray(rows[lo:hi])
+        ye = np.empty((B, sub.size), dtype=np.float64)
+        yb = np.empty((B, sub.size), dtype=np.uint16)
+        lib.orc_int4_gemv(_ptr(x_bits), _ptr(w_packed), _ptr(scale_bits), B, n, k, group,
+                          _ptr(sub), sub.size, _ptr(ye), _ptr(yb))
+        y_exact[:, lo:hi] = ye
+        y[:, lo:hi] = yb
+
+    if threads <= 1 or rows.size <= 1:
+        run(0, rows.size)
+    else:
+        bounds = np.linspace(0, rows.size, min(threads, rows.size) + 1).astype(int)
+        with ThreadPoolExecutor(max_workers=len(bounds) - 1) as ex:
+            list(ex.map(lambda i: run(bounds[i], bounds[i + 1]), range(len(bounds) - 1)))
+    return y_exact, y

@@ -448,3 +448,65 @@ void orc_paged_decode_attn(int32_t kv_dtype, const uint16_t* q,
         free(scores);
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* INT4 weight dequantisation GEMV (decode)                                 */
+/* ------------------------------------------------------------------------ */
+/*
+ * [T] section "压缩模型权重", [S] section "模型權重壓縮：GLM 5.2 從 705 GB
+ * 縮到 421 GB" (Table 2) and [R] section "GLM 权重压缩改变了阶段权衡": model
+ * weights are stored as 4-bit integers, streamed from memory once per
+ * generated token, and expanded back to floating point before they are
+ * multiplied.  The pages fix no format; the reading used here:
+ *   - a code is a signed 4-bit integer in two's complement, -8..7;
+ *   - row j of W (one output feature) holds k codes, two per byte: the code
+ *     of column 2i in the low nibble of byte i, column 2i+1 in the high one;
+ *   - every run of `group` consecutive columns of a row shares one bf16
+ *     scale, stored group-major: scales[i / group][j];
+ *   - w[j][i] = code * scale (exact in fp64), and
+ *     y[b][j] = bf16_rne( sum_i x[b][i] * w[j][i] ) with x in bf16.
+ */
+
+/* Code of column i of row j as a signed integer. */
+int32_t orc_int4_code(const uint8_t* w_packed, int32_t k, int32_t j, int32_t i)
+{
+    uint8_t byte = w_packed[(int64_t)j * (k / 2) + i / 2];
+    int32_t nibble = (i % 2 == 0) ? (byte & 0x0F) : (byte >> 4);
+    return nibble >= 8 ? nibble - 16 : nibble;
+}
+
+/* All codes of rows [0, n) as int8, row-major [n][k]. */
+void orc_int4_unpack(const uint8_t* w_packed, int32_t n, int32_t k, int8_t* codes)
+{
+    for (int32_t j = 0; j < n; ++j)
+        for (int32_t i = 0; i < k; ++i)
+            codes[(int64_t)j * k + i] = (int8_t)orc_int4_code(w_packed, k, j, i);
+}
+
+/*
+ * y = x W^T for the rows listed in rows[0..nrows) (all n rows in order when
+ * rows is NULL).  y_exact [batch][nrows] receives the fp64 sums, y
+ * [batch][nrows] their bf16 rounding; either may be NULL.
+ */
+void orc_int4_gemv(const uint16_t* x, const uint8_t* w_packed, const uint16_t* scales,
+                   int32_t batch, int32_t n, int32_t k, int32_t group,
+                   const int32_t* rows, int32_t nrows, double* y_exact, uint16_t* y)
+{
+    if (rows == NULL)
+        nrows = n;
+    for (int32_t r = 0; r < nrows; ++r) {
+        int32_t j = rows ? rows[r] : r;
+        for (int32_t b = 0; b < batch; ++b) {
+            double sum = 0.0;
+            for (int32_t i = 0; i < k; ++i) {
+                double scale = orc_bf16_to_double(scales[(int64_t)(i / group) * n + j]);
+                double w = (double)orc_int4_code(w_packed, k, j, i) * scale;
+                sum += orc_bf16_to_double(x[(int64_t)b * k + i]) * w;
+            }
+            if (y_exact)
+                y_exact[(int64_t)b * nrows + r] = sum;
+            if (y)
+                y[(int64_t)b * nrows + r] = orc_bf16_from_double(sum);
+        }
+    }
+}

@@ -29,6 +29,13 @@ MUTANTS = {
                                    "for (int32_t j = 0; j < used - 1; ++j) {\n                int32_t pid = page_table[(int64_t)b * max_pages + j];\n                if (pid < 0 || pid >= num_pages) {"),
     "append_slot_off_by_one": ("int32_t pos = L - 1;\n        int32_t pid = page_table[(int64_t)b * max_pages + pos / page_size];\n        if (pid < 0 || pid >= num_pages)\n            continue;\n        int32_t slot = pos % page_size;\n        for (int32_t h = 0; h < num_kv_heads; ++h) {\n            for (int32_t d = 0; d < head_dim; ++d) {\n                int64_t src = ((int64_t)b * num_kv_heads + h) * head_dim + d;\n                int64_t dst = (((int64_t)pid * num_kv_heads + h) * page_size + slot) * head_dim + d;\n                k_cache[dst] = orc_quantize_bf16",
                                "int32_t pos = L - 1;\n        int32_t pid = page_table[(int64_t)b * max_pages + pos / page_size];\n        if (pid < 0 || pid >= num_pages)\n            continue;\n        int32_t slot = (pos + 1) % page_size;\n        for (int32_t h = 0; h < num_kv_heads; ++h) {\n            for (int32_t d = 0; d < head_dim; ++d) {\n                int64_t src = ((int64_t)b * num_kv_heads + h) * head_dim + d;\n                int64_t dst = (((int64_t)pid * num_kv_heads + h) * page_size + slot) * head_dim + d;\n                k_cache[dst] = orc_quantize_bf16"),
+    "int4_nibble_order": ("int32_t nibble = (i % 2 == 0) ? (byte & 0x0F) : (byte >> 4);",
+                          "int32_t nibble = (i % 2 == 0) ? (byte >> 4) : (byte & 0x0F);"),
+    "int4_unsigned_codes": ("return nibble >= 8 ? nibble - 16 : nibble;", "return nibble;"),
+    "int4_scales_row_major": ("double scale = orc_bf16_to_double(scales[(int64_t)(i / group) * n + j]);",
+                              "double scale = orc_bf16_to_double(scales[(int64_t)j * (k / group) + i / group]);"),
+    "int4_group_off_by_one": ("double scale = orc_bf16_to_double(scales[(int64_t)(i / group) * n + j]);",
+                              "double scale = orc_bf16_to_double(scales[(int64_t)((i + 1) % k / group) * n + j]);"),
     "transposed_v_index": ("o[d] += w * kv_element(kv_dtype, v_cache, (double)v_scale, pid,\n                                           num_kv_heads, hk, page_size, t % page_size,\n                                           head_dim, d);",
                            "o[d] += w * kv_element(kv_dtype, v_cache, (double)v_scale, pid,\n                                           num_kv_heads, hk, page_size, d % page_size,\n                                           head_dim, t % head_dim);"),
 }
@@ -48,6 +55,7 @@ def test_planted_mistake_is_caught(name, tmp_path):
     env = dict(os.environ, PAGEDKV_ORACLE_LIB=str(lib))
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                         os.path.join(ROOT, "tests", "test_oracle_codec.py"),
-                        os.path.join(ROOT, "tests", "test_oracle_paths.py")],
+                        os.path.join(ROOT, "tests", "test_oracle_paths.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_int4.py")],
                        env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"planted mistake {name} passed every pin:\n{r.stdout[-2000:]}"

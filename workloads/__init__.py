@@ -265,6 +265,61 @@ def ragged_prefix(seed=5, device="cpu", batch=512, group=8, prefix_pages=64) -> 
                    notes="prefix pages shared within groups of 8")
 
 
+# --------------------------------------------------------------------------
+# INT4 weight dequantisation GEMV (decode)
+# --------------------------------------------------------------------------
+
+INT4_GROUP = 128          # columns of one row sharing a scale
+INT4_N = 32768            # output features of the synthetic projection
+INT4_K = 8192             # input features
+INT4_BATCHES = (1, 8, 16, 32, 64)   # the concurrency levels the pages tabulate
+
+
+@dataclass
+class Int4Gemv:
+    """Inputs of one decode-time INT4 GEMV y = x W^T.
+
+    ``w_packed`` holds uniformly random bytes: every byte is a valid pair of
+    signed 4-bit codes, so the codes are uniform over -8..7 without this
+    module packing anything.  Scales are bf16 values drawn log-uniformly in
+    [2^-10, 2^-4]; x ~ N(0, 1) rounded to bf16.
+    """
+    name: str
+    seed: int
+    group: int
+    x: torch.Tensor          # bf16 [B][k]
+    w_packed: torch.Tensor   # uint8 [n][k/2]
+    scales: torch.Tensor     # bf16 [k/group][n]
+
+    @property
+    def batch(self) -> int:
+        return int(self.x.shape[0])
+
+    @property
+    def n(self) -> int:
+        return int(self.w_packed.shape[0])
+
+    @property
+    def k(self) -> int:
+        return int(self.x.shape[1])
+
+
+def int4_gemv_case(batch, n=INT4_N, k=INT4_K, group=INT4_GROUP, seed=6, device="cpu",
+                   w_packed=None, scales=None) -> Int4Gemv:
+    """A seeded INT4 GEMV case.  ``w_packed``/``scales`` may be passed in to
+    share one weight matrix between several batch sizes."""
+    g = _gen(seed, device)
+    if w_packed is None:
+        w_packed = torch.randint(0, 256, (n, k // 2), generator=g, device=device,
+                                 dtype=torch.int32).to(torch.uint8)
+    if scales is None:
+        e = torch.rand((k // group, n), generator=g, device=device, dtype=torch.float32)
+        scales = torch.exp2(-10.0 + 6.0 * e).to(torch.bfloat16)
+    gx = _gen(seed * 1000 + batch, device)
+    x = _draw_q((batch, k), gx, device)
+    return Int4Gemv(f"int4_gemv_b{batch}", seed, group, x, w_packed, scales)
+
+
 def bf16_bits(t: torch.Tensor) -> np.ndarray:
     """Raw uint16 bit patterns of a bf16 tensor, on the host."""
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)

@@ -464,6 +464,9 @@ def gpu_arm(args, rank, world):
             del wlb
             torch.cuda.empty_cache()
 
+    # ---- INT4 weight dequantisation GEMV (decode), against concurrency ----
+    int4 = [] if args.no_int4 else int4_gemv_lines(args, rank, peak)
+
     line = {
         "metric": METRIC,
         "value": round(value, 1),
@@ -502,8 +505,50 @@ def gpu_arm(args, rank, world):
         "gpu_launches": 3 * args.steps,
         "clocks": clk,
         "sweep": sweep,
+        "int4_gemv": int4,
     }
     return line
+
+
+def int4_algorithmic_bytes(batch, n, k, group):
+    """Codes + scales + x + y of one GEMV call."""
+    return n * k // 2 + n * (k // group) * 2 + batch * k * 2 + batch * n * 2
+
+
+def int4_gemv_lines(args, rank, peak):
+    """One entry per concurrency level: device time of int4_dequant_gemv on
+    one synthetic [32768 x 8192] INT4 weight matrix (134 MB of codes and
+    scales, larger than L2, so no flush is needed)."""
+    import torch
+    import paged_fp8_kv_attn_b200 as pkv
+    import workloads
+    rows = []
+    base = workloads.int4_gemv_case(1, seed=replica_seed(6, rank), device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for b in workloads.INT4_BATCHES:
+        case = workloads.int4_gemv_case(b, seed=replica_seed(6, rank), device="cuda",
+                                        w_packed=base.w_packed, scales=base.scales)
+        y = torch.empty((b, case.n), dtype=torch.bfloat16, device="cuda")
+        g = _graph(lambda: pkv.int4_dequant_gemv(case.x, case.w_packed, case.scales, y,
+                                                 case.group, status=status))
+        t_med, t_mean = time_per_call(g.replay, max(args.steps, 20), args.warmup)
+        byts = int4_algorithmic_bytes(b, case.n, case.k, case.group)
+        gbs = byts / (t_med * 1e-6) / 1e9
+        rows.append({"batch": b, "us": round(t_med, 2), "us_mean": round(t_mean, 2),
+                     "gbs": round(gbs, 1), "frac_of_measured": round(gbs / peak, 4),
+                     "frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
+                     "tflops": round(2.0 * b * case.n * case.k / (t_med * 1e-6) / 1e12, 1),
+                     "tokens_per_s": round(b / (t_med * 1e-6), 1)})
+        del g, y, case
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, "int4_dequant_gemv reported an expired wait"
+    shape = {"n": base.n, "k": base.k, "group": base.group,
+             "algorithmic_bytes": "n k/2 + 2 n k/group + 2 B k + 2 B n",
+             "l2": "weights larger than L2 (no flush)",
+             "dtype": "int4 codes, bf16 scales and x, bf16 tensor-core products, f32 accumulate"}
+    del base
+    torch.cuda.empty_cache()
+    return {"shape": shape, "rows": rows}
 
 
 def pkv_status_ok(st) -> bool:
@@ -635,9 +680,11 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel-only", choices=["fp8", "bf16"], default=None,
-                    help="profiling target: run only the attention call (warmup + steps "
-                         "times) on a --batch request concurrency-sweep batch; prints nothing")
+    ap.add_argument("--no-int4", action="store_true")
+    ap.add_argument("--kernel-only", choices=["fp8", "bf16", "int4"], default=None,
+                    help="profiling target: run only the decode step (fp8/bf16) on a --batch "
+                         "request concurrency-sweep batch, or only the INT4 GEMV at --batch; "
+                         "warmup + steps times; prints nothing")
     ap.add_argument("--batch", type=int, default=16)
     args = ap.parse_args()
     if args.warmup < 3:
@@ -652,6 +699,17 @@ def main():
         return
 
     import torch
+    if args.kernel_only == "int4":
+        import paged_fp8_kv_attn_b200 as pkv
+        import workloads
+        case = workloads.int4_gemv_case(args.batch, device="cuda")
+        y = torch.empty((case.batch, case.n), dtype=torch.bfloat16, device="cuda")
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        for _ in range(args.warmup + args.steps):
+            pkv.int4_dequant_gemv(case.x, case.w_packed, case.scales, y, case.group, status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        return
     if args.kernel_only:
         import workloads
         wl = workloads.concurrency_sweep(args.batch, device="cuda")

@@ -326,6 +326,36 @@ PKV_API pkv_status paged_decode_attn_fp8_noalloc(const uint16_t* q, const uint8_
 /* Bytes of the built-in scratch used by paged_decode_attn_fp8_noalloc. */
 PKV_API size_t paged_decode_attn_fp8_noalloc_scratch_bytes(void);
 
+/*
+ * int4_dequant_gemv -- y = x W^T with W stored as 4-bit integer codes and
+ * expanded to floating point before the multiply, the decode-time use of
+ * INT4 weights ([T] "压缩模型权重": decode streams every weight once per
+ * token, so 4-bit codes cut the bytes per token; [S] "模型權重壓縮：GLM 5.2
+ * 從 705 GB 縮到 421 GB", Table 2: FP8 vs INT4 decode throughput against
+ * concurrency; [R] "GLM 权重压缩改变了阶段权衡").  The pages fix no format;
+ * this call's:
+ *   x        [batch][k] bf16 activations (16-byte aligned);
+ *   w_packed [n][k/2] bytes (16-byte aligned): byte i of row j holds the
+ *            code of w[j][2i] in its low nibble and of w[j][2i+1] in its
+ *            high nibble, each a signed two's complement integer in -8..7;
+ *   scales   [k/group_size][n] bf16 (16-byte aligned): scales[g][j] applies
+ *            to columns g*group_size .. (g+1)*group_size - 1 of row j;
+ *   y        [batch][n] bf16 (2-byte aligned), written as
+ *            y[b][j] = bf16_rne( sum_i x[b][i] * code[j][i] * scales[i/group_size][j] )
+ *            with fp32 accumulation (the codes are exact in bf16 and each
+ *            group is summed before it is scaled).
+ * Sizes: 1 <= batch <= 64, n a positive multiple of 128, k a positive
+ * multiple of 256, group_size = 128; anything else returns
+ * PKV_ERR_INVALID_ARG or PKV_ERR_UNSUPPORTED without launching.
+ * status: nullable device word; the kernel sets bit 0 if an internal bounded
+ * wait expires (never expected; y is then unspecified).  All buffers are the
+ * caller's; the call allocates nothing and is asynchronous on `stream`.
+ */
+PKV_API pkv_status int4_dequant_gemv(const uint16_t* x, const uint8_t* w_packed,
+                                     const uint16_t* scales, int32_t batch, int32_t n,
+                                     int32_t k, int32_t group_size, uint16_t* y,
+                                     uint32_t* status, void* stream);
+
 /* Message describing the last non-OK status returned on this thread. */
 PKV_API const char* pkv_last_error(void);
 

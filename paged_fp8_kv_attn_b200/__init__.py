@@ -16,6 +16,12 @@ Tensors (all on one CUDA device, contiguous):
   page_tags    [NP]            torch.int32 / uint32 view (raw 32-bit tags)
   expected     [B][MP]         same dtype as page_tags
   abort        [B]             torch.uint8
+
+INT4 weight dequantisation GEMV (int4_dequant_gemv):
+  x            [B][k]          torch.bfloat16
+  w_packed     [n][k/2]        torch.uint8   (two signed 4-bit codes per byte)
+  scales       [k/group][n]    torch.bfloat16
+  y            [B][n]          torch.bfloat16
 """
 from __future__ import annotations
 
@@ -67,6 +73,7 @@ def _load():
                                       f32, P, P, P, P, sz, i32, P],
             "paged_decode_attn_bf16": [P, P, P, P, i32, P, i32, i32, i32, i32, i32, i32, f32, P,
                                        P, P, P, sz, i32, P],
+            "int4_dequant_gemv": [P, P, P, i32, i32, i32, i32, P, P, P],
         }
         for name, args in sig.items():
             fn = getattr(lib, name)
@@ -351,3 +358,21 @@ def noalloc_scratch_bytes() -> int:
 
 def version() -> int:
     return int(_load().pkv_version())
+
+
+def int4_dequant_gemv(x, w_packed, scales, y, group_size=128, status=None, stream=None):
+    """y = x W^T with W expanded from INT4 codes and per-group bf16 scales."""
+    _need(x, torch.bfloat16, 2, "x")
+    _need(w_packed, torch.uint8, 2, "w_packed")
+    _need(scales, torch.bfloat16, 2, "scales")
+    _need(y, torch.bfloat16, 2, "y")
+    if status is not None:
+        _need(status, _TAG_DTYPES, 1, "status")
+    B, k = x.shape
+    n = w_packed.shape[0]
+    if w_packed.shape[1] * 2 != k or y.shape != (B, n) or k % group_size or \
+            scales.shape != (k // group_size, n):
+        raise ValueError("inconsistent INT4 GEMV shapes")
+    _check("int4_dequant_gemv", _load().int4_dequant_gemv(
+        _ptr(x), _ptr(w_packed), _ptr(scales), B, n, k, group_size, _ptr(y), _ptr(status),
+        _stream(stream)))

@@ -137,6 +137,24 @@ pkv_status encode_pool_map(CUtensorMap* map, const void* pool, bool fp8, int hea
     return PKV_OK;
 }
 
+// Generic 2-D map: `rows` rows of `inner` elements, rows `row_bytes` apart.
+pkv_status encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
+                     uint64_t inner, uint64_t rows, uint64_t row_bytes, uint32_t box_inner,
+                     uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+    EncodeTiledFn encode = nullptr;
+    pkv_status st = get_encoder(&encode);
+    if (st != PKV_OK) return st;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return PKV_OK;
+}
+
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 pkv_status check_common_kv(int32_t batch, int32_t num_kv_heads, int32_t head_dim,
@@ -507,6 +525,74 @@ pkv_status paged_decode_attn_bf16(const uint16_t* q, const uint16_t* k_cache,
     return attn_impl(false, q, k_cache, v_cache, 1.f, 1.f, page_table, max_pages, seq_lens, batch,
                      num_q_heads, num_kv_heads, head_dim, page_size, num_pages, sm_scale, abort,
                      out, lse, workspace, workspace_bytes, num_ctas, stream);
+}
+
+pkv_status int4_dequant_gemv(const uint16_t* x, const uint8_t* w_packed, const uint16_t* scales,
+                             int32_t batch, int32_t n, int32_t k, int32_t group_size, uint16_t* y,
+                             uint32_t* status, void* stream) {
+    if (!x || !w_packed || !scales || !y)
+        return fail(PKV_ERR_INVALID_ARG, "x, w_packed, scales and y must be non-null");
+    if (!aligned(x, 16) || !aligned(w_packed, 16) || !aligned(scales, 16) || !aligned(y, 2) ||
+        (status && !aligned(status, 4)))
+        return fail(PKV_ERR_INVALID_ARG,
+                    "misaligned pointer (x, w_packed and scales need 16 bytes, y 2, status 4)");
+    if (batch < 1 || batch > pkv::kGemvMaxBatch)
+        return fail(PKV_ERR_INVALID_ARG, "batch must be in [1, %d] (got %d)", pkv::kGemvMaxBatch,
+                    batch);
+    if (n < pkv::kGemvRows || n % pkv::kGemvRows != 0)
+        return fail(PKV_ERR_INVALID_ARG, "n must be a positive multiple of %d (got %d)",
+                    pkv::kGemvRows, n);
+    if (k < pkv::kGemvKTile || k % pkv::kGemvKTile != 0)
+        return fail(PKV_ERR_INVALID_ARG, "k must be a positive multiple of %d (got %d)",
+                    pkv::kGemvKTile, k);
+    if (group_size != pkv::kGemvGroup)
+        return fail(PKV_ERR_UNSUPPORTED, "group_size %d not supported (%d)", group_size,
+                    pkv::kGemvGroup);
+
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    const int nb = pkv::gemv_batch_blocks(batch);
+    {
+        static std::mutex m;
+        static bool ready[kMaxDevices][3] = {};
+        const int slot = nb == 1 ? 0 : (nb == 2 ? 1 : 2);
+        if (dev < 0 || dev >= kMaxDevices) return fail(PKV_ERR_UNSUPPORTED, "device %d", dev);
+        std::lock_guard<std::mutex> lock(m);
+        if (!ready[dev][slot]) {
+            e = pkv::gemv_set_smem_attr(nb);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+            ready[dev][slot] = true;
+        }
+    }
+
+    // codes: [n][k/2] bytes, 128-byte x 128-row boxes; x: [batch][k] bf16,
+    // 64-column x (8 nb)-row boxes (rows past batch read as zero); scales:
+    // [k/group][n] bf16, 128 x 2 boxes
+    CUtensorMap tw, tx, ts;
+    pkv_status st = encode_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_packed,
+                              static_cast<uint64_t>(k) / 2, static_cast<uint64_t>(n),
+                              static_cast<uint64_t>(k) / 2, pkv::kGemvKTile / 2, pkv::kGemvRows,
+                              CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != PKV_OK) return st;
+    st = encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, static_cast<uint64_t>(k),
+                   static_cast<uint64_t>(batch), static_cast<uint64_t>(k) * 2, 64, 8 * nb,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != PKV_OK) return st;
+    st = encode_2d(&ts, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, scales, static_cast<uint64_t>(n),
+                   static_cast<uint64_t>(k / group_size), static_cast<uint64_t>(n) * 2,
+                   pkv::kGemvRows, pkv::kGemvKTile / pkv::kGemvGroup, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != PKV_OK) return st;
+
+    pkv::GemvArgs a{};
+    a.y = y;
+    a.status = status;
+    a.batch = batch;
+    a.n = n;
+    a.k = k;
+    e = pkv::launch_int4_gemv(nb, as_stream(stream), tw, tx, ts, a);
+    if (e != cudaSuccess) return cuda_fail(e, "int4_dequant_gemv launch");
+    return PKV_OK;
 }
 
 }  // extern "C"

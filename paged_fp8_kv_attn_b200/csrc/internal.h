@@ -101,6 +101,30 @@ cudaError_t launch_requant(const uint16_t* src_pool, int32_t src_num_pages,
                            const int32_t* dst_pages, int32_t num_pairs, int64_t page_elems,
                            float scale, cudaStream_t stream);
 
+// INT4 weight dequantisation GEMV: CTA tile (weight rows), k-tile (columns
+// per pipeline stage), scale group and largest batch.
+constexpr int kGemvRows = 128;
+constexpr int kGemvKTile = 256;
+constexpr int kGemvGroup = 128;
+constexpr int kGemvMaxBatch = 64;
+
+struct GemvArgs {
+    uint16_t* y;          // [batch][n] bf16
+    uint32_t* status;     // nullable: bit 0 set if a bounded wait expired
+    int32_t batch;
+    int32_t n;
+    int32_t k;
+};
+
+// Batch blocks of 8 one CTA covers (1, 2 or 4; larger batches use
+// several CTAs per row tile).
+int gemv_batch_blocks(int batch);
+size_t gemv_smem_bytes(int nb);
+cudaError_t gemv_set_smem_attr(int nb);
+cudaError_t launch_int4_gemv(int nb, cudaStream_t stream, const CUtensorMap& tmap_w,
+                             const CUtensorMap& tmap_x, const CUtensorMap& tmap_s,
+                             const GemvArgs& args);
+
 // Launch configuration with the programmatic-stream-serialisation attribute.
 struct PdlLaunch {
     cudaLaunchConfig_t cfg;

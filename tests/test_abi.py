@@ -30,7 +30,8 @@ def lib():
 def test_header_declares_the_hot_path(lib):
     names = _declared_functions()
     for want in ("kv_tag_check", "kv_append_fp8", "paged_decode_attn_fp8",
-                 "paged_decode_attn_bf16", "paged_decode_attn_workspace_size", "pkv_last_error"):
+                 "paged_decode_attn_bf16", "paged_decode_attn_workspace_size", "pkv_last_error",
+                 "int4_dequant_gemv"):
         assert want in names
 
 
@@ -71,3 +72,16 @@ def test_host_validation_without_a_gpu(lib):
     assert lib.paged_decode_attn_workspace_size(0, 4, 6, 4, 64, 10) == 0
     # explicit grid: size is computable without a device
     assert lib.paged_decode_attn_workspace_size(0, 4, 64, 8, 128, 296) > 0
+
+
+def test_int4_gemv_host_validation_without_a_gpu(lib):
+    P = ctypes.c_void_p
+    # batch above 64, n not a multiple of 128, k not a multiple of 256,
+    # unsupported group size, misaligned x: all rejected before any device work
+    assert lib.int4_dequant_gemv(P(256), P(256), P(256), 65, 128, 256, 128, P(256), None, None) == 1
+    assert b"batch" in lib.pkv_last_error()
+    assert lib.int4_dequant_gemv(P(256), P(256), P(256), 4, 96, 256, 128, P(256), None, None) == 1
+    assert lib.int4_dequant_gemv(P(256), P(256), P(256), 4, 128, 320, 128, P(256), None, None) == 1
+    assert lib.int4_dequant_gemv(P(256), P(256), P(256), 4, 128, 256, 64, P(256), None, None) == 3
+    assert lib.int4_dequant_gemv(P(258), P(256), P(256), 4, 128, 256, 128, P(256), None, None) == 1
+    assert lib.int4_dequant_gemv(None, P(256), P(256), 4, 128, 256, 128, P(256), None, None) == 1

@@ -1,0 +1,123 @@
+"""INT4 weight dequantisation GEMV on the GPU against the fp64 oracle.
+
+Tolerance, from the arithmetic: the kernel's products x * code are exact in
+fp32; each 128-column group is summed in fp32 (at most 128 roundings), scaled
+once and added to the running sum (k / 128 more), so the fp32 result is
+within E = (k/128 + 130) * 2^-24 * sum_i |x_i w_i| of the exact sum; the
+bf16 output adds at most 2^-9 of its magnitude.  The test allows
+2^-8 |y| + 4 E (a factor 4 for the tensor cores' accumulation order).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_fp8_kv_attn_b200 as pkv
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+def _abs_weights(case):
+    codes = oracle.int4_unpack(case.w_packed.cpu().numpy()).astype(np.float64)
+    s = oracle.bf16_to_double(workloads.bf16_bits(case.scales))          # [k/g][n]
+    return np.abs(codes) * np.repeat(s.T, case.group, axis=1)           # |w| [n][k]
+
+
+def run_gpu(case, y=None):
+    y = torch.full((case.batch, case.n), float("nan"), dtype=torch.bfloat16, device="cuda") \
+        if y is None else y
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pkv.int4_dequant_gemv(case.x, case.w_packed, case.scales, y, case.group, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return y
+
+
+def compare(case, y_gpu, rows=None):
+    xb = workloads.bf16_bits(case.x)
+    sb = workloads.bf16_bits(case.scales)
+    w = case.w_packed.cpu().numpy()
+    y_exact, _ = oracle.int4_gemv(xb, w, sb, case.group, rows=rows, threads=8)
+    absw = _abs_weights(case) if rows is None else _abs_weights(case)[rows]
+    mag = np.abs(oracle.bf16_to_double(xb)) @ absw.T                    # sum |x w|
+    got = oracle.bf16_to_double(workloads.bf16_bits(y_gpu.cpu()))
+    if rows is not None:
+        got = got[:, rows]
+    E = (case.k / 128 + 130) * 2.0 ** -24 * mag
+    tol = 2.0 ** -8 * np.abs(y_exact) + 4 * E
+    err = np.abs(got - y_exact)
+    bad = ~(err <= tol)
+    assert not bad.any(), (f"{bad.sum()} of {bad.size} outside tolerance; worst "
+                           f"err {err.max():.3e} at {np.unravel_index(np.argmax(err - tol), err.shape)}")
+
+
+@pytest.mark.parametrize("batch,n,k", [(1, 128, 256), (3, 256, 512), (8, 128, 1024),
+                                       (9, 384, 256), (16, 256, 768), (17, 128, 512),
+                                       (32, 256, 1024), (33, 128, 256), (64, 256, 512)])
+def test_small_cases_every_output(batch, n, k):
+    case = workloads.int4_gemv_case(batch, n=n, k=k, seed=7, device="cuda")
+    compare(case, run_gpu(case))
+
+
+def test_extreme_codes_and_scales():
+    # every byte 0x88 (codes -8) and 0x77 (7) in alternate rows, scales at
+    # the ends of the bf16 exponent range a model would use
+    n, k = 256, 512
+    case = workloads.int4_gemv_case(5, n=n, k=k, seed=8, device="cuda")
+    case.w_packed[0::2] = 0x88
+    case.w_packed[1::2] = 0x77
+    case.scales[0::2] = 2.0 ** -14
+    case.scales[1::2] = 2.0 ** 6
+    compare(case, run_gpu(case))
+
+
+def test_one_hot_x_reads_weights_exactly():
+    n, k = 128, 256
+    case = workloads.int4_gemv_case(8, n=n, k=k, seed=9, device="cuda")
+    cols = [0, 1, 15, 16, 127, 128, 200, 255]
+    case.x.zero_()
+    for b, i in enumerate(cols):
+        case.x[b, i] = 1.0
+    y = run_gpu(case)
+    codes = oracle.int4_unpack(case.w_packed.cpu().numpy())
+    s = oracle.bf16_to_double(workloads.bf16_bits(case.scales))
+    want = np.stack([codes[:, i] * s[i // 128] for i in cols])
+    assert np.array_equal(oracle.bf16_to_double(workloads.bf16_bits(y.cpu())),
+                          oracle.bf16_to_double(oracle.bf16_from_double(want)))
+
+
+@pytest.mark.parametrize("batch", workloads.INT4_BATCHES)
+def test_full_size_sampled_rows(batch):
+    """The benchmark's shape (n = 32768, k = 8192): 48 sampled rows against
+    the oracle, and every output finite."""
+    case = workloads.int4_gemv_case(batch, device="cuda")
+    y = run_gpu(case)
+    assert torch.isfinite(y.float()).all()
+    rng = np.random.default_rng(batch)
+    rows = np.unique(np.concatenate([[0, 127, 128, case.n - 1],
+                                     rng.integers(0, case.n, 44)])).astype(np.int32)
+    compare(case, y, rows=rows)
+
+
+def test_batch_slices_are_independent():
+    # batch 64 runs as two 32-row slices: each row of y must equal the same
+    # row computed alone
+    case = workloads.int4_gemv_case(64, n=256, k=512, seed=10, device="cuda")
+    y = run_gpu(case)
+    for b in (0, 31, 32, 63):
+        one = workloads.Int4Gemv("one", 0, case.group, case.x[b:b + 1].contiguous(),
+                                 case.w_packed, case.scales)
+        y1 = run_gpu(one)
+        assert torch.equal(y1[0], y[b])
+
+
+def test_stream_ordering_and_reuse():
+    s = torch.cuda.Stream()
+    case = workloads.int4_gemv_case(4, n=128, k=256, seed=11, device="cuda")
+    y = torch.empty((4, 128), dtype=torch.bfloat16, device="cuda")
+    with torch.cuda.stream(s):
+        for _ in range(3):
+            pkv.int4_dequant_gemv(case.x, case.w_packed, case.scales, y)
+    s.synchronize()
+    compare(case, y)

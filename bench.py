@@ -527,9 +527,9 @@ def int4_gemv_lines(args, rank, peak):
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     for b in workloads.INT4_BATCHES:
         case = workloads.int4_gemv_case(b, seed=replica_seed(6, rank), device="cuda",
-                                        w_packed=base.w_packed, scales=base.scales)
+                                        w_tiles=base.w_tiles, scales=base.scales)
         y = torch.empty((b, case.n), dtype=torch.bfloat16, device="cuda")
-        g = _graph(lambda: pkv.int4_dequant_gemv(case.x, case.w_packed, case.scales, y,
+        g = _graph(lambda: pkv.int4_dequant_gemv(case.x, case.w_tiles, case.scales, y,
                                                  case.group, status=status))
         t_med, t_mean = time_per_call(g.replay, max(args.steps, 20), args.warmup)
         byts = int4_algorithmic_bytes(b, case.n, case.k, case.group)
@@ -706,7 +706,7 @@ def main():
         y = torch.empty((case.batch, case.n), dtype=torch.bfloat16, device="cuda")
         status = torch.zeros(1, dtype=torch.int32, device="cuda")
         for _ in range(args.warmup + args.steps):
-            pkv.int4_dequant_gemv(case.x, case.w_packed, case.scales, y, case.group, status=status)
+            pkv.int4_dequant_gemv(case.x, case.w_tiles, case.scales, y, case.group, status=status)
         torch.cuda.synchronize()
         assert int(status.item()) == 0
         return

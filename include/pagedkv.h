@@ -334,16 +334,22 @@ PKV_API size_t paged_decode_attn_fp8_noalloc_scratch_bytes(void);
  * 從 705 GB 縮到 421 GB", Table 2: FP8 vs INT4 decode throughput against
  * concurrency; [R] "GLM 权重压缩改变了阶段权衡").  The pages fix no format;
  * this call's:
- *   x        [batch][k] bf16 activations (16-byte aligned);
- *   w_packed [n][k/2] bytes (16-byte aligned): byte i of row j holds the
- *            code of w[j][2i] in its low nibble and of w[j][2i+1] in its
- *            high nibble, each a signed two's complement integer in -8..7;
- *   scales   [k/group_size][n] bf16 (16-byte aligned): scales[g][j] applies
- *            to columns g*group_size .. (g+1)*group_size - 1 of row j;
- *   y        [batch][n] bf16 (2-byte aligned), written as
- *            y[b][j] = bf16_rne( sum_i x[b][i] * code[j][i] * scales[i/group_size][j] )
- *            with fp32 accumulation (the codes are exact in bf16 and each
- *            group is summed before it is scaled).
+ *   x       [batch][k] bf16 activations (16-byte aligned);
+ *   w_tiles n * k / 2 bytes (16-byte aligned) of signed two's complement
+ *           4-bit codes (-8..7) in tiles of 128 rows x 256 columns: tile
+ *           (r, t), rows 128r.. and columns 256t.., is 16384 bytes at byte
+ *           (r * (k/256) + t) * 16384; inside it row j's 128 bytes start at
+ *           (j mod 128) * 128, and byte b holds column 256t + 2b in its low
+ *           nibble and 256t + 2b + 1 in its high nibble (each tile is one
+ *           contiguous read; a row-major [n][k/2] matrix m is tiled by
+ *           m.reshape(n/128, 128, k/256, 128).transpose(0, 2, 1, 3));
+ *   scales  n * k / group_size bf16 (16-byte aligned): the scale of rows
+ *           128r.. for columns g*group_size.. is the 128-value run starting
+ *           at element (r * (k/group_size) + g) * 128, one value per row;
+ *   y       [batch][n] bf16 (2-byte aligned), written as
+ *           y[b][j] = bf16_rne( sum_i x[b][i] * code(j, i) * scale(j, i / group_size) )
+ *           with fp32 accumulation (the codes are exact in bf16 and each
+ *           group is summed before it is scaled).
  * Sizes: 1 <= batch <= 64, n a positive multiple of 128, k a positive
  * multiple of 256, group_size = 128; anything else returns
  * PKV_ERR_INVALID_ARG or PKV_ERR_UNSUPPORTED without launching.
@@ -351,7 +357,7 @@ PKV_API size_t paged_decode_attn_fp8_noalloc_scratch_bytes(void);
  * wait expires (never expected; y is then unspecified).  All buffers are the
  * caller's; the call allocates nothing and is asynchronous on `stream`.
  */
-PKV_API pkv_status int4_dequant_gemv(const uint16_t* x, const uint8_t* w_packed,
+PKV_API pkv_status int4_dequant_gemv(const uint16_t* x, const uint8_t* w_tiles,
                                      const uint16_t* scales, int32_t batch, int32_t n,
                                      int32_t k, int32_t group_size, uint16_t* y,
                                      uint32_t* status, void* stream);

@@ -76,6 +76,8 @@ def _load():
                                                   P, P]
             lib.orc_int4_code.argtypes = [P, i32, i32, i32]
             lib.orc_int4_code.restype = i32
+            lib.orc_int4_scale.argtypes = [P, i32, i32, i32, i32]
+            lib.orc_int4_scale.restype = ctypes.c_double
             lib.orc_int4_unpack.argtypes = [P, i32, i32, P]
             lib.orc_int4_gemv.argtypes = [P, P, P, i32, i32, i32, i32, P, i32, P, P]
             _lib = lib
@@ -286,31 +288,42 @@ def paged_decode_attn(q_bits, k_cache, v_cache, page_table, seq_lens, num_kv_hea
 # INT4 weight dequantisation GEMV
 # --------------------------------------------------------------------------
 
-def int4_unpack(w_packed) -> np.ndarray:
-    """Signed codes [n][k] (int8) of a packed INT4 matrix [n][k/2]."""
+def int4_unpack(w_tiles, n: int, k: int) -> np.ndarray:
+    """Signed codes [n][k] (int8) of a tiled INT4 matrix (n * k / 2 bytes)."""
     lib = _load()
-    w_packed = _c(w_packed, np.uint8)
-    n, half = w_packed.shape
-    codes = np.empty((n, 2 * half), dtype=np.int8)
-    lib.orc_int4_unpack(_ptr(w_packed), n, 2 * half, _ptr(codes))
+    w_tiles = _c(w_tiles, np.uint8)
+    if w_tiles.size * 2 != n * k:
+        raise ValueError("w_tiles must hold n * k / 2 bytes")
+    codes = np.empty((n, k), dtype=np.int8)
+    lib.orc_int4_unpack(_ptr(w_tiles), n, k, _ptr(codes))
     return codes
 
 
-def int4_gemv(x_bits, w_packed, scale_bits, group: int, rows=None, threads: int = 1):
-    """y = x W^T with W expanded from INT4 codes and group scales.
+def int4_scales(scale_bits, n: int, k: int, group: int) -> np.ndarray:
+    """fp64 scale of every (row, group): [n][k/group]."""
+    lib = _load()
+    scale_bits = _c(scale_bits, np.uint16)
+    if scale_bits.size != n * (k // group):
+        raise ValueError("scales must hold n * k / group values")
+    return np.array([[lib.orc_int4_scale(_ptr(scale_bits), k, group, j, g * group)
+                      for g in range(k // group)] for j in range(n)], dtype=np.float64)
 
-    ``x_bits`` [B][k] bf16 bits, ``w_packed`` [n][k/2] uint8, ``scale_bits``
-    [k/group][n] bf16 bits.  Returns (y_exact fp64 [B][r], y bf16 bits
-    [B][r]) for the listed ``rows`` (default: all n, in order); ``threads``
-    > 1 splits the rows over host threads (the C call releases the GIL).
+
+def int4_gemv(x_bits, w_tiles, scale_bits, n: int, group: int, rows=None, threads: int = 1):
+    """y = x W^T with W expanded from tiled INT4 codes and group scales.
+
+    ``x_bits`` [B][k] bf16 bits, ``w_tiles`` the n * k / 2 code bytes in the
+    tiled layout, ``scale_bits`` the n * k / group bf16 scale bits.  Returns
+    (y_exact fp64 [B][r], y bf16 bits [B][r]) for the listed ``rows``
+    (default: all n, in order); ``threads`` > 1 splits the rows over host
+    threads (the C call releases the GIL).
     """
     lib = _load()
     x_bits = _c(x_bits, np.uint16)
-    w_packed = _c(w_packed, np.uint8)
+    w_tiles = _c(w_tiles, np.uint8)
     scale_bits = _c(scale_bits, np.uint16)
     B, k = x_bits.shape
-    n = w_packed.shape[0]
-    if w_packed.shape[1] * 2 != k or scale_bits.shape != (k // group, n) or k % group:
+    if w_tiles.size * 2 != n * k or scale_bits.size * group != n * k or k % group:
         raise ValueError("inconsistent INT4 GEMV shapes")
     rows = np.arange(n, dtype=np.int32) if rows is None else _c(np.asarray(rows, dtype=np.int32), np.int32)
     y_exact = np.empty((B, rows.size), dtype=np.float64)
@@ -320,7 +333,7 @@ def int4_gemv(x_bits, w_packed, scale_bits, group: int, rows=None, threads: int 
         sub = np.ascontiguousarray(rows[lo:hi])
         ye = np.empty((B, sub.size), dtype=np.float64)
         yb = np.empty((B, sub.size), dtype=np.uint16)
-        lib.orc_int4_gemv(_ptr(x_bits), _ptr(w_packed), _ptr(scale_bits), B, n, k, group,
+        lib.orc_int4_gemv(_ptr(x_bits), _ptr(w_tiles), _ptr(scale_bits), B, n, k, group,
                           _ptr(sub), sub.size, _ptr(ye), _ptr(yb))
         y_exact[:, lo:hi] = ye
         y[:, lo:hi] = yb

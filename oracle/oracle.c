@@ -459,28 +459,42 @@ void orc_paged_decode_attn(int32_t kv_dtype, const uint16_t* q,
  * generated token, and expanded back to floating point before they are
  * multiplied.  The pages fix no format; the reading used here:
  *   - a code is a signed 4-bit integer in two's complement, -8..7;
- *   - row j of W (one output feature) holds k codes, two per byte: the code
- *     of column 2i in the low nibble of byte i, column 2i+1 in the high one;
+ *   - W (n rows = output features, k columns) is stored in tiles of 128 rows
+ *     x 256 columns, 16384 bytes each; tile (r, t) covers rows 128r.. and
+ *     columns 256t.. and starts at byte (r * (k/256) + t) * 16384; inside
+ *     it, row j's 128 bytes start at (j mod 128) * 128, and byte b of that
+ *     row holds column 256t + 2b in its low nibble and 256t + 2b + 1 in its
+ *     high nibble;
  *   - every run of `group` consecutive columns of a row shares one bf16
- *     scale, stored group-major: scales[i / group][j];
+ *     scale; the scales of 128-row block r and group g are 128 consecutive
+ *     values starting at element (r * (k/group) + g) * 128;
  *   - w[j][i] = code * scale (exact in fp64), and
  *     y[b][j] = bf16_rne( sum_i x[b][i] * w[j][i] ) with x in bf16.
  */
 
 /* Code of column i of row j as a signed integer. */
-int32_t orc_int4_code(const uint8_t* w_packed, int32_t k, int32_t j, int32_t i)
+int32_t orc_int4_code(const uint8_t* w_tiles, int32_t k, int32_t j, int32_t i)
 {
-    uint8_t byte = w_packed[(int64_t)j * (k / 2) + i / 2];
+    int64_t tile = (int64_t)(j / 128) * (k / 256) + i / 256;
+    int64_t at = tile * 16384 + (int64_t)(j % 128) * 128 + (i % 256) / 2;
+    uint8_t byte = w_tiles[at];
     int32_t nibble = (i % 2 == 0) ? (byte & 0x0F) : (byte >> 4);
     return nibble >= 8 ? nibble - 16 : nibble;
 }
 
+/* Scale of column i of row j. */
+double orc_int4_scale(const uint16_t* scales, int32_t k, int32_t group, int32_t j, int32_t i)
+{
+    int64_t at = ((int64_t)(j / 128) * (k / group) + i / group) * 128 + j % 128;
+    return orc_bf16_to_double(scales[at]);
+}
+
 /* All codes of rows [0, n) as int8, row-major [n][k]. */
-void orc_int4_unpack(const uint8_t* w_packed, int32_t n, int32_t k, int8_t* codes)
+void orc_int4_unpack(const uint8_t* w_tiles, int32_t n, int32_t k, int8_t* codes)
 {
     for (int32_t j = 0; j < n; ++j)
         for (int32_t i = 0; i < k; ++i)
-            codes[(int64_t)j * k + i] = (int8_t)orc_int4_code(w_packed, k, j, i);
+            codes[(int64_t)j * k + i] = (int8_t)orc_int4_code(w_tiles, k, j, i);
 }
 
 /*
@@ -488,7 +502,7 @@ void orc_int4_unpack(const uint8_t* w_packed, int32_t n, int32_t k, int8_t* code
  * rows is NULL).  y_exact [batch][nrows] receives the fp64 sums, y
  * [batch][nrows] their bf16 rounding; either may be NULL.
  */
-void orc_int4_gemv(const uint16_t* x, const uint8_t* w_packed, const uint16_t* scales,
+void orc_int4_gemv(const uint16_t* x, const uint8_t* w_tiles, const uint16_t* scales,
                    int32_t batch, int32_t n, int32_t k, int32_t group,
                    const int32_t* rows, int32_t nrows, double* y_exact, uint16_t* y)
 {
@@ -499,8 +513,7 @@ void orc_int4_gemv(const uint16_t* x, const uint8_t* w_packed, const uint16_t* s
         for (int32_t b = 0; b < batch; ++b) {
             double sum = 0.0;
             for (int32_t i = 0; i < k; ++i) {
-                double scale = orc_bf16_to_double(scales[(int64_t)(i / group) * n + j]);
-                double w = (double)orc_int4_code(w_packed, k, j, i) * scale;
+                double w = (double)orc_int4_code(w_tiles, k, j, i) * orc_int4_scale(scales, k, group, j, i);
                 sum += orc_bf16_to_double(x[(int64_t)b * k + i]) * w;
             }
             if (y_exact)

@@ -18,10 +18,10 @@ Tensors (all on one CUDA device, contiguous):
   abort        [B]             torch.uint8
 
 INT4 weight dequantisation GEMV (int4_dequant_gemv):
-  x            [B][k]          torch.bfloat16
-  w_packed     [n][k/2]        torch.uint8   (two signed 4-bit codes per byte)
-  scales       [k/group][n]    torch.bfloat16
-  y            [B][n]          torch.bfloat16
+  x            [B][k]                      torch.bfloat16
+  w_tiles      [n/128][k/256][128][128]    torch.uint8 (two signed 4-bit codes per byte)
+  scales       [n/128][k/group][128]       torch.bfloat16
+  y            [B][n]                      torch.bfloat16
 """
 from __future__ import annotations
 
@@ -360,19 +360,34 @@ def version() -> int:
     return int(_load().pkv_version())
 
 
-def int4_dequant_gemv(x, w_packed, scales, y, group_size=128, status=None, stream=None):
-    """y = x W^T with W expanded from INT4 codes and per-group bf16 scales."""
+def int4_dequant_gemv(x, w_tiles, scales, y, group_size=128, status=None, stream=None):
+    """y = x W^T with W expanded from tiled INT4 codes and per-group bf16
+    scales (layouts in include/pagedkv.h; int4_tile_layout builds them)."""
     _need(x, torch.bfloat16, 2, "x")
-    _need(w_packed, torch.uint8, 2, "w_packed")
-    _need(scales, torch.bfloat16, 2, "scales")
+    _need(w_tiles, torch.uint8, 4, "w_tiles")
+    _need(scales, torch.bfloat16, 3, "scales")
     _need(y, torch.bfloat16, 2, "y")
     if status is not None:
         _need(status, _TAG_DTYPES, 1, "status")
     B, k = x.shape
-    n = w_packed.shape[0]
-    if w_packed.shape[1] * 2 != k or y.shape != (B, n) or k % group_size or \
-            scales.shape != (k // group_size, n):
+    n = w_tiles.shape[0] * 128
+    if tuple(w_tiles.shape) != (n // 128, k // 256, 128, 128) or y.shape != (B, n) or \
+            k % group_size or tuple(scales.shape) != (n // 128, k // group_size, 128):
         raise ValueError("inconsistent INT4 GEMV shapes")
     _check("int4_dequant_gemv", _load().int4_dequant_gemv(
-        _ptr(x), _ptr(w_packed), _ptr(scales), B, n, k, group_size, _ptr(y), _ptr(status),
+        _ptr(x), _ptr(w_tiles), _ptr(scales), B, n, k, group_size, _ptr(y), _ptr(status),
         _stream(stream)))
+
+
+def int4_tile_layout(w_rowmajor, scales_rows, group_size=128):
+    """Re-lay a row-major code matrix [n][k/2] (uint8, two codes per byte,
+    even column in the low nibble) and row-wise scales [n][k/group_size]
+    into the tiled layouts int4_dequant_gemv reads.  Pure data movement
+    (a reshape and a transpose), done once per weight matrix."""
+    n, half = w_rowmajor.shape
+    k = 2 * half
+    if n % 128 or k % 256 or tuple(scales_rows.shape) != (n, k // group_size):
+        raise ValueError("n must be a multiple of 128, k of 256, scales [n][k/group]")
+    tiles = w_rowmajor.reshape(n // 128, 128, k // 256, 128).permute(0, 2, 1, 3).contiguous()
+    sc = scales_rows.reshape(n // 128, 128, k // group_size).permute(0, 2, 1).contiguous()
+    return tiles, sc

@@ -527,15 +527,15 @@ pkv_status paged_decode_attn_bf16(const uint16_t* q, const uint16_t* k_cache,
                      out, lse, workspace, workspace_bytes, num_ctas, stream);
 }
 
-pkv_status int4_dequant_gemv(const uint16_t* x, const uint8_t* w_packed, const uint16_t* scales,
+pkv_status int4_dequant_gemv(const uint16_t* x, const uint8_t* w_tiles, const uint16_t* scales,
                              int32_t batch, int32_t n, int32_t k, int32_t group_size, uint16_t* y,
                              uint32_t* status, void* stream) {
-    if (!x || !w_packed || !scales || !y)
-        return fail(PKV_ERR_INVALID_ARG, "x, w_packed, scales and y must be non-null");
-    if (!aligned(x, 16) || !aligned(w_packed, 16) || !aligned(scales, 16) || !aligned(y, 2) ||
+    if (!x || !w_tiles || !scales || !y)
+        return fail(PKV_ERR_INVALID_ARG, "x, w_tiles, scales and y must be non-null");
+    if (!aligned(x, 16) || !aligned(w_tiles, 16) || !aligned(scales, 16) || !aligned(y, 2) ||
         (status && !aligned(status, 4)))
         return fail(PKV_ERR_INVALID_ARG,
-                    "misaligned pointer (x, w_packed and scales need 16 bytes, y 2, status 4)");
+                    "misaligned pointer (x, w_tiles and scales need 16 bytes, y 2, status 4)");
     if (batch < 1 || batch > pkv::kGemvMaxBatch)
         return fail(PKV_ERR_INVALID_ARG, "batch must be in [1, %d] (got %d)", pkv::kGemvMaxBatch,
                     batch);
@@ -566,22 +566,23 @@ pkv_status int4_dequant_gemv(const uint16_t* x, const uint8_t* w_packed, const u
         }
     }
 
-    // codes: [n][k/2] bytes, 128-byte x 128-row boxes; x: [batch][k] bf16,
-    // 64-column x (8 nb)-row boxes (rows past batch read as zero); scales:
-    // [k/group][n] bf16, 128 x 2 boxes
+    // codes: the tiles as rows of 128 bytes (one box = one 128 x 256 tile);
+    // x: [batch][k] bf16, 64-column x (8 nb)-row boxes (rows past batch read
+    // as zero); scales: rows of 128 (one row block, one group), 2-row boxes
     CUtensorMap tw, tx, ts;
-    pkv_status st = encode_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_packed,
-                              static_cast<uint64_t>(k) / 2, static_cast<uint64_t>(n),
-                              static_cast<uint64_t>(k) / 2, pkv::kGemvKTile / 2, pkv::kGemvRows,
+    pkv_status st = encode_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_tiles, pkv::kGemvKTile / 2,
+                              static_cast<uint64_t>(n) * (k / pkv::kGemvKTile),
+                              pkv::kGemvKTile / 2, pkv::kGemvKTile / 2, pkv::kGemvRows,
                               CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != PKV_OK) return st;
     st = encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, static_cast<uint64_t>(k),
                    static_cast<uint64_t>(batch), static_cast<uint64_t>(k) * 2, 64, 8 * nb,
                    CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != PKV_OK) return st;
-    st = encode_2d(&ts, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, scales, static_cast<uint64_t>(n),
-                   static_cast<uint64_t>(k / group_size), static_cast<uint64_t>(n) * 2,
-                   pkv::kGemvRows, pkv::kGemvKTile / pkv::kGemvGroup, CU_TENSOR_MAP_SWIZZLE_NONE);
+    st = encode_2d(&ts, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, scales, pkv::kGemvRows,
+                   static_cast<uint64_t>(n / pkv::kGemvRows) * (k / group_size),
+                   pkv::kGemvRows * 2, pkv::kGemvRows, pkv::kGemvKTile / pkv::kGemvGroup,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
     if (st != PKV_OK) return st;
 
     pkv::GemvArgs a{};

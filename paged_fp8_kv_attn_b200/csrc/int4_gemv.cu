@@ -7,14 +7,18 @@
 // "模型權重壓縮：GLM 5.2 從 705 GB 縮到 421 GB" (Table 2: FP8 vs INT4 weight
 // decode throughput against concurrency); remio.ai commentary, section
 // "GLM 权重压缩改变了阶段权衡".  The pages fix no format; the one here:
-// signed two's complement codes, two per byte with the even column in the
-// low nibble, one bf16 scale per 128-column group of a row stored
-// [k/128][n], y[b][j] = bf16(sum_i x[b][i] * q[j][i] * scale[i/128][j]).
+// signed two's complement codes in tiles of 128 rows x 256 columns (16 KiB,
+// row-major, two codes per byte with the even column in the low nibble;
+// tiles ordered by row block, then column block), one bf16 scale per
+// 128-column group of a row stored [row block][group][row in block], and
+// y[b][j] = bf16(sum_i x[b][i] * q[j][i] * scale(j, i / 128)).  The tiles
+// make each pipeline stage one contiguous 16 KiB read: with row-major rows
+// a stage would gather 128 separate 128-byte pieces 4 KiB apart.
 //
 // Design:
 //  * One CTA per 128 weight rows (output features) and slice of up to 32
 //    batch rows (two slices above 32, as adjacent CTAs that read the same
-//    codes at the same time, the second copy from L2).  Warp 4 (the producer)
+//    codes at the same time, the second copy from L2).  The last warp (the producer)
 //    streams the rows' codes (16 KiB per 256 columns), the matching x
 //    columns of the whole batch and the two groups' scales into a ring of
 //    shared-memory stages with 2-D TMA loads on full/empty mbarriers; the
@@ -43,7 +47,7 @@
 
 namespace pkv {
 
-template <int kNB>
+template <int kNB, int kCW>
 struct GemvCfg {
     static constexpr int kWBytes = kGemvRows * kGemvKTile / 2;     // codes of a stage: 16 KiB
     static constexpr int kXBoxBytes = kNB * 8 * 128;               // x rows x 64 columns (bf16)
@@ -52,11 +56,12 @@ struct GemvCfg {
     static constexpr int kStageBytes = (kWBytes + kXBytes + kSBytes + 1023) / 1024 * 1024;
     // two CTAs per SM in every variant; the depth fills what is left
     static constexpr int kStages = kNB <= 2 ? 4 : 3;
-    // m-blocks of a warp processed together (sharing x fragments)
-    static constexpr int kMbTogether = 2;
+    static constexpr int kThreads = 32 * (kCW + 1);                // consumer warps + producer
+    static constexpr int kMB = kGemvRows / 16 / kCW;               // m16 blocks per consumer warp
     static constexpr int kBarOff = kStages * kStageBytes;
     static constexpr int kSmemBytes = kBarOff + 2 * kStages * 8 + 16 + 1024;   // + alignment slack
     static_assert(kNB == 1 || kNB == 2 || kNB == 4, "batch blocks");
+    static_assert(kCW == 4 || kCW == 8, "consumer warps");
 };
 
 // bf16x2 (q_lo, q_hi) of the two codes in byte `b` of w (w4 = w >> 4).
@@ -80,12 +85,13 @@ __device__ __forceinline__ bool gemv_wait(uint64_t* bar, uint32_t parity, volati
     return false;
 }
 
-template <int kNB>
-__global__ void __launch_bounds__(kAttnThreads, 2)
+template <int kNB, int kCW>
+__global__ void __launch_bounds__(GemvCfg<kNB, kCW>::kThreads, 2)
 int4_gemv_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                  const __grid_constant__ CUtensorMap tmap_s, const GemvArgs a) {
-    using C = GemvCfg<kNB>;
+    using C = GemvCfg<kNB, kCW>;
     constexpr int S = C::kStages;
+    constexpr int MB = C::kMB;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -107,34 +113,36 @@ int4_gemv_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full_bar[s], 1);
-            mbar_init(&empty_bar[s], 4);
+            mbar_init(&empty_bar[s], kCW);
         }
         *failed = 0;
         fence_barrier_init();
     }
     __syncthreads();
 
-    if (warp == 4) {
+    if (warp == kCW) {
         // ================= producer =================
         if (lane == 0) {
             prefetch_tensormap(&tmap_w);
             prefetch_tensormap(&tmap_x);
             prefetch_tensormap(&tmap_s);
             // the weights are not written by preceding kernels: start early
-            for (int t = 0; t < S && t < KT; ++t) tma_prefetch_l2_2d(&tmap_w, t * (kGemvKTile / 2), row0);
+            const int tile0 = (row0 / kGemvRows) * KT;     // first code tile of the row block
+            for (int t = 0; t < S && t < KT; ++t) tma_prefetch_l2_2d(&tmap_w, 0, (tile0 + t) * kGemvRows);
             grid_dependency_wait();
             for (int t = 0; t < KT; ++t) {
                 const int stage = t % S;
                 if (t >= S) gemv_wait(&empty_bar[stage], ((t / S) + 1) & 1, failed, a.status);
                 const uint32_t base = smem_addr(smem + stage * C::kStageBytes);
                 mbar_arrive_expect_tx(&full_bar[stage], C::kWBytes + C::kXBytes + C::kSBytes);
-                tma_load_2d(base, &tmap_w, t * (kGemvKTile / 2), row0, &full_bar[stage]);
+                tma_load_2d(base, &tmap_w, 0, (tile0 + t) * kGemvRows, &full_bar[stage]);
 #pragma unroll
                 for (int i = 0; i < kGemvKTile / 64; ++i)
                     tma_load_2d(base + C::kWBytes + i * C::kXBoxBytes, &tmap_x, t * kGemvKTile + i * 64, b0,
                                 &full_bar[stage]);
-                tma_load_2d(base + C::kWBytes + C::kXBytes, &tmap_s, row0,
-                            t * (kGemvKTile / kGemvGroup), &full_bar[stage]);
+                tma_load_2d(base + C::kWBytes + C::kXBytes, &tmap_s, 0,
+                            (row0 / kGemvRows) * (a.k / kGemvGroup) + t * (kGemvKTile / kGemvGroup),
+                            &full_bar[stage]);
             }
         }
         return;
@@ -144,11 +152,11 @@ int4_gemv_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
     const int g = lane >> 2;
     const int c = lane & 3;
     const int pg = ((g & 3) << 1) | (g >> 2);      // tile row of MMA row g in its 8-row half
-    const int rw = 32 * warp;                        // first tile row of this warp
+    const int rw = 16 * MB * warp;                   // first tile row of this warp
 
-    float acc[2][kNB][4];
+    float acc[MB][kNB][4];
 #pragma unroll
-    for (int mb = 0; mb < 2; ++mb)
+    for (int mb = 0; mb < MB; ++mb)
 #pragma unroll
         for (int nb = 0; nb < kNB; ++nb) acc[mb][nb][0] = acc[mb][nb][1] = acc[mb][nb][2] = acc[mb][nb][3] = 0.f;
 
@@ -161,68 +169,61 @@ int4_gemv_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
             reinterpret_cast<const uint16_t*>(smem + stage * C::kStageBytes + C::kWBytes + C::kXBytes);
 #pragma unroll
         for (int grp = 0; grp < kGemvKTile / kGemvGroup; ++grp) {
-            // m-blocks handled together (x fragments shared) or one after
-            // the other (half the live accumulators, x read twice)
+            float gacc[MB][kNB][4];
 #pragma unroll
-            for (int mo = 0; mo < 2 / C::kMbTogether; ++mo) {
-                constexpr int MT = C::kMbTogether;
-                float gacc[MT][kNB][4];
+            for (int m = 0; m < MB; ++m)
 #pragma unroll
-                for (int m = 0; m < MT; ++m)
+                for (int nb = 0; nb < kNB; ++nb)
+                    gacc[m][nb][0] = gacc[m][nb][1] = gacc[m][nb][2] = gacc[m][nb][3] = 0.f;
 #pragma unroll
-                    for (int nb = 0; nb < kNB; ++nb)
-                        gacc[m][nb][0] = gacc[m][nb][1] = gacc[m][nb][2] = gacc[m][nb][3] = 0.f;
+            for (int bb = 0; bb < kGemvGroup / 64; ++bb) {
+                const int blk = grp * (kGemvGroup / 64) + bb;       // 64-column block of the tile
+                // codes: 8 bytes (columns 64 blk + 16c .. +15) of rows rlo and rlo + 8
+                uint2 wl[MB], wh[MB];
 #pragma unroll
-                for (int bb = 0; bb < kGemvGroup / 64; ++bb) {
-                    const int blk = grp * (kGemvGroup / 64) + bb;       // 64-column block of the tile
-                    // codes: 8 bytes (columns 64 blk + 16c .. +15) of rows rlo and rlo + 8
-                    uint2 wl[MT], wh[MT];
+                for (int m = 0; m < MB; ++m) {
+                    const int rlo = rw + 16 * m + pg;
+                    wl[m] = lds64(wbase + swz<128, 128>(rlo, 32 * blk + 8 * c));
+                    wh[m] = lds64(wbase + swz<128, 128>(rlo + 8, 32 * blk + 8 * c));
+                }
+                const uint32_t xbox = xbase + blk * C::kXBoxBytes;
+                uint4 xv[kNB];
 #pragma unroll
-                    for (int m = 0; m < MT; ++m) {
-                        const int rlo = rw + 16 * (mo * MT + m) + pg;
-                        wl[m] = lds64(wbase + swz<128, 128>(rlo, 32 * blk + 8 * c));
-                        wh[m] = lds64(wbase + swz<128, 128>(rlo + 8, 32 * blk + 8 * c));
+                for (int j = 0; j < 4; ++j) {
+                    // x: columns 64 blk + 16c + 8 (j/2) .. +7 of batch row 8 nb + g
+                    if ((j & 1) == 0) {
+#pragma unroll
+                        for (int nb = 0; nb < kNB; ++nb)
+                            xv[nb] = lds128(xbox + swz<128, 128>(8 * nb + g, 32 * c + 16 * (j >> 1)));
                     }
-                    const uint32_t xbox = xbase + blk * C::kXBoxBytes;
-                    uint4 xv[kNB];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        // x: columns 64 blk + 16c + 8 (j/2) .. +7 of batch row 8 nb + g
-                        if ((j & 1) == 0) {
+                    for (int m = 0; m < MB; ++m) {
+                        const uint32_t lo = (j < 2) ? wl[m].x : wl[m].y;
+                        const uint32_t hi = (j < 2) ? wh[m].x : wh[m].y;
+                        const uint32_t by = 2 * (j & 1);
+                        const uint32_t a0 = int4x2_to_bf16x2(lo, lo >> 4, by);
+                        const uint32_t a2 = int4x2_to_bf16x2(lo, lo >> 4, by + 1);
+                        const uint32_t a1 = int4x2_to_bf16x2(hi, hi >> 4, by);
+                        const uint32_t a3 = int4x2_to_bf16x2(hi, hi >> 4, by + 1);
 #pragma unroll
-                            for (int nb = 0; nb < kNB; ++nb)
-                                xv[nb] = lds128(xbox + swz<128, 128>(8 * nb + g, 32 * c + 16 * (j >> 1)));
-                        }
-#pragma unroll
-                        for (int m = 0; m < MT; ++m) {
-                            const uint32_t lo = (j < 2) ? wl[m].x : wl[m].y;
-                            const uint32_t hi = (j < 2) ? wh[m].x : wh[m].y;
-                            const uint32_t by = 2 * (j & 1);
-                            const uint32_t a0 = int4x2_to_bf16x2(lo, lo >> 4, by);
-                            const uint32_t a2 = int4x2_to_bf16x2(lo, lo >> 4, by + 1);
-                            const uint32_t a1 = int4x2_to_bf16x2(hi, hi >> 4, by);
-                            const uint32_t a3 = int4x2_to_bf16x2(hi, hi >> 4, by + 1);
-#pragma unroll
-                            for (int nb = 0; nb < kNB; ++nb)
-                                mma_bf16(gacc[m][nb], a0, a1, a2, a3, (j & 1) ? xv[nb].z : xv[nb].x,
-                                         (j & 1) ? xv[nb].w : xv[nb].y);
-                        }
+                        for (int nb = 0; nb < kNB; ++nb)
+                            mma_bf16(gacc[m][nb], a0, a1, a2, a3, (j & 1) ? xv[nb].z : xv[nb].x,
+                                     (j & 1) ? xv[nb].w : xv[nb].y);
                     }
                 }
-                // scale the group's sums by the rows' scales (rows rlo: c0, c1; rlo + 8: c2, c3)
+            }
+            // scale the group's sums by the rows' scales (rows rlo: c0, c1; rlo + 8: c2, c3)
 #pragma unroll
-                for (int m = 0; m < MT; ++m) {
-                    const int mb = mo * MT + m;
-                    const int rlo = rw + 16 * mb + pg;
-                    const float s_lo = bf16_bits_to_f32(sbase[grp * kGemvRows + rlo]);
-                    const float s_hi = bf16_bits_to_f32(sbase[grp * kGemvRows + rlo + 8]);
+            for (int m = 0; m < MB; ++m) {
+                const int rlo = rw + 16 * m + pg;
+                const float s_lo = bf16_bits_to_f32(sbase[grp * kGemvRows + rlo]);
+                const float s_hi = bf16_bits_to_f32(sbase[grp * kGemvRows + rlo + 8]);
 #pragma unroll
-                    for (int nb = 0; nb < kNB; ++nb) {
-                        acc[mb][nb][0] = fmaf(s_lo, gacc[m][nb][0], acc[mb][nb][0]);
-                        acc[mb][nb][1] = fmaf(s_lo, gacc[m][nb][1], acc[mb][nb][1]);
-                        acc[mb][nb][2] = fmaf(s_hi, gacc[m][nb][2], acc[mb][nb][2]);
-                        acc[mb][nb][3] = fmaf(s_hi, gacc[m][nb][3], acc[mb][nb][3]);
-                    }
+                for (int nb = 0; nb < kNB; ++nb) {
+                    acc[m][nb][0] = fmaf(s_lo, gacc[m][nb][0], acc[m][nb][0]);
+                    acc[m][nb][1] = fmaf(s_lo, gacc[m][nb][1], acc[m][nb][1]);
+                    acc[m][nb][2] = fmaf(s_hi, gacc[m][nb][2], acc[m][nb][2]);
+                    acc[m][nb][3] = fmaf(s_hi, gacc[m][nb][3], acc[m][nb][3]);
                 }
             }
         }
@@ -233,18 +234,26 @@ int4_gemv_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
     // y[b][n]: accumulator (row, col) = (weight row, batch row)
     grid_dependency_wait();
 #pragma unroll
-    for (int mb = 0; mb < 2; ++mb) {
-        const int nlo = row0 + rw + 16 * mb + pg;
+    for (int m = 0; m < MB; ++m) {
+        const int nlo = row0 + rw + 16 * m + pg;
 #pragma unroll
         for (int nb = 0; nb < kNB; ++nb)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int b = b0 + 8 * nb + 2 * c + (i & 1);
                 const int nn = nlo + ((i & 2) ? 8 : 0);
-                if (b < a.batch) a.y[static_cast<int64_t>(b) * a.n + nn] = f32_to_bf16_bits(acc[mb][nb][i]);
+                if (b < a.batch) a.y[static_cast<int64_t>(b) * a.n + nn] = f32_to_bf16_bits(acc[m][nb][i]);
             }
     }
 }
+
+// Consumer warps per CTA: four warps of 32 rows (eight warps of 16 rows
+// measured the same on B200 and spill at batch 32).
+template <int kNB>
+struct GemvVariant {
+    static constexpr int kCW = 4;
+    using Cfg = GemvCfg<kNB, kCW>;
+};
 
 int gemv_batch_blocks(int batch) {
     const int nb = (batch + 7) / 8;
@@ -260,16 +269,17 @@ int gemv_batch_blocks(int batch) {
     }
 
 cudaError_t gemv_set_smem_attr(int nb) {
-    PKV_GEMV_DISPATCH(nb, return cudaFuncSetAttribute(int4_gemv_kernel<NB>,
-                                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                      GemvCfg<NB>::kSmemBytes))
+    PKV_GEMV_DISPATCH(nb, return cudaFuncSetAttribute(
+                              int4_gemv_kernel<NB, GemvVariant<NB>::kCW>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              GemvVariant<NB>::Cfg::kSmemBytes))
 }
 
 size_t gemv_smem_bytes(int nb) {
     switch (nb) {
-        case 1: return GemvCfg<1>::kSmemBytes;
-        case 2: return GemvCfg<2>::kSmemBytes;
-        case 4: return GemvCfg<4>::kSmemBytes;
+        case 1: return GemvVariant<1>::Cfg::kSmemBytes;
+        case 2: return GemvVariant<2>::Cfg::kSmemBytes;
+        case 4: return GemvVariant<4>::Cfg::kSmemBytes;
         default: return 0;
     }
 }
@@ -277,9 +287,12 @@ size_t gemv_smem_bytes(int nb) {
 cudaError_t launch_int4_gemv(int nb, cudaStream_t stream, const CUtensorMap& tmap_w,
                              const CUtensorMap& tmap_x, const CUtensorMap& tmap_s, const GemvArgs& args) {
     const int slices = (args.batch + 8 * nb - 1) / (8 * nb);
-    PdlLaunch l(dim3(args.n / kGemvRows * slices), dim3(kAttnThreads), gemv_smem_bytes(nb), stream);
-    PKV_GEMV_DISPATCH(nb, return cudaLaunchKernelEx(&l.cfg, int4_gemv_kernel<NB>, tmap_w, tmap_x,
-                                                   tmap_s, args))
+    PKV_GEMV_DISPATCH(nb, {
+        PdlLaunch l(dim3(args.n / kGemvRows * slices), dim3(GemvVariant<NB>::Cfg::kThreads),
+                    GemvVariant<NB>::Cfg::kSmemBytes, stream);
+        return cudaLaunchKernelEx(&l.cfg, int4_gemv_kernel<NB, GemvVariant<NB>::kCW>, tmap_w, tmap_x,
+                                  tmap_s, args);
+    })
 }
 
 }  // namespace pkv

@@ -18,17 +18,26 @@ import workloads
 pytestmark = pytest.mark.gpu
 
 
-def _abs_weights(case):
-    codes = oracle.int4_unpack(case.w_packed.cpu().numpy()).astype(np.float64)
-    s = oracle.bf16_to_double(workloads.bf16_bits(case.scales))          # [k/g][n]
-    return np.abs(codes) * np.repeat(s.T, case.group, axis=1)           # |w| [n][k]
+def _abs_weights(case, rows=None):
+    """|w| [rows][k] for the tolerance bound, read straight from the tiled
+    bytes with numpy (only the listed rows, so the full shape stays small)."""
+    rows = np.arange(case.n) if rows is None else np.asarray(rows)
+    tiles = case.w_tiles.cpu().numpy()                      # [n/128][k/256][128][128]
+    sc = oracle.bf16_to_double(workloads.bf16_bits(case.scales))   # [n/128][k/g][128]
+    by = tiles[rows // 128, :, rows % 128, :].reshape(rows.size, -1).astype(np.int16)
+    codes = np.empty((rows.size, case.k), dtype=np.int16)
+    codes[:, 0::2] = by & 0xF
+    codes[:, 1::2] = by >> 4
+    codes = np.where(codes >= 8, codes - 16, codes)
+    s = sc[rows // 128, :, rows % 128]                      # [rows][k/g]
+    return np.abs(codes) * np.repeat(s, case.group, axis=1)
 
 
 def run_gpu(case, y=None):
     y = torch.full((case.batch, case.n), float("nan"), dtype=torch.bfloat16, device="cuda") \
         if y is None else y
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    pkv.int4_dequant_gemv(case.x, case.w_packed, case.scales, y, case.group, status=status)
+    pkv.int4_dequant_gemv(case.x, case.w_tiles, case.scales, y, case.group, status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     return y
@@ -37,9 +46,9 @@ def run_gpu(case, y=None):
 def compare(case, y_gpu, rows=None):
     xb = workloads.bf16_bits(case.x)
     sb = workloads.bf16_bits(case.scales)
-    w = case.w_packed.cpu().numpy()
-    y_exact, _ = oracle.int4_gemv(xb, w, sb, case.group, rows=rows, threads=8)
-    absw = _abs_weights(case) if rows is None else _abs_weights(case)[rows]
+    w = case.w_tiles.cpu().numpy()
+    y_exact, _ = oracle.int4_gemv(xb, w, sb, case.n, case.group, rows=rows, threads=8)
+    absw = _abs_weights(case, rows)
     mag = np.abs(oracle.bf16_to_double(xb)) @ absw.T                    # sum |x w|
     got = oracle.bf16_to_double(workloads.bf16_bits(y_gpu.cpu()))
     if rows is not None:
@@ -65,10 +74,10 @@ def test_extreme_codes_and_scales():
     # the ends of the bf16 exponent range a model would use
     n, k = 256, 512
     case = workloads.int4_gemv_case(5, n=n, k=k, seed=8, device="cuda")
-    case.w_packed[0::2] = 0x88
-    case.w_packed[1::2] = 0x77
-    case.scales[0::2] = 2.0 ** -14
-    case.scales[1::2] = 2.0 ** 6
+    case.w_tiles[:, :, 0::2] = 0x88
+    case.w_tiles[:, :, 1::2] = 0x77
+    case.scales[:, :, 0::2] = 2.0 ** -14
+    case.scales[:, :, 1::2] = 2.0 ** 6
     compare(case, run_gpu(case))
 
 
@@ -80,9 +89,9 @@ def test_one_hot_x_reads_weights_exactly():
     for b, i in enumerate(cols):
         case.x[b, i] = 1.0
     y = run_gpu(case)
-    codes = oracle.int4_unpack(case.w_packed.cpu().numpy())
-    s = oracle.bf16_to_double(workloads.bf16_bits(case.scales))
-    want = np.stack([codes[:, i] * s[i // 128] for i in cols])
+    codes = oracle.int4_unpack(case.w_tiles.cpu().numpy(), n, k)
+    s = oracle.int4_scales(workloads.bf16_bits(case.scales), n, k, case.group)   # [n][k/g]
+    want = np.stack([codes[:, i] * s[:, i // 128] for i in cols])
     assert np.array_equal(oracle.bf16_to_double(workloads.bf16_bits(y.cpu())),
                           oracle.bf16_to_double(oracle.bf16_from_double(want)))
 
@@ -107,7 +116,7 @@ def test_batch_slices_are_independent():
     y = run_gpu(case)
     for b in (0, 31, 32, 63):
         one = workloads.Int4Gemv("one", 0, case.group, case.x[b:b + 1].contiguous(),
-                                 case.w_packed, case.scales)
+                                 case.w_tiles, case.scales)
         y1 = run_gpu(one)
         assert torch.equal(y1[0], y[b])
 
@@ -118,6 +127,20 @@ def test_stream_ordering_and_reuse():
     y = torch.empty((4, 128), dtype=torch.bfloat16, device="cuda")
     with torch.cuda.stream(s):
         for _ in range(3):
-            pkv.int4_dequant_gemv(case.x, case.w_packed, case.scales, y)
+            pkv.int4_dequant_gemv(case.x, case.w_tiles, case.scales, y)
     s.synchronize()
     compare(case, y)
+
+
+def test_tile_layout_helper_matches_the_format():
+    """int4_tile_layout re-lays row-major codes and row-wise scales into the
+    layout whose definition the oracle reads."""
+    rng = np.random.default_rng(12)
+    n, k = 256, 512
+    codes = rng.integers(-8, 8, size=(n, k), dtype=np.int8)
+    c = codes.astype(np.int16) & 0xF
+    rowmajor = torch.from_numpy((c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)).cuda()
+    s = torch.exp2(torch.from_numpy(rng.integers(-9, -3, size=(n, k // 128)).astype(np.float32)))
+    tiles, sc = pkv.int4_tile_layout(rowmajor, s.to(torch.bfloat16).cuda())
+    assert np.array_equal(oracle.int4_unpack(tiles.cpu().numpy(), n, k), codes)
+    assert np.array_equal(oracle.int4_scales(workloads.bf16_bits(sc), n, k, 128), s.double().numpy())

@@ -3,13 +3,15 @@ not come from the oracle itself.
 
 Format reading (the pages say only that weights are 4-bit integers expanded
 to floating point before the multiply: "压缩模型权重" on the first-party
-post, "模型權重壓縮" on the siami.tw editorial): signed two's complement codes,
-two per byte with the even column in the low nibble, one bf16 scale per
-group of 128 columns of a row stored group-major [k/group][n].
+post, "模型權重壓縮" on the siami.tw editorial): signed two's complement codes
+in tiles of 128 rows x 256 columns (row-major inside a tile, two codes per
+byte with the even column in the low nibble, tiles ordered by row block then
+column block); one bf16 scale per group of 128 columns of a row, stored as
+[row block][group][row in block].
 
 - Two's complement by hand: the nibble 0x8 is -8, 0xF is -1, 0x7 is 7.
-- Packing round trip: codes packed by numpy bit operations written here
-  unpack to the same codes.
+- Layout round trip: codes and scales laid out by numpy reshapes written
+  here unpack to the same values.
 - y equals numpy's fp64 matrix product of x and the expanded weights (a
   library routine), and its bf16 output is the RNE rounding of that.
 - Closed forms: all-ones codes with unit scales sum x; a one-hot x reads one
@@ -25,10 +27,18 @@ import workloads
 GROUP = 128
 
 
-def pack(codes: np.ndarray) -> np.ndarray:
-    """Independent packer: low nibble = even column, two's complement."""
+def tile_codes(codes: np.ndarray) -> np.ndarray:
+    """Independent packer: row-major nibble pairs, then 128 x 128-byte tiles."""
+    n, k = codes.shape
     c = codes.astype(np.int16) & 0xF
-    return (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)
+    rowmajor = (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)          # [n][k/2]
+    return rowmajor.reshape(n // 128, 128, k // 256, 128).transpose(0, 2, 1, 3).copy()
+
+
+def tile_scales(scales: np.ndarray) -> np.ndarray:
+    """[n][k/group] -> [n/128][k/group][128]."""
+    n, groups = scales.shape
+    return scales.reshape(n // 128, 128, groups).transpose(0, 2, 1).copy()
 
 
 def bf16_bits_of(values: np.ndarray) -> np.ndarray:
@@ -39,73 +49,77 @@ def bf16_bits_of(values: np.ndarray) -> np.ndarray:
     return (bits >> 16).astype(np.uint16)
 
 
-def expand(codes: np.ndarray, scale_bits: np.ndarray, group: int) -> np.ndarray:
-    scales = oracle.bf16_to_double(scale_bits)            # [k/group][n]
-    return codes.astype(np.float64) * np.repeat(scales.T, group, axis=1)
+def expand(codes: np.ndarray, scales: np.ndarray, group: int) -> np.ndarray:
+    """w [n][k] from codes [n][k] and logical scales [n][k/group] (fp64)."""
+    return codes.astype(np.float64) * np.repeat(scales, group, axis=1)
 
 
 def test_twos_complement_nibbles():
-    # byte 0x8F: column 0 = 0xF = -1, column 1 = 0x8 = -8; byte 0x70: 0, 7
-    w = np.array([[0x8F, 0x70, 0x21, 0xE9]], dtype=np.uint8)
-    assert oracle.int4_unpack(w).tolist() == [[-1, -8, 0, 7, 1, 2, -7, -2]]
+    # tile row 0 starts with bytes 0x8F, 0x70, 0x21, 0xE9
+    w = np.zeros((1, 1, 128, 128), dtype=np.uint8)
+    w[0, 0, 0, :4] = [0x8F, 0x70, 0x21, 0xE9]
+    assert oracle.int4_unpack(w, 128, 256)[0, :8].tolist() == [-1, -8, 0, 7, 1, 2, -7, -2]
 
 
-def test_pack_round_trip_all_codes():
+def test_layout_round_trip():
     rng = np.random.default_rng(0)
-    codes = rng.integers(-8, 8, size=(37, 256), dtype=np.int8)
+    n, k = 256, 768
+    codes = rng.integers(-8, 8, size=(n, k), dtype=np.int8)
     codes[0, :16] = np.arange(-8, 8)
-    assert np.array_equal(oracle.int4_unpack(pack(codes)), codes)
+    assert np.array_equal(oracle.int4_unpack(tile_codes(codes), n, k), codes)
+    s = np.exp2(rng.integers(-12, 0, size=(n, k // GROUP))).astype(np.float32)
+    got = oracle.int4_scales(bf16_bits_of(tile_scales(s)), n, k, GROUP)
+    assert np.array_equal(got, s.astype(np.float64))
 
 
-@pytest.mark.parametrize("batch,n,k", [(1, 16, 256), (5, 40, 512), (8, 3, 1024)])
+@pytest.mark.parametrize("batch,n,k", [(1, 128, 256), (5, 256, 512), (8, 128, 1024)])
 def test_matches_numpy_fp64_product(batch, n, k):
     rng = np.random.default_rng(batch * 1000 + n)
     codes = rng.integers(-8, 8, size=(n, k), dtype=np.int8)
     x = rng.standard_normal((batch, k)).astype(np.float32)
     x_bits = (x.view(np.uint32) >> 16).astype(np.uint16)   # truncated to bf16
-    s = np.exp2(rng.integers(-12, -2, size=(k // GROUP, n))).astype(np.float32) * \
-        (1 + rng.integers(0, 128, size=(k // GROUP, n)) / 128.0).astype(np.float32)
-    s_bits = bf16_bits_of(s)
-    y_exact, y = oracle.int4_gemv(x_bits, pack(codes), s_bits, GROUP)
-    ref = oracle.bf16_to_double(x_bits) @ expand(codes, s_bits, GROUP).T
+    s = np.exp2(rng.integers(-12, -2, size=(n, k // GROUP))).astype(np.float32) * \
+        (1 + rng.integers(0, 128, size=(n, k // GROUP)) / 128.0).astype(np.float32)
+    y_exact, y = oracle.int4_gemv(x_bits, tile_codes(codes), bf16_bits_of(tile_scales(s)), n, GROUP)
+    ref = oracle.bf16_to_double(x_bits) @ expand(codes, s.astype(np.float64), GROUP).T
     np.testing.assert_allclose(y_exact, ref, rtol=1e-12, atol=1e-12)
     assert np.array_equal(y, oracle.bf16_from_double(y_exact))
 
 
 def test_all_ones_sum_x():
     rng = np.random.default_rng(3)
-    n, k = 8, 512
+    n, k = 128, 512
     x_bits = bf16_bits_of(rng.integers(-64, 64, size=(2, k)).astype(np.float32))
-    w = np.full((n, k // 2), 0x11, dtype=np.uint8)
-    s_bits = bf16_bits_of(np.ones((k // GROUP, n), dtype=np.float32))
-    y_exact, _ = oracle.int4_gemv(x_bits, w, s_bits, GROUP)
+    w = np.full(n * k // 2, 0x11, dtype=np.uint8)
+    s_bits = bf16_bits_of(np.ones(n * k // GROUP, dtype=np.float32))
+    y_exact, _ = oracle.int4_gemv(x_bits, w, s_bits, n, GROUP)
     expect = oracle.bf16_to_double(x_bits).sum(axis=1)
     assert np.array_equal(y_exact, np.repeat(expect[:, None], n, axis=1))
 
 
 def test_one_hot_reads_one_weight():
     rng = np.random.default_rng(4)
-    n, k = 24, 384
+    n, k = 256, 512
     codes = rng.integers(-8, 8, size=(n, k), dtype=np.int8)
-    s_bits = bf16_bits_of(np.exp2(rng.integers(-8, 0, size=(k // GROUP, n))).astype(np.float32))
-    cols = [0, 1, 127, 128, 255, 383]
+    s = np.exp2(rng.integers(-8, 0, size=(n, k // GROUP))).astype(np.float32)
+    cols = [0, 1, 127, 128, 255, 256, 383, 511]
     x = np.zeros((len(cols), k), dtype=np.float32)
     x[np.arange(len(cols)), cols] = 1.0
-    y_exact, _ = oracle.int4_gemv(bf16_bits_of(x), pack(codes), s_bits, GROUP)
-    scales = oracle.bf16_to_double(s_bits)
+    y_exact, _ = oracle.int4_gemv(bf16_bits_of(x), tile_codes(codes), bf16_bits_of(tile_scales(s)),
+                                  n, GROUP)
     for b, i in enumerate(cols):
-        assert np.array_equal(y_exact[b], codes[:, i] * scales[i // GROUP, :])
+        assert np.array_equal(y_exact[b], codes[:, i] * s[:, i // GROUP].astype(np.float64))
 
 
 def test_group_scale_linearity():
     rng = np.random.default_rng(5)
-    n, k = 6, 512
+    n, k = 128, 512
     codes = rng.integers(-8, 8, size=(n, k), dtype=np.int8)
     x_bits = bf16_bits_of(rng.integers(-16, 16, size=(1, k)).astype(np.float32))
-    s = np.ones((k // GROUP, n), dtype=np.float32)
-    y1, _ = oracle.int4_gemv(x_bits, pack(codes), bf16_bits_of(s), GROUP)
-    s[2, :] = 2.0
-    y2, _ = oracle.int4_gemv(x_bits, pack(codes), bf16_bits_of(s), GROUP)
+    s = np.ones((n, k // GROUP), dtype=np.float32)
+    y1, _ = oracle.int4_gemv(x_bits, tile_codes(codes), bf16_bits_of(tile_scales(s)), n, GROUP)
+    s[:, 2] = 2.0
+    y2, _ = oracle.int4_gemv(x_bits, tile_codes(codes), bf16_bits_of(tile_scales(s)), n, GROUP)
     xs = oracle.bf16_to_double(x_bits)[0, 2 * GROUP:3 * GROUP]
     part = codes[:, 2 * GROUP:3 * GROUP].astype(np.float64) @ xs
     assert np.array_equal(y2[0] - y1[0], part)
@@ -115,8 +129,8 @@ def test_row_subset_matches_full():
     case = workloads.int4_gemv_case(3, n=256, k=512)
     xb = workloads.bf16_bits(case.x)
     sb = workloads.bf16_bits(case.scales)
-    w = case.w_packed.numpy()
-    full_e, full = oracle.int4_gemv(xb, w, sb, case.group)
+    w = case.w_tiles.numpy()
+    full_e, full = oracle.int4_gemv(xb, w, sb, case.n, case.group)
     rows = np.array([255, 0, 17, 128], dtype=np.int32)
-    sub_e, sub = oracle.int4_gemv(xb, w, sb, case.group, rows=rows, threads=2)
+    sub_e, sub = oracle.int4_gemv(xb, w, sb, case.n, case.group, rows=rows, threads=2)
     assert np.array_equal(sub_e, full_e[:, rows]) and np.array_equal(sub, full[:, rows])

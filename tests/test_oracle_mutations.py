@@ -32,10 +32,12 @@ MUTANTS = {
     "int4_nibble_order": ("int32_t nibble = (i % 2 == 0) ? (byte & 0x0F) : (byte >> 4);",
                           "int32_t nibble = (i % 2 == 0) ? (byte >> 4) : (byte & 0x0F);"),
     "int4_unsigned_codes": ("return nibble >= 8 ? nibble - 16 : nibble;", "return nibble;"),
-    "int4_scales_row_major": ("double scale = orc_bf16_to_double(scales[(int64_t)(i / group) * n + j]);",
-                              "double scale = orc_bf16_to_double(scales[(int64_t)j * (k / group) + i / group]);"),
-    "int4_group_off_by_one": ("double scale = orc_bf16_to_double(scales[(int64_t)(i / group) * n + j]);",
-                              "double scale = orc_bf16_to_double(scales[(int64_t)((i + 1) % k / group) * n + j]);"),
+    "int4_tile_transposed": ("int64_t at = tile * 16384 + (int64_t)(j % 128) * 128 + (i % 256) / 2;",
+                             "int64_t at = tile * 16384 + (int64_t)((i % 256) / 2) * 128 + j % 128;"),
+    "int4_scale_group_major": ("int64_t at = ((int64_t)(j / 128) * (k / group) + i / group) * 128 + j % 128;",
+                               "int64_t at = (int64_t)j * (k / group) + i / group;"),
+    "int4_group_off_by_one": ("int64_t at = ((int64_t)(j / 128) * (k / group) + i / group) * 128 + j % 128;",
+                              "int64_t at = ((int64_t)(j / 128) * (k / group) + (i + 1) % k / group) * 128 + j % 128;"),
     "transposed_v_index": ("o[d] += w * kv_element(kv_dtype, v_cache, (double)v_scale, pid,\n                                           num_kv_heads, hk, page_size, t % page_size,\n                                           head_dim, d);",
                            "o[d] += w * kv_element(kv_dtype, v_cache, (double)v_scale, pid,\n                                           num_kv_heads, hk, page_size, d % page_size,\n                                           head_dim, t % head_dim);"),
 }

@@ -279,17 +279,19 @@ INT4_BATCHES = (1, 8, 16, 32, 64)   # the concurrency levels the pages tabulate
 class Int4Gemv:
     """Inputs of one decode-time INT4 GEMV y = x W^T.
 
-    ``w_packed`` holds uniformly random bytes: every byte is a valid pair of
-    signed 4-bit codes, so the codes are uniform over -8..7 without this
-    module packing anything.  Scales are bf16 values drawn log-uniformly in
+    ``w_tiles`` holds the codes in the tiled layout ([n/128][k/256] tiles of
+    128 rows x 128 bytes); it is filled with uniformly random bytes, and
+    every byte is a valid pair of signed 4-bit codes, so the codes are
+    uniform over -8..7 and this module packs nothing.  ``scales``
+    [n/128][k/group][128] are bf16 values drawn log-uniformly in
     [2^-10, 2^-4]; x ~ N(0, 1) rounded to bf16.
     """
     name: str
     seed: int
     group: int
     x: torch.Tensor          # bf16 [B][k]
-    w_packed: torch.Tensor   # uint8 [n][k/2]
-    scales: torch.Tensor     # bf16 [k/group][n]
+    w_tiles: torch.Tensor    # uint8 [n/128][k/256][128][128]
+    scales: torch.Tensor     # bf16 [n/128][k/group][128]
 
     @property
     def batch(self) -> int:
@@ -297,7 +299,7 @@ class Int4Gemv:
 
     @property
     def n(self) -> int:
-        return int(self.w_packed.shape[0])
+        return int(self.w_tiles.shape[0]) * 128
 
     @property
     def k(self) -> int:
@@ -305,19 +307,19 @@ class Int4Gemv:
 
 
 def int4_gemv_case(batch, n=INT4_N, k=INT4_K, group=INT4_GROUP, seed=6, device="cpu",
-                   w_packed=None, scales=None) -> Int4Gemv:
-    """A seeded INT4 GEMV case.  ``w_packed``/``scales`` may be passed in to
+                   w_tiles=None, scales=None) -> Int4Gemv:
+    """A seeded INT4 GEMV case.  ``w_tiles``/``scales`` may be passed in to
     share one weight matrix between several batch sizes."""
     g = _gen(seed, device)
-    if w_packed is None:
-        w_packed = torch.randint(0, 256, (n, k // 2), generator=g, device=device,
-                                 dtype=torch.int32).to(torch.uint8)
+    if w_tiles is None:
+        w_tiles = torch.randint(0, 256, (n // 128, k // 256, 128, 128), generator=g, device=device,
+                                dtype=torch.int32).to(torch.uint8)
     if scales is None:
-        e = torch.rand((k // group, n), generator=g, device=device, dtype=torch.float32)
+        e = torch.rand((n // 128, k // group, 128), generator=g, device=device, dtype=torch.float32)
         scales = torch.exp2(-10.0 + 6.0 * e).to(torch.bfloat16)
     gx = _gen(seed * 1000 + batch, device)
     x = _draw_q((batch, k), gx, device)
-    return Int4Gemv(f"int4_gemv_b{batch}", seed, group, x, w_packed, scales)
+    return Int4Gemv(f"int4_gemv_b{batch}", seed, group, x, w_tiles, scales)
 
 
 def bf16_bits(t: torch.Tensor) -> np.ndarray:

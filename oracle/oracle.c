@@ -462,9 +462,11 @@ void orc_paged_decode_attn(int32_t kv_dtype, const uint16_t* q,
  *   - W (n rows = output features, k columns) is stored in tiles of 128 rows
  *     x 256 columns, 16384 bytes each; tile (r, t) covers rows 128r.. and
  *     columns 256t.. and starts at byte (r * (k/256) + t) * 16384; inside
- *     it, row j's 128 bytes start at (j mod 128) * 128, and byte b of that
- *     row holds column 256t + 2b in its low nibble and 256t + 2b + 1 in its
- *     high nibble;
+ *     it, row j's 128 bytes start at (j mod 128) * 128 and hold 32
+ *     little-endian 32-bit words; word w holds the 8 columns
+ *     c = 256t + 8w .. c + 7: bits 4i..4i+3 hold column c + 2i and bits
+ *     16+4i..16+4i+3 hold column c + 2i + 1 (i = 0..3), i.e. the even
+ *     columns in the low half-word and the odd ones in the high half-word;
  *   - every run of `group` consecutive columns of a row shares one bf16
  *     scale; the scales of 128-row block r and group g are 128 consecutive
  *     values starting at element (r * (k/group) + g) * 128;
@@ -476,9 +478,12 @@ void orc_paged_decode_attn(int32_t kv_dtype, const uint16_t* q,
 int32_t orc_int4_code(const uint8_t* w_tiles, int32_t k, int32_t j, int32_t i)
 {
     int64_t tile = (int64_t)(j / 128) * (k / 256) + i / 256;
-    int64_t at = tile * 16384 + (int64_t)(j % 128) * 128 + (i % 256) / 2;
-    uint8_t byte = w_tiles[at];
-    int32_t nibble = (i % 2 == 0) ? (byte & 0x0F) : (byte >> 4);
+    int64_t at = tile * 16384 + (int64_t)(j % 128) * 128 + (int64_t)((i % 256) / 8) * 4;
+    uint32_t word = (uint32_t)w_tiles[at] | ((uint32_t)w_tiles[at + 1] << 8) |
+                    ((uint32_t)w_tiles[at + 2] << 16) | ((uint32_t)w_tiles[at + 3] << 24);
+    int32_t m = i % 8;
+    int32_t bit = (m % 2 == 0) ? 4 * (m / 2) : 16 + 4 * (m / 2);
+    int32_t nibble = (int32_t)((word >> bit) & 0x0Fu);
     return nibble >= 8 ? nibble - 16 : nibble;
 }
 

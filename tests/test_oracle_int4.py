@@ -4,10 +4,11 @@ not come from the oracle itself.
 Format reading (the pages say only that weights are 4-bit integers expanded
 to floating point before the multiply: "压缩模型权重" on the first-party
 post, "模型權重壓縮" on the siami.tw editorial): signed two's complement codes
-in tiles of 128 rows x 256 columns (row-major inside a tile, two codes per
-byte with the even column in the low nibble, tiles ordered by row block then
-column block); one bf16 scale per group of 128 columns of a row, stored as
-[row block][group][row in block].
+in tiles of 128 rows x 256 columns (row-major inside a tile, tiles ordered by
+row block then column block); each little-endian 32-bit word holds 8
+consecutive columns, the even ones in nibbles 0-3 of the low half-word and
+the odd ones in nibbles 0-3 of the high half-word; one bf16 scale per group
+of 128 columns of a row, stored as [row block][group][row in block].
 
 - Two's complement by hand: the nibble 0x8 is -8, 0xF is -1, 0x7 is 7.
 - Layout round trip: codes and scales laid out by numpy reshapes written
@@ -28,10 +29,15 @@ GROUP = 128
 
 
 def tile_codes(codes: np.ndarray) -> np.ndarray:
-    """Independent packer: row-major nibble pairs, then 128 x 128-byte tiles."""
+    """Independent packer: 32-bit words of 8 columns (even columns in the low
+    half-word, odd in the high), then 128 x 128-byte tiles."""
     n, k = codes.shape
-    c = codes.astype(np.int16) & 0xF
-    rowmajor = (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)          # [n][k/2]
+    c = (codes.astype(np.int64) & 0xF).reshape(n, k // 8, 8)
+    words = np.zeros((n, k // 8), dtype=np.uint64)
+    for i in range(4):
+        words |= (c[:, :, 2 * i] << (4 * i)).astype(np.uint64)
+        words |= (c[:, :, 2 * i + 1] << (16 + 4 * i)).astype(np.uint64)
+    rowmajor = words.astype("<u4").view(np.uint8).reshape(n, k // 2)     # [n][k/2]
     return rowmajor.reshape(n // 128, 128, k // 256, 128).transpose(0, 2, 1, 3).copy()
 
 
@@ -55,10 +61,12 @@ def expand(codes: np.ndarray, scales: np.ndarray, group: int) -> np.ndarray:
 
 
 def test_twos_complement_nibbles():
-    # tile row 0 starts with bytes 0x8F, 0x70, 0x21, 0xE9
+    # tile row 0 starts with the word 0xE921708F (bytes 8F 70 21 E9): low
+    # half-word 0x708F holds columns 0, 2, 4, 6 = F, 8, 0, 7 -> -1, -8, 0, 7;
+    # high half-word 0xE921 holds columns 1, 3, 5, 7 = 1, 2, 9, E -> 1, 2, -7, -2
     w = np.zeros((1, 1, 128, 128), dtype=np.uint8)
     w[0, 0, 0, :4] = [0x8F, 0x70, 0x21, 0xE9]
-    assert oracle.int4_unpack(w, 128, 256)[0, :8].tolist() == [-1, -8, 0, 7, 1, 2, -7, -2]
+    assert oracle.int4_unpack(w, 128, 256)[0, :8].tolist() == [-1, 1, -8, 2, 0, -7, 7, -2]
 
 
 def test_layout_round_trip():

@@ -29,11 +29,13 @@ MUTANTS = {
                                    "for (int32_t j = 0; j < used - 1; ++j) {\n                int32_t pid = page_table[(int64_t)b * max_pages + j];\n                if (pid < 0 || pid >= num_pages) {"),
     "append_slot_off_by_one": ("int32_t pos = L - 1;\n        int32_t pid = page_table[(int64_t)b * max_pages + pos / page_size];\n        if (pid < 0 || pid >= num_pages)\n            continue;\n        int32_t slot = pos % page_size;\n        for (int32_t h = 0; h < num_kv_heads; ++h) {\n            for (int32_t d = 0; d < head_dim; ++d) {\n                int64_t src = ((int64_t)b * num_kv_heads + h) * head_dim + d;\n                int64_t dst = (((int64_t)pid * num_kv_heads + h) * page_size + slot) * head_dim + d;\n                k_cache[dst] = orc_quantize_bf16",
                                "int32_t pos = L - 1;\n        int32_t pid = page_table[(int64_t)b * max_pages + pos / page_size];\n        if (pid < 0 || pid >= num_pages)\n            continue;\n        int32_t slot = (pos + 1) % page_size;\n        for (int32_t h = 0; h < num_kv_heads; ++h) {\n            for (int32_t d = 0; d < head_dim; ++d) {\n                int64_t src = ((int64_t)b * num_kv_heads + h) * head_dim + d;\n                int64_t dst = (((int64_t)pid * num_kv_heads + h) * page_size + slot) * head_dim + d;\n                k_cache[dst] = orc_quantize_bf16"),
-    "int4_nibble_order": ("int32_t nibble = (i % 2 == 0) ? (byte & 0x0F) : (byte >> 4);",
-                          "int32_t nibble = (i % 2 == 0) ? (byte >> 4) : (byte & 0x0F);"),
+    "int4_nibble_order": ("int32_t bit = (m % 2 == 0) ? 4 * (m / 2) : 16 + 4 * (m / 2);",
+                          "int32_t bit = 4 * m;"),
+    "int4_word_big_endian": ("uint32_t word = (uint32_t)w_tiles[at] | ((uint32_t)w_tiles[at + 1] << 8) |",
+                             "uint32_t word = ((uint32_t)w_tiles[at] << 24) | ((uint32_t)w_tiles[at + 1] << 8) |"),
     "int4_unsigned_codes": ("return nibble >= 8 ? nibble - 16 : nibble;", "return nibble;"),
-    "int4_tile_transposed": ("int64_t at = tile * 16384 + (int64_t)(j % 128) * 128 + (i % 256) / 2;",
-                             "int64_t at = tile * 16384 + (int64_t)((i % 256) / 2) * 128 + j % 128;"),
+    "int4_tile_transposed": ("int64_t at = tile * 16384 + (int64_t)(j % 128) * 128 + (int64_t)((i % 256) / 8) * 4;",
+                             "int64_t at = tile * 16384 + (int64_t)((i % 256) / 8) * 512 + (j % 128) * 4;"),
     "int4_scale_group_major": ("int64_t at = ((int64_t)(j / 128) * (k / group) + i / group) * 128 + j % 128;",
                                "int64_t at = (int64_t)j * (k / group) + i / group;"),
     "int4_group_off_by_one": ("int64_t at = ((int64_t)(j / 128) * (k / group) + i / group) * 128 + j % 128;",

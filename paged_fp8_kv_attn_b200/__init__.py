@@ -382,12 +382,18 @@ def int4_dequant_gemv(x, w_tiles, scales, y, group_size=128, status=None, stream
 def int4_tile_layout(w_rowmajor, scales_rows, group_size=128):
     """Re-lay a row-major code matrix [n][k/2] (uint8, two codes per byte,
     even column in the low nibble) and row-wise scales [n][k/group_size]
-    into the tiled layouts int4_dequant_gemv reads.  Pure data movement
-    (a reshape and a transpose), done once per weight matrix."""
+    into the layouts int4_dequant_gemv reads: each 32-bit word of 8 columns
+    holds the even columns in its low half-word and the odd ones in its high
+    half-word, and rows are cut into 128 x 256 tiles.  Pure data movement,
+    done once per weight matrix."""
     n, half = w_rowmajor.shape
     k = 2 * half
     if n % 128 or k % 256 or tuple(scales_rows.shape) != (n, k // group_size):
         raise ValueError("n must be a multiple of 128, k of 256, scales [n][k/group]")
-    tiles = w_rowmajor.reshape(n // 128, 128, k // 256, 128).permute(0, 2, 1, 3).contiguous()
+    c = torch.stack([w_rowmajor & 0xF, w_rowmajor >> 4], dim=-1).reshape(n, k // 8, 8)
+    words = torch.stack([c[..., 0] | (c[..., 2] << 4), c[..., 4] | (c[..., 6] << 4),
+                         c[..., 1] | (c[..., 3] << 4), c[..., 5] | (c[..., 7] << 4)], dim=-1)
+    packed = words.reshape(n, half)
+    tiles = packed.reshape(n // 128, 128, k // 256, 128).permute(0, 2, 1, 3).contiguous()
     sc = scales_rows.reshape(n // 128, 128, k // group_size).permute(0, 2, 1).contiguous()
     return tiles, sc

@@ -552,22 +552,24 @@ pkv_status int4_dequant_gemv(const uint16_t* x, const uint8_t* w_tiles, const ui
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-    const int nb = pkv::gemv_batch_blocks(batch);
+    // batches up to 16 on the warp-level MMA kernel, larger ones on tcgen05
+    const bool small = batch <= pkv::kGemvMmaMaxBatch;
+    const int xrows = small ? 8 * pkv::gemv_mma_batch_blocks(batch) : pkv::gemv_batch_cols(batch);
     {
         static std::mutex m;
-        static bool ready[kMaxDevices][3] = {};
-        const int slot = nb == 1 ? 0 : (nb == 2 ? 1 : 2);
+        static bool ready[kMaxDevices][5] = {};
+        const int slot = small ? (xrows == 8 ? 0 : 1) : (xrows == 16 ? 2 : (xrows == 32 ? 3 : 4));
         if (dev < 0 || dev >= kMaxDevices) return fail(PKV_ERR_UNSUPPORTED, "device %d", dev);
         std::lock_guard<std::mutex> lock(m);
         if (!ready[dev][slot]) {
-            e = pkv::gemv_set_smem_attr(nb);
+            e = small ? pkv::gemv_mma_set_smem_attr(xrows / 8) : pkv::gemv_set_smem_attr(xrows);
             if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
             ready[dev][slot] = true;
         }
     }
 
     // codes: the tiles as rows of 128 bytes (one box = one 128 x 256 tile);
-    // x: [batch][k] bf16, 64-column x (8 nb)-row boxes (rows past batch read
+    // x: [batch][k] bf16, 64-column x xrows-row boxes (rows past batch read
     // as zero); scales: rows of 128 (one row block, one group), 2-row boxes
     CUtensorMap tw, tx, ts;
     pkv_status st = encode_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_tiles, pkv::kGemvKTile / 2,
@@ -576,7 +578,7 @@ pkv_status int4_dequant_gemv(const uint16_t* x, const uint8_t* w_tiles, const ui
                               CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != PKV_OK) return st;
     st = encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, static_cast<uint64_t>(k),
-                   static_cast<uint64_t>(batch), static_cast<uint64_t>(k) * 2, 64, 8 * nb,
+                   static_cast<uint64_t>(batch), static_cast<uint64_t>(k) * 2, 64, xrows,
                    CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != PKV_OK) return st;
     st = encode_2d(&ts, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, scales, pkv::kGemvRows,
@@ -591,7 +593,8 @@ pkv_status int4_dequant_gemv(const uint16_t* x, const uint8_t* w_tiles, const ui
     a.batch = batch;
     a.n = n;
     a.k = k;
-    e = pkv::launch_int4_gemv(nb, as_stream(stream), tw, tx, ts, a);
+    e = small ? pkv::launch_int4_gemv_mma(xrows / 8, as_stream(stream), tw, tx, ts, a)
+              : pkv::launch_int4_gemv(xrows, as_stream(stream), tw, tx, ts, a);
     if (e != cudaSuccess) return cuda_fail(e, "int4_dequant_gemv launch");
     return PKV_OK;
 }

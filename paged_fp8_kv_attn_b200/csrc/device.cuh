@@ -248,6 +248,27 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return r;
 }
 
+// bf16x2 (q_even, q_odd) of the two codes at bits 0-3 and 16-19 of v.
+__device__ __forceinline__ uint32_t int4_pair_to_bf16x2(uint32_t v) {
+    uint32_t t;   // (v & 0x000F000F) ^ 0x43084308: mantissa = nibble ^ 8 = q + 8 under 2^7
+    asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(t) : "r"(v), "r"(0x000F000Fu), "r"(0x43084308u));
+    uint32_t r;   // (136 + q) * 1 - 136, exact in bf16
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(t), "r"(0x3F803F80u), "r"(0xC308C308u));
+    return r;
+}
+
+// Bounded mbarrier wait of the GEMV kernels: after a timeout in this CTA every
+// later wait returns at once and bit 0 of *status (if given) is set.
+__device__ __forceinline__ bool gemv_wait(uint64_t* bar, uint32_t parity, volatile int* failed,
+                                          uint32_t* status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*failed) return false;
+    if (mbar_wait(bar, parity)) return true;
+    *failed = 1;
+    if (status != nullptr) atomicOr(status, 1u);
+    return false;
+}
+
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }

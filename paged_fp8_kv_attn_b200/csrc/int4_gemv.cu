@@ -8,290 +8,400 @@
 // decode throughput against concurrency); remio.ai commentary, section
 // "GLM 权重压缩改变了阶段权衡".  The pages fix no format; the one here:
 // signed two's complement codes in tiles of 128 rows x 256 columns (16 KiB,
-// row-major, two codes per byte with the even column in the low nibble;
-// tiles ordered by row block, then column block), one bf16 scale per
-// 128-column group of a row stored [row block][group][row in block], and
-// y[b][j] = bf16(sum_i x[b][i] * q[j][i] * scale(j, i / 128)).  The tiles
-// make each pipeline stage one contiguous 16 KiB read: with row-major rows
-// a stage would gather 128 separate 128-byte pieces 4 KiB apart.
+// row-major, tiles ordered by row block then column block); each 32-bit
+// word of a row holds 8 consecutive columns, the even ones in the low
+// half-word and the odd ones in the high half-word; one bf16 scale per
+// 128-column group of a row stored [row block][group][row in block]; and
+// y[b][j] = bf16(sum_i x[b][i] * q[j][i] * scale(j, i / 128)).
 //
-// Design:
-//  * One CTA per 128 weight rows (output features) and slice of up to 32
-//    batch rows (two slices above 32, as adjacent CTAs that read the same
-//    codes at the same time, the second copy from L2).  The last warp (the producer)
-//    streams the rows' codes (16 KiB per 256 columns), the matching x
-//    columns of the whole batch and the two groups' scales into a ring of
-//    shared-memory stages with 2-D TMA loads on full/empty mbarriers; the
-//    first stages' codes are prefetched into L2 before the grid-dependency
-//    wait.  Warps 0-3 each own 32 rows (two m16 blocks).
-//  * Math on tensor cores: m16n8k16 bf16 MMAs, weight rows as M, the batch
-//    as N in blocks of 8 (kNB blocks; padding rows of x are zero-filled by
-//    TMA).  A code pair becomes bf16x2 (136 + q_lo, 136 + q_hi) by moving
-//    each nibble into the low mantissa bits of 128.0 with its sign bit
-//    flipped (one PRMT + one LOP3), then (q_lo, q_hi) exactly by one bf16x2
-//    FMA with -136.  Codes are integers, so each 128-column group is
-//    accumulated unscaled in fp32 and then added to the output accumulator
-//    times the row's group scale: no bf16 rounding of q * scale.
-//  * Column order inside a 64-column block: thread c of a quad feeds MMA
-//    columns 2c, 2c+1 (and 2c+8, 2c+9) of k-step j from physical columns
-//    16c + 4j + {0, 1} ({2, 3}); the same map picks x, so every dot product
-//    is unchanged while each thread reads 8 contiguous code bytes and 32
-//    contiguous x bytes per block.
-//  * Bank conflicts: TMA writes 128-byte rows with the 128-byte swizzle
-//    (16-byte unit XOR row mod 8).  A half-warp's 8-byte code loads touch
-//    two adjacent units in each of 4 rows; MMA row g reads tile row
-//    2 (g mod 4) + g / 4 of its 8-row half, so those 4 rows have row mod 8 in
-//    {0, 2, 4, 6} (or the odd ones) and the 8 units fall in distinct banks.
+// Design (tcgen05 / tensor memory):
+//  * Used for batches above 16 (int4_gemv_mma.cu covers smaller ones).
+//  * One CTA per 128 weight rows.  Warp 4 streams, with 2-D TMA loads, the
+//    rows' codes (one contiguous 16 KiB tile per 256 columns) and the two
+//    groups' scales into one ring of shared-memory stages (lane 0), and the
+//    matching columns of x for the whole batch (zero-filled up to N = 32 or 64
+//    rows) into a second ring (lane 1); the first code tiles are
+//    prefetched into L2 before the grid-dependency wait.
+//  * Warps 0-3 convert: warp w owns rows 32 w .. 32 w + 31 (thread = row =
+//    tensor-memory lane).  Per 128-column group a thread expands its row's
+//    128 codes to bf16 in
+//    registers (per pair of columns: one shift, one LOP3 that puts the two
+//    offset-binary nibbles into the mantissas of 128.0, one bf16x2 FMA that
+//    subtracts 136) and writes them to a tensor-memory A buffer with
+//    tcgen05.st.
+//  * Warp 5 issues the tensor-core work: per group eight
+//    tcgen05.mma.kind::f16 (M = 128 rows, N = batch, K = 16) with A from
+//    tensor memory and x (B, K-major, 128-byte swizzle) straight from the
+//    TMA tile, accumulating the group's unscaled sums in a tensor-memory
+//    accumulator; tcgen05.commit signals the converter warps and, after a
+//    stage's last group, frees the stage.
+//  * A and the accumulator are double-buffered by group parity, so a group's
+//    expansion overlaps the previous group's MMAs.  Each thread reads its
+//    row of a finished group's accumulator (tcgen05.ld) and adds it times
+//    the row's group scale to fp32 registers: the codes are exact in bf16,
+//    the products exact in fp32, and nothing is rounded to bf16 before the
+//    final output.
+//  * Every mbarrier wait is bounded; the tensor memory is always freed.
 #include "device.cuh"
 #include "internal.h"
 
 namespace pkv {
 
-template <int kNB, int kCW>
+// ---------------------------------------------------------------------------
+// tcgen05 / tensor-memory primitives (cta_group::1)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t smem_dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_dst),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Arrive once on an mbarrier when every tcgen05.mma issued so far by this
+// thread has completed.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_addr(bar))
+                 : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem descriptor]^T, kind::f16.
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// 16 consecutive 32-bit columns of this thread's lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+          "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&v)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+                   "=r"(v[7])
+                 : "r"(taddr)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// Waits for this thread's tcgen05.ld and ties the loaded registers to the
+// wait, so no use of them is scheduled before it.
+template <int kLen>
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&v)[kLen]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < kLen; ++i) asm volatile("" : "+r"(v[i]));
+}
+
+// Shared-memory descriptor of a K-major operand tile written by TMA with the
+// 128-byte swizzle: rows of 128 bytes, 8-row atoms 1024 bytes apart.
+__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_byte_addr) {
+    return static_cast<uint64_t>((smem_byte_addr >> 4) & 0x3FFFu)   // start address / 16
+           | (static_cast<uint64_t>(1) << 16)                        // leading offset (unused here)
+           | (static_cast<uint64_t>(1024 >> 4) << 32)                // stride offset: 8 rows
+           | (static_cast<uint64_t>(1) << 46)                        // descriptor version
+           | (static_cast<uint64_t>(2) << 61);                       // 128-byte swizzle
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
+// K-major, M = 128, N = n.
+__host__ __device__ constexpr uint32_t mma_idesc_bf16(int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+           (static_cast<uint32_t>(128 >> 4) << 24);
+}
+
+template <int kN>
 struct GemvCfg {
-    static constexpr int kWBytes = kGemvRows * kGemvKTile / 2;     // codes of a stage: 16 KiB
-    static constexpr int kXBoxBytes = kNB * 8 * 128;               // x rows x 64 columns (bf16)
-    static constexpr int kXBytes = (kGemvKTile / 64) * kXBoxBytes;
+    // Two rings.  Code ring: a 16 KiB code tile and the two groups' scales
+    // per 256 columns, freed as soon as the converter warps hold them in
+    // registers.  x ring: the batch's 256 columns of x, freed by the MMA
+    // commit.  Splitting them keeps a code stage's lifetime short (TMA
+    // latency plus a register copy) instead of TMA + expansion + MMA.
+    static constexpr int kWBytes = kGemvRows * kGemvKTile / 2;      // 16 KiB
     static constexpr int kSBytes = (kGemvKTile / kGemvGroup) * kGemvRows * 2;
-    static constexpr int kStageBytes = (kWBytes + kXBytes + kSBytes + 1023) / 1024 * 1024;
-    // two CTAs per SM in every variant; the depth fills what is left
-    static constexpr int kStages = kNB <= 2 ? 4 : 3;
-    static constexpr int kThreads = 32 * (kCW + 1);                // consumer warps + producer
-    static constexpr int kMB = kGemvRows / 16 / kCW;               // m16 blocks per consumer warp
-    static constexpr int kBarOff = kStages * kStageBytes;
-    static constexpr int kSmemBytes = kBarOff + 2 * kStages * 8 + 16 + 1024;   // + alignment slack
-    static_assert(kNB == 1 || kNB == 2 || kNB == 4, "batch blocks");
-    static_assert(kCW == 4 || kCW == 8, "consumer warps");
+    static constexpr int kWStageBytes = (kWBytes + kSBytes + 1023) / 1024 * 1024;
+    static constexpr int kXBoxBytes = kN * 128;                     // kN rows x 64 columns (bf16)
+    static constexpr int kXStageBytes = (kGemvKTile / 64) * kXBoxBytes;
+    // two CTAs per SM; the depths fill what is left of the shared memory
+    static constexpr int kXStages = 2;
+    static constexpr int kWStages = kN == 32 ? 4 : 2;
+    static constexpr int kXOff = kWStages * kWStageBytes;
+    // converter warps: kSplit per tensor-memory lane quarter, each taking
+    // 1 / kSplit of a group's columns and of the batch columns (one per
+    // quarter measured faster than two: the MMA issue is the bottleneck);
+    // then the TMA warp and the MMA warp
+    static constexpr int kSplit = 1;
+    static constexpr int kConverters = 4 * kSplit;
+    static constexpr int kThreads = 32 * (kConverters + 2);
+    static constexpr int kPartN = kN / kSplit;                     // accumulator columns per converter
+    static constexpr int kPartUnits = 4 / kSplit;                  // 16-byte code units per group
+    static constexpr int kGroupCols = kGemvGroup / 2;              // A columns of one group (bf16x2)
+    static constexpr int kACol = 0;                                // A buffers: 2 x 64 columns
+    static constexpr int kDCol = 2 * kGroupCols;                   // accumulators: 2 x kN columns
+    static constexpr int kTmemCols = 256;
+    static constexpr int kBarOff = kXOff + kXStages * kXStageBytes;
+    static constexpr int kBars = 2 * kWStages + 2 * kXStages + 4;
+    static constexpr int kSmemBytes = kBarOff + kBars * 8 + 16 + 1024;   // + alignment slack
+    static_assert(kN == 32 || kN == 64, "batch columns");
+    static_assert(kDCol + 2 * kN <= kTmemCols, "tensor memory");
 };
 
-// bf16x2 (q_lo, q_hi) of the two codes in byte `b` of w (w4 = w >> 4).
-__device__ __forceinline__ uint32_t int4x2_to_bf16x2(uint32_t w, uint32_t w4, uint32_t b) {
-    // result byte 0 = byte b of w (low nibble q_lo), byte 2 = byte b of w4 (q_hi)
-    const uint32_t t = prmt(w, w4, b | (b << 4) | ((b + 4) << 8) | ((b + 4) << 12));
-    uint32_t v;   // (t & 0x000F000F) ^ 0x43084308: mantissa = nibble ^ 8 = q + 8 under 2^7
-    asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(v) : "r"(t), "r"(0x000F000Fu), "r"(0x43084308u));
-    uint32_t r;   // (136 + q) * 1 - 136, exact in bf16
-    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(v), "r"(0x3F803F80u), "r"(0xC308C308u));
-    return r;
-}
-
-__device__ __forceinline__ bool gemv_wait(uint64_t* bar, uint32_t parity, volatile int* failed,
-                                          uint32_t* status) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*failed) return false;
-    if (mbar_wait(bar, parity)) return true;
-    *failed = 1;
-    if (status != nullptr) atomicOr(status, 1u);
-    return false;
-}
-
-template <int kNB, int kCW>
-__global__ void __launch_bounds__(GemvCfg<kNB, kCW>::kThreads, 2)
+template <int kN>
+__global__ void __launch_bounds__(GemvCfg<kN>::kThreads, 2)
 int4_gemv_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                  const __grid_constant__ CUtensorMap tmap_s, const GemvArgs a) {
-    using C = GemvCfg<kNB, kCW>;
-    constexpr int S = C::kStages;
-    constexpr int MB = C::kMB;
+    using C = GemvCfg<kN>;
+    constexpr int SW = C::kWStages;
+    constexpr int SX = C::kXStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
-    uint64_t* empty_bar = full_bar + S;
-    volatile int* failed = reinterpret_cast<volatile int*>(empty_bar + S);
+    uint64_t* full_w = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+    uint64_t* empty_w = full_w + SW;
+    uint64_t* full_x = empty_w + SW;
+    uint64_t* empty_x = full_x + SX;
+    uint64_t* a_ready = empty_x + SX;     // [2] A buffer written (the converter warps)
+    uint64_t* d_ready = a_ready + 2;      // [2] group's MMAs complete (tcgen05.commit)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(d_ready + 2);
+    volatile int* failed = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    // CTA -> (row tile, batch slice of 8 kNB rows); the slices of one tile are
-    // adjacent CTAs, so they run together and share the tile's codes in L2
-    const int slices = (a.batch + 8 * kNB - 1) / (8 * kNB);
-    const int row0 = (blockIdx.x / slices) * kGemvRows;
-    const int b0 = (blockIdx.x % slices) * 8 * kNB;
+    const int row0 = blockIdx.x * kGemvRows;
     const int KT = a.k / kGemvKTile;
+    const int NG = KT * (kGemvKTile / kGemvGroup);    // groups
 
     launch_dependents();
     if (tid == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full_bar[s], 1);
-            mbar_init(&empty_bar[s], kCW);
+        for (int s = 0; s < SW; ++s) {
+            mbar_init(&full_w[s], 1);
+            mbar_init(&empty_w[s], C::kConverters);
+        }
+        for (int s = 0; s < SX; ++s) {
+            mbar_init(&full_x[s], 1);
+            mbar_init(&empty_x[s], 1);              // the MMA commit
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&a_ready[b], C::kConverters);
+            mbar_init(&d_ready[b], 1);
         }
         *failed = 0;
         fence_barrier_init();
     }
+    if (warp == 0) {
+        tmem_alloc(smem_addr(tmem_slot), C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
 
-    if (warp == kCW) {
-        // ================= producer =================
+    if (warp == C::kConverters) {
+        // ================= TMA producers: lane 0 codes, lane 1 x =================
         if (lane == 0) {
             prefetch_tensormap(&tmap_w);
-            prefetch_tensormap(&tmap_x);
             prefetch_tensormap(&tmap_s);
-            // the weights are not written by preceding kernels: start early
-            const int tile0 = (row0 / kGemvRows) * KT;     // first code tile of the row block
-            for (int t = 0; t < S && t < KT; ++t) tma_prefetch_l2_2d(&tmap_w, 0, (tile0 + t) * kGemvRows);
+            // the first code tiles into L2 while the preceding kernel finishes
+            const int tile0 = blockIdx.x * KT;     // first code tile of the row block
+            for (int t = 0; t < SW && t < KT; ++t) tma_prefetch_l2_2d(&tmap_w, 0, (tile0 + t) * kGemvRows);
             grid_dependency_wait();
             for (int t = 0; t < KT; ++t) {
-                const int stage = t % S;
-                if (t >= S) gemv_wait(&empty_bar[stage], ((t / S) + 1) & 1, failed, a.status);
-                const uint32_t base = smem_addr(smem + stage * C::kStageBytes);
-                mbar_arrive_expect_tx(&full_bar[stage], C::kWBytes + C::kXBytes + C::kSBytes);
-                tma_load_2d(base, &tmap_w, 0, (tile0 + t) * kGemvRows, &full_bar[stage]);
+                const int stage = t % SW;
+                if (t >= SW) gemv_wait(&empty_w[stage], ((t / SW) + 1) & 1, failed, a.status);
+                const uint32_t base = smem_addr(smem + stage * C::kWStageBytes);
+                mbar_arrive_expect_tx(&full_w[stage], C::kWBytes + C::kSBytes);
+                tma_load_2d(base, &tmap_w, 0, (tile0 + t) * kGemvRows, &full_w[stage]);
+                tma_load_2d(base + C::kWBytes, &tmap_s, 0,
+                            blockIdx.x * (a.k / kGemvGroup) + t * (kGemvKTile / kGemvGroup), &full_w[stage]);
+            }
+        } else if (lane == 1) {
+            prefetch_tensormap(&tmap_x);
+            grid_dependency_wait();
+            for (int t = 0; t < KT; ++t) {
+                const int stage = t % SX;
+                if (t >= SX) gemv_wait(&empty_x[stage], ((t / SX) + 1) & 1, failed, a.status);
+                const uint32_t base = smem_addr(smem + C::kXOff + stage * C::kXStageBytes);
+                mbar_arrive_expect_tx(&full_x[stage], C::kXStageBytes);
 #pragma unroll
                 for (int i = 0; i < kGemvKTile / 64; ++i)
-                    tma_load_2d(base + C::kWBytes + i * C::kXBoxBytes, &tmap_x, t * kGemvKTile + i * 64, b0,
-                                &full_bar[stage]);
-                tma_load_2d(base + C::kWBytes + C::kXBytes, &tmap_s, 0,
-                            (row0 / kGemvRows) * (a.k / kGemvGroup) + t * (kGemvKTile / kGemvGroup),
-                            &full_bar[stage]);
+                    tma_load_2d(base + i * C::kXBoxBytes, &tmap_x, t * kGemvKTile + i * 64, 0, &full_x[stage]);
             }
         }
-        return;
-    }
-
-    // ================= consumers =================
-    const int g = lane >> 2;
-    const int c = lane & 3;
-    const int pg = ((g & 3) << 1) | (g >> 2);      // tile row of MMA row g in its 8-row half
-    const int rw = 16 * MB * warp;                   // first tile row of this warp
-
-    float acc[MB][kNB][4];
+    } else if (warp == C::kConverters + 1) {
+        // ================= MMA issuer =================
+        if (lane == 0) {
+            constexpr uint32_t idesc = mma_idesc_bf16(kN);
+            for (int t = 0; t < KT; ++t) {
+                const int stage = t % SX;
+                gemv_wait(&full_x[stage], (t / SX) & 1, failed, a.status);
+                const uint32_t xaddr = smem_addr(smem + C::kXOff + stage * C::kXStageBytes);
 #pragma unroll
-    for (int mb = 0; mb < MB; ++mb)
+                for (int grp = 0; grp < kGemvKTile / kGemvGroup; ++grp) {
+                    const int g = t * (kGemvKTile / kGemvGroup) + grp;
+                    const int b = g & 1;
+                    gemv_wait(&a_ready[b], (g >> 1) & 1, failed, a.status);
+                    tc_fence_after();
 #pragma unroll
-        for (int nb = 0; nb < kNB; ++nb) acc[mb][nb][0] = acc[mb][nb][1] = acc[mb][nb][2] = acc[mb][nb][3] = 0.f;
-
-    for (int t = 0; t < KT; ++t) {
-        const int stage = t % S;
-        gemv_wait(&full_bar[stage], (t / S) & 1, failed, a.status);
-        const uint32_t wbase = smem_addr(smem + stage * C::kStageBytes);
-        const uint32_t xbase = wbase + C::kWBytes;
-        const uint16_t* sbase =
-            reinterpret_cast<const uint16_t*>(smem + stage * C::kStageBytes + C::kWBytes + C::kXBytes);
-#pragma unroll
-        for (int grp = 0; grp < kGemvKTile / kGemvGroup; ++grp) {
-            float gacc[MB][kNB][4];
-#pragma unroll
-            for (int m = 0; m < MB; ++m)
-#pragma unroll
-                for (int nb = 0; nb < kNB; ++nb)
-                    gacc[m][nb][0] = gacc[m][nb][1] = gacc[m][nb][2] = gacc[m][nb][3] = 0.f;
-#pragma unroll
-            for (int bb = 0; bb < kGemvGroup / 64; ++bb) {
-                const int blk = grp * (kGemvGroup / 64) + bb;       // 64-column block of the tile
-                // codes: 8 bytes (columns 64 blk + 16c .. +15) of rows rlo and rlo + 8
-                uint2 wl[MB], wh[MB];
-#pragma unroll
-                for (int m = 0; m < MB; ++m) {
-                    const int rlo = rw + 16 * m + pg;
-                    wl[m] = lds64(wbase + swz<128, 128>(rlo, 32 * blk + 8 * c));
-                    wh[m] = lds64(wbase + swz<128, 128>(rlo + 8, 32 * blk + 8 * c));
-                }
-                const uint32_t xbox = xbase + blk * C::kXBoxBytes;
-                uint4 xv[kNB];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    // x: columns 64 blk + 16c + 8 (j/2) .. +7 of batch row 8 nb + g
-                    if ((j & 1) == 0) {
-#pragma unroll
-                        for (int nb = 0; nb < kNB; ++nb)
-                            xv[nb] = lds128(xbox + swz<128, 128>(8 * nb + g, 32 * c + 16 * (j >> 1)));
+                    for (int j = 0; j < kGemvGroup / 16; ++j) {
+                        // k-step j of the group: x columns 128 grp + 16 j .. +15, in box
+                        // (2 grp + j / 4) at byte 32 (j mod 4) of each 128-byte row
+                        const uint32_t xk = xaddr + (2 * grp + j / 4) * C::kXBoxBytes + 32 * (j % 4);
+                        tc_mma_ts(tmem + C::kDCol + b * kN, tmem + C::kACol + b * C::kGroupCols + 8 * j,
+                                  sw128_kmajor_desc(xk), idesc, j > 0 ? 1u : 0u);
                     }
-#pragma unroll
-                    for (int m = 0; m < MB; ++m) {
-                        const uint32_t lo = (j < 2) ? wl[m].x : wl[m].y;
-                        const uint32_t hi = (j < 2) ? wh[m].x : wh[m].y;
-                        const uint32_t by = 2 * (j & 1);
-                        const uint32_t a0 = int4x2_to_bf16x2(lo, lo >> 4, by);
-                        const uint32_t a2 = int4x2_to_bf16x2(lo, lo >> 4, by + 1);
-                        const uint32_t a1 = int4x2_to_bf16x2(hi, hi >> 4, by);
-                        const uint32_t a3 = int4x2_to_bf16x2(hi, hi >> 4, by + 1);
-#pragma unroll
-                        for (int nb = 0; nb < kNB; ++nb)
-                            mma_bf16(gacc[m][nb], a0, a1, a2, a3, (j & 1) ? xv[nb].z : xv[nb].x,
-                                     (j & 1) ? xv[nb].w : xv[nb].y);
-                    }
+                    tc_commit(&d_ready[b]);
                 }
-            }
-            // scale the group's sums by the rows' scales (rows rlo: c0, c1; rlo + 8: c2, c3)
-#pragma unroll
-            for (int m = 0; m < MB; ++m) {
-                const int rlo = rw + 16 * m + pg;
-                const float s_lo = bf16_bits_to_f32(sbase[grp * kGemvRows + rlo]);
-                const float s_hi = bf16_bits_to_f32(sbase[grp * kGemvRows + rlo + 8]);
-#pragma unroll
-                for (int nb = 0; nb < kNB; ++nb) {
-                    acc[m][nb][0] = fmaf(s_lo, gacc[m][nb][0], acc[m][nb][0]);
-                    acc[m][nb][1] = fmaf(s_lo, gacc[m][nb][1], acc[m][nb][1]);
-                    acc[m][nb][2] = fmaf(s_hi, gacc[m][nb][2], acc[m][nb][2]);
-                    acc[m][nb][3] = fmaf(s_hi, gacc[m][nb][3], acc[m][nb][3]);
-                }
+                tc_commit(&empty_x[stage]);    // this stage's x reads are done
             }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty_bar[stage]);
+    } else {
+        // ====== converters: warp w owns rows 32 (w mod 4) .., part w / 4 ======
+        // (thread = row = tensor-memory lane; the part picks 1 / kSplit of a
+        // group's columns for A and of the batch columns for the output)
+        constexpr int PU = C::kPartUnits;
+        const int quarter = warp & 3;
+        const int part = warp >> 2;
+        const int r = 32 * quarter + lane;                         // row in the tile
+        const uint32_t tlane = tmem + (static_cast<uint32_t>(32 * quarter) << 16);
+        float acc[C::kPartN];
+#pragma unroll
+        for (int n = 0; n < C::kPartN; ++n) acc[n] = 0.f;
+        float s_cur[2] = {0.f, 0.f}, s_prev[2] = {0.f, 0.f};
+
+        // acc += s * (this row's part of the accumulator of group g)
+        auto readout = [&](int g, float s) {
+            const int b = g & 1;
+            gemv_wait(&d_ready[b], (g >> 1) & 1, failed, a.status);
+            tc_fence_after();
+            const uint32_t dcol = tlane + C::kDCol + b * kN + part * C::kPartN;
+#pragma unroll
+            for (int q = 0; q < C::kPartN / 16; ++q) {
+                uint32_t v[16];
+                tmem_ld16(dcol + 16 * q, v);
+                tmem_wait_ld(v);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) acc[16 * q + i] = fmaf(s, __uint_as_float(v[i]), acc[16 * q + i]);
+            }
+        };
+
+        for (int t = 0; t < KT; ++t) {
+            const int stage = t % SW;
+            gemv_wait(&full_w[stage], (t / SW) & 1, failed, a.status);
+            const uint32_t wrow = smem_addr(smem + stage * C::kWStageBytes) + r * 128;
+            const uint16_t* sb = reinterpret_cast<const uint16_t*>(smem + stage * C::kWStageBytes + C::kWBytes);
+            // this row's code units of this part: group grp, units 4 grp + PU part + e;
+            // 16-byte unit u of a row sits at unit u ^ (r mod 8)
+            uint4 raw[2 * PU];
+#pragma unroll
+            for (int grp = 0; grp < 2; ++grp)
+#pragma unroll
+                for (int e = 0; e < PU; ++e) {
+                    const int u = 4 * grp + PU * part + e;
+                    raw[PU * grp + e] = lds128(wrow + ((u ^ (r & 7)) << 4));
+                }
+            s_prev[0] = s_cur[0];
+            s_prev[1] = s_cur[1];
+            s_cur[0] = bf16_bits_to_f32(sb[r]);
+            s_cur[1] = bf16_bits_to_f32(sb[kGemvRows + r]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty_w[stage]);     // codes and scales are in registers
+
+#pragma unroll
+            for (int grp = 0; grp < kGemvKTile / kGemvGroup; ++grp) {
+                const int g = t * (kGemvKTile / kGemvGroup) + grp;
+                const int b = g & 1;
+                // group g - 2 used the same A and accumulator buffers: read its
+                // result out (its MMAs are then complete) before overwriting A
+                if (g >= 2) readout(g - 2, s_prev[grp]);
+                // expand this part of the group's codes: unit e gives 16 bf16x2 A
+                // columns, column 4w + i = columns (8w + 2i, 8w + 2i + 1) of the unit
+#pragma unroll
+                for (int e = 0; e < PU; ++e) {
+                    const uint32_t wds[4] = {raw[PU * grp + e].x, raw[PU * grp + e].y, raw[PU * grp + e].z,
+                                             raw[PU * grp + e].w};
+                    uint32_t v[16];
+#pragma unroll
+                    for (int w = 0; w < 4; ++w)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) v[4 * w + i] = int4_pair_to_bf16x2(wds[w] >> (4 * i));
+                    tmem_st16(tlane + C::kACol + b * C::kGroupCols + 16 * (PU * part + e), v);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&a_ready[b]);
+            }
+        }
+        // the last two groups
+        for (int g = (NG >= 2 ? NG - 2 : 0); g < NG; ++g) readout(g, s_cur[g & 1]);
+
+        grid_dependency_wait();
+#pragma unroll
+        for (int n = 0; n < C::kPartN; ++n) {
+            const int bn = part * C::kPartN + n;
+            if (bn < a.batch) a.y[static_cast<int64_t>(bn) * a.n + row0 + r] = f32_to_bf16_bits(acc[n]);
+        }
     }
 
-    // y[b][n]: accumulator (row, col) = (weight row, batch row)
-    grid_dependency_wait();
-#pragma unroll
-    for (int m = 0; m < MB; ++m) {
-        const int nlo = row0 + rw + 16 * m + pg;
-#pragma unroll
-        for (int nb = 0; nb < kNB; ++nb)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int b = b0 + 8 * nb + 2 * c + (i & 1);
-                const int nn = nlo + ((i & 2) ? 8 : 0);
-                if (b < a.batch) a.y[static_cast<int64_t>(b) * a.n + nn] = f32_to_bf16_bits(acc[m][nb][i]);
-            }
+    // every tensor-memory access and MMA of this CTA is complete here (the
+    // converters waited for the last groups' commits): free the columns
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
     }
 }
 
-// Consumer warps per CTA: four warps of 32 rows (eight warps of 16 rows
-// measured the same on B200 and spill at batch 32).
-template <int kNB>
-struct GemvVariant {
-    static constexpr int kCW = 4;
-    using Cfg = GemvCfg<kNB, kCW>;
-};
+int gemv_batch_cols(int batch) { return batch <= 32 ? 32 : 64; }
 
-int gemv_batch_blocks(int batch) {
-    const int nb = (batch + 7) / 8;
-    return nb <= 1 ? 1 : (nb <= 2 ? 2 : 4);
-}
-
-#define PKV_GEMV_DISPATCH(nb, EXPR) \
-    switch (nb) {                    \
-        case 1: { constexpr int NB = 1; EXPR; } \
-        case 2: { constexpr int NB = 2; EXPR; } \
-        case 4: { constexpr int NB = 4; EXPR; } \
+#define PKV_GEMV_DISPATCH(ncols, EXPR) \
+    switch (ncols) {                     \
+        case 32: { constexpr int N = 32; EXPR; } \
+        case 64: { constexpr int N = 64; EXPR; } \
         default: return cudaErrorInvalidValue; \
     }
 
-cudaError_t gemv_set_smem_attr(int nb) {
-    PKV_GEMV_DISPATCH(nb, return cudaFuncSetAttribute(
-                              int4_gemv_kernel<NB, GemvVariant<NB>::kCW>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              GemvVariant<NB>::Cfg::kSmemBytes))
+cudaError_t gemv_set_smem_attr(int ncols) {
+    PKV_GEMV_DISPATCH(ncols, return cudaFuncSetAttribute(int4_gemv_kernel<N>,
+                                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                         GemvCfg<N>::kSmemBytes))
 }
 
-size_t gemv_smem_bytes(int nb) {
-    switch (nb) {
-        case 1: return GemvVariant<1>::Cfg::kSmemBytes;
-        case 2: return GemvVariant<2>::Cfg::kSmemBytes;
-        case 4: return GemvVariant<4>::Cfg::kSmemBytes;
-        default: return 0;
-    }
-}
-
-cudaError_t launch_int4_gemv(int nb, cudaStream_t stream, const CUtensorMap& tmap_w,
+cudaError_t launch_int4_gemv(int ncols, cudaStream_t stream, const CUtensorMap& tmap_w,
                              const CUtensorMap& tmap_x, const CUtensorMap& tmap_s, const GemvArgs& args) {
-    const int slices = (args.batch + 8 * nb - 1) / (8 * nb);
-    PKV_GEMV_DISPATCH(nb, {
-        PdlLaunch l(dim3(args.n / kGemvRows * slices), dim3(GemvVariant<NB>::Cfg::kThreads),
-                    GemvVariant<NB>::Cfg::kSmemBytes, stream);
-        return cudaLaunchKernelEx(&l.cfg, int4_gemv_kernel<NB, GemvVariant<NB>::kCW>, tmap_w, tmap_x,
-                                  tmap_s, args);
+    PKV_GEMV_DISPATCH(ncols, {
+        PdlLaunch l(dim3(args.n / kGemvRows), dim3(GemvCfg<N>::kThreads), GemvCfg<N>::kSmemBytes, stream);
+        return cudaLaunchKernelEx(&l.cfg, int4_gemv_kernel<N>, tmap_w, tmap_x, tmap_s, args);
     })
 }
 

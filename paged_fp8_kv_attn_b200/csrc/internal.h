@@ -116,12 +116,20 @@ struct GemvArgs {
     int32_t k;
 };
 
-// Batch blocks of 8 one CTA covers (1, 2 or 4; larger batches use
-// several CTAs per row tile).
-int gemv_batch_blocks(int batch);
-size_t gemv_smem_bytes(int nb);
-cudaError_t gemv_set_smem_attr(int nb);
-cudaError_t launch_int4_gemv(int nb, cudaStream_t stream, const CUtensorMap& tmap_w,
+// Batches up to kGemvMmaMaxBatch run on the warp-level MMA kernel
+// (int4_gemv_mma.cu), larger ones on the tcgen05 kernel (int4_gemv.cu).
+constexpr int kGemvMmaMaxBatch = 16;
+
+// tcgen05 kernel: batch columns of the tensor-core tile (16, 32 or 64).
+int gemv_batch_cols(int batch);
+cudaError_t gemv_set_smem_attr(int ncols);
+// warp-level MMA kernel: batch blocks of 8 (1 or 2).
+int gemv_mma_batch_blocks(int batch);
+cudaError_t gemv_mma_set_smem_attr(int nb);
+cudaError_t launch_int4_gemv_mma(int nb, cudaStream_t stream, const CUtensorMap& tmap_w,
+                                 const CUtensorMap& tmap_x, const CUtensorMap& tmap_s,
+                                 const GemvArgs& args);
+cudaError_t launch_int4_gemv(int ncols, cudaStream_t stream, const CUtensorMap& tmap_w,
                              const CUtensorMap& tmap_x, const CUtensorMap& tmap_s,
                              const GemvArgs& args);
 

@@ -24,10 +24,13 @@ def _abs_weights(case, rows=None):
     rows = np.arange(case.n) if rows is None else np.asarray(rows)
     tiles = case.w_tiles.cpu().numpy()                      # [n/128][k/256][128][128]
     sc = oracle.bf16_to_double(workloads.bf16_bits(case.scales))   # [n/128][k/g][128]
-    by = tiles[rows // 128, :, rows % 128, :].reshape(rows.size, -1).astype(np.int16)
-    codes = np.empty((rows.size, case.k), dtype=np.int16)
-    codes[:, 0::2] = by & 0xF
-    codes[:, 1::2] = by >> 4
+    by = tiles[rows // 128, :, rows % 128, :].reshape(rows.size, -1, 4).astype(np.int64)
+    words = by[..., 0] | (by[..., 1] << 8) | (by[..., 2] << 16) | (by[..., 3] << 24)   # 8 columns each
+    codes = np.empty((rows.size, case.k // 8, 8), dtype=np.int64)
+    for i in range(4):
+        codes[:, :, 2 * i] = (words >> (4 * i)) & 0xF
+        codes[:, :, 2 * i + 1] = (words >> (16 + 4 * i)) & 0xF
+    codes = codes.reshape(rows.size, case.k)
     codes = np.where(codes >= 8, codes - 16, codes)
     s = sc[rows // 128, :, rows % 128]                      # [rows][k/g]
     return np.abs(codes) * np.repeat(s, case.group, axis=1)

@@ -275,8 +275,13 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
         total += t;
     }
     const int64_t U = static_cast<int64_t>(IPR) * total;
-    const int64_t u_lo = static_cast<int64_t>(blockIdx.x) * U / a.num_ctas;
-    const int64_t u_hi = static_cast<int64_t>(blockIdx.x + 1) * U / a.num_ctas;
+    // The units are cut over NE = min(grid, U) CTAs, so that every CTA of the
+    // partition holds at least one unit and therefore writes the partial of
+    // every item it touches: the merge reads only slots written by this call
+    // (the rest of the grid, if any, has nothing to do).
+    const int64_t NE = U < a.num_ctas ? U : a.num_ctas;
+    const int64_t u_lo = (blockIdx.x < NE) ? static_cast<int64_t>(blockIdx.x) * U / NE : U;
+    const int64_t u_hi = (blockIdx.x < NE) ? static_cast<int64_t>(blockIdx.x + 1) * U / NE : U;
     {
         int run = warp_base + incl - local;
         for (int b = b_lo; b < b_hi; ++b) {
@@ -959,9 +964,10 @@ attn_merge_kernel(const AttnArgs a) {
         return;
     }
     const int64_t U = static_cast<int64_t>(IPR) * tot;
+    const int NE = static_cast<int>(U < a.num_ctas ? U : a.num_ctas);   // as in the partial kernel
     const int64_t u0 = static_cast<int64_t>(IPR) * pre + static_cast<int64_t>(h) * n;
-    const int64_t c0 = cta_of_unit(u0, U, a.num_ctas);
-    const int64_t c1 = cta_of_unit(u0 + n - 1, U, a.num_ctas);
+    const int64_t c0 = cta_of_unit(u0, U, NE);
+    const int64_t c1 = cta_of_unit(u0 + n - 1, U, NE);
     if (c0 == c1) return;   // finished by the partial kernel
     const int nseg = static_cast<int>(c1 - c0 + 1);
     if (tid < 16) {

@@ -249,6 +249,36 @@ def test_attention_small_all_items(cuda_device, case, kv):
 
 
 @pytest.mark.parametrize("kv", ["fp8", "bf16"])
+def test_attention_workspace_reused_across_calls(cuda_device, kv):
+    """One workspace serves consecutive calls with different grids and a
+    different batch: the per-item arrival counters that pick the CTA merging
+    a split item must be back at zero after every call."""
+    wl1 = workloads.custom([3000, 70, 9000, 1, 640], page_size=64, num_q_heads=64, num_kv_heads=8,
+                           head_dim=128, seed=41, spare_pages=2)
+    wl2 = workloads.custom([129] * 9 + [2000], page_size=64, num_q_heads=64, num_kv_heads=8,
+                           head_dim=128, seed=42, spare_pages=2)
+    db1 = DeviceBatch(wl1, kv_dtype=kv)
+    db2 = DeviceBatch(wl2, kv_dtype=kv)
+    n1 = pkv.paged_decode_attn_workspace_size(db1.kv_code, wl1.batch, 64, 8, 128, 0)
+    n2 = pkv.paged_decode_attn_workspace_size(db2.kv_code, wl2.batch, 64, 8, 128, 0)
+    ws = torch.zeros(max(n1, n2), dtype=torch.uint8, device=db1.q.device)
+    db1.ws = ws
+    db2.ws = ws
+    items1 = list(range(wl1.batch * 8))
+    items2 = list(range(wl2.batch * 8))
+    ref1 = oracle_step(wl1, items1, kv_dtype=kv, check=False, append=True)
+    ref2 = oracle_step(wl2, items2, kv_dtype=kv, check=False, append=True)
+    for db, wl, items, ref, ctas in ((db1, wl1, items1, ref1, 37), (db2, wl2, items2, ref2, 5),
+                                     (db1, wl1, items1, ref1, 0), (db2, wl2, items2, ref2, 0),
+                                     (db1, wl1, items1, ref1, 3)):
+        db.out.fill_(float("nan"))
+        db.step(check=False, append=True, num_ctas=ctas)
+        out, lse = db.outputs()
+        compare(wl, items, out, lse, ref[0], ref[1], label=f"{kv} B={wl.batch} ctas={ctas}")
+        assert pkv.workspace_status(ws) == 0
+
+
+@pytest.mark.parametrize("kv", ["fp8", "bf16"])
 def test_attention_tiny_decode_with_check(cuda_device, kv):
     wl = workloads.tiny_decode()
     ref_o, ref_l, ref_abort = oracle_step(wl, [0, 1], kv_dtype=kv)

@@ -194,6 +194,8 @@ class Step:
         outs = [("out", torch.empty((B, Hq, D), dtype=torch.bfloat16)),
                 ("lse", torch.empty((B, Hq), dtype=torch.float32)),
                 ("abort", torch.zeros(B, dtype=torch.uint8))]
+        self._ins_meta = [(n, t.dtype, tuple(t.shape)) for n, t in ins]
+        self._outs_meta = [(n, t.dtype, tuple(t.shape)) for n, t in outs]
         self.dev_in, self.in_views = self._pack(ins, dev)
         self.dev_out, self.out_views = self._pack(outs, dev)
         for name, t in {**self.in_views, **self.out_views}.items():
@@ -214,6 +216,22 @@ class Step:
             code = pkv.PKV_KV_BF16
         self.ws = pkv.alloc_workspace(code, B, Hq, wl.num_kv_heads, D, device=dev)
         torch.cuda.synchronize()
+
+    def twin(self):
+        """The same step over a second set of packed input/output buffers
+        (shared caches, tags and workspace), for double-buffered end-to-end
+        steps: one set is copied while the other computes."""
+        import copy
+        import torch
+        t = copy.copy(self)
+        ins = [(n, torch.empty(shape, dtype=dt)) for n, dt, shape in self._ins_meta]
+        outs = [(n, torch.empty(shape, dtype=dt)) for n, dt, shape in self._outs_meta]
+        t.dev_in, t.in_views = self._pack(ins, self.dev_in.device)
+        t.dev_out, t.out_views = self._pack(outs, self.dev_out.device)
+        for name, v in {**t.in_views, **t.out_views}.items():
+            setattr(t, name, v)
+        t.dev_in.copy_(self.dev_in)
+        return t
 
     @staticmethod
     def _pack(named, dev):
@@ -409,29 +427,60 @@ def gpu_arm(args, rank, world):
     B = HEADLINE_BATCH
     # pinned host staging with the device buffers' packed layout: the step's
     # inputs (q, new K/V, lengths, page table, expected tags) go in with one
-    # copy; its results (out, lse, abort mask) come back with one copy
+    # copy; its results (out, lse, abort mask) come back with one copy.  Two
+    # device buffer sets alternate (double buffering, as a serving loop
+    # would): the inputs of step i+1 are copied in on one stream and the
+    # results of step i-1 copied out on another while step i computes.
     h_in = st.dev_in.cpu().pin_memory()
-    h_out = torch.empty_like(st.dev_out, device="cpu").pin_memory()
+    h_outs = [torch.empty_like(st.dev_out, device="cpu").pin_memory() for _ in range(2)]
     h2d = h_in.numel()       # bytes copied in per step (packed, 256-byte aligned slots)
-    d2h = h_out.numel()      # bytes copied out per step
+    d2h = h_outs[0].numel()  # bytes copied out per step
+    sts = [st, st.twin()]
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step():
-        st.dev_in.copy_(h_in, non_blocking=True)
-        st.full()
-        h_out.copy_(st.dev_out, non_blocking=True)
+    def e2e_run(n):
+        """n double-buffered steps; returns after enqueueing, with every copy
+        ordered before the compute stream's next work."""
+        with torch.cuda.stream(s_in):
+            s_in.wait_stream(comp)
+            sts[0].dev_in.copy_(h_in, non_blocking=True)
+            ev_in[0].record(s_in)
+        for i in range(n):
+            cur, nxt = i % 2, (i + 1) % 2
+            comp.wait_event(ev_in[cur])
+            if i >= 2:
+                comp.wait_event(ev_out[cur])      # step i-2's results have left this set
+            sts[cur].full()
+            ev_done[cur].record(comp)
+            if i + 1 < n:
+                with torch.cuda.stream(s_in):
+                    if i >= 1:
+                        s_in.wait_event(ev_done[nxt])   # step i-1 no longer reads this set
+                    sts[nxt].dev_in.copy_(h_in, non_blocking=True)
+                    ev_in[nxt].record(s_in)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[cur])
+                h_outs[cur].copy_(sts[cur].dev_out, non_blocking=True)
+                ev_out[cur].record(s_out)
+        comp.wait_stream(s_out)
+        comp.wait_stream(s_in)
 
-    for _ in range(args.warmup):
-        e2e_step()
+    e2e_run(max(args.warmup, 2))
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     e0.record()
-    for _ in range(args.steps):
-        e2e_step()
+    e2e_run(args.steps)
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = reduce_max_time(e0.elapsed_time(e1), world) / args.steps
     e2e_value = world * B / (e2e_ms / 1e3)
+    assert all(pkv_status_ok(x) for x in sts)
+    del sts
     assert pkv_status_ok(st)
     del g_full, g_unchecked, st
     torch.cuda.empty_cache()
@@ -506,7 +555,9 @@ def gpu_arm(args, rank, world):
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "api": "python binding -> C ABI, eager calls; one pinned H2D copy of the "
-                       "packed inputs and one D2H copy of the packed results per step"},
+                       "packed inputs and one D2H copy of the packed results per step, "
+                       "double-buffered on two copy streams (step i+1 in and step i-1 out "
+                       "while step i computes)"},
         "gpu_launches": 3 * args.steps,
         "clocks": clk,
         "sweep": sweep,

@@ -59,6 +59,23 @@ def attn_algorithmic_bytes(seq_lens, page_size, num_q_heads, num_kv_heads, head_
     return kv + qo + pt
 
 
+def unique_kv_tokens(seq_lens, page_table, page_size):
+    """Distinct (physical page, slot) positions attention reads in one step:
+    a page shared by several requests counts once, with the most slots any of
+    them reads from it."""
+    import numpy as np
+    per_page = {}
+    for b, L in enumerate(seq_lens):
+        L = int(L)
+        n = (L + page_size - 1) // page_size
+        for j in range(n):
+            pg = int(page_table[b][j])
+            used = min(page_size, L - j * page_size)
+            if used > per_page.get(pg, 0):
+                per_page[pg] = used
+    return int(sum(per_page.values()))
+
+
 def reduce_max_time(local_ms: float, world: int) -> float:
     """Max of a per-rank time over the process group (identity if world == 1)."""
     if world <= 1:
@@ -315,6 +332,27 @@ def _graph(fn):
     return g
 
 
+class L2Flush:
+    """Evicts L2 between timed calls: writes one buffer of twice the L2 size,
+    then reads another of the same size, so that neither the previous call's
+    inputs nor dirty lines (which the timed call would otherwise have to
+    write back) remain in L2."""
+
+    def __init__(self):
+        import torch
+        n = 2 * L2_BYTES // 4
+        self.w = torch.zeros(n, dtype=torch.float32, device="cuda")
+        self.r = torch.zeros(n, dtype=torch.float32, device="cuda")
+        self.sink = torch.zeros((), dtype=torch.float32, device="cuda")
+
+    def __call__(self):
+        import torch
+        self.w.add_(1)
+        torch.sum(self.r, dim=0, out=self.sink)
+
+    describe = f"flushed between calls (write {2 * L2_BYTES >> 20} MiB, then read another {2 * L2_BYTES >> 20} MiB)"
+
+
 def time_per_call(fn, steps, warmup, flush=None):
     """Median/mean device time (us) of fn, one CUDA-event pair per call on the
     current stream; an optional L2 flush between calls is outside the events."""
@@ -326,7 +364,7 @@ def time_per_call(fn, steps, warmup, flush=None):
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     for i in range(steps):
         if flush is not None:
-            flush.add_(1)
+            flush()
         starts[i].record()
         fn()
         ends[i].record()
@@ -347,7 +385,7 @@ def time_pair(fn_a, fn_b, steps, warmup, flush=None):
     for i in range(steps):
         for j, fn in enumerate((fn_a, fn_b)):
             if flush is not None:
-                flush.add_(1)
+                flush()
             ev[i][2 * j].record()
             fn()
             ev[i][2 * j + 1].record()
@@ -370,7 +408,7 @@ def gpu_arm(args, rank, world):
     except AttributeError:
         gpu_index = str(torch.cuda.current_device())
     peak, peak_kind = load_peaks()
-    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+    flush = L2Flush()
 
     # ---- headline: full step on the B=64 batch, CUDA-graph replays ------
     wl = workloads.concurrency_sweep(HEADLINE_BATCH, seed=replica_seed(2, rank), device="cuda")
@@ -510,7 +548,7 @@ def gpu_arm(args, rank, world):
                            "attn_frac_of_measured": round(byts / (t_a * 1e-6) / 1e9 / peak, 4),
                            "attn_frac_of_8tbs": round(byts / (t_a * 1e-6) / 1e9 / NOMINAL_HBM_GBS, 4),
                            "check_overhead_pct": round(100.0 * (t_step - t_u) / t_u, 3),
-                           "l2": "flushed between calls" if small else "inputs larger than L2"}
+                           "l2": L2Flush.describe if small else "inputs larger than L2"}
                 del gf, gu, ga, sb
                 torch.cuda.empty_cache()
             sweep.append(row)
@@ -519,6 +557,9 @@ def gpu_arm(args, rank, world):
 
     # ---- INT4 weight dequantisation GEMV (decode), against concurrency ----
     int4 = [] if args.no_int4 else int4_gemv_lines(args, rank, peak)
+
+    # ---- capacity, integrity stress, ragged + prefix workloads -----------
+    configs = {} if args.no_configs else config_lines(args, rank, peak)
 
     line = {
         "metric": METRIC,
@@ -562,8 +603,131 @@ def gpu_arm(args, rank, world):
         "clocks": clk,
         "sweep": sweep,
         "int4_gemv": int4,
+        "configs": configs,
     }
     return line
+
+
+def _kv_row(byts, t_us, peak):
+    gbs = byts / (t_us * 1e-6) / 1e9
+    return {"gbs": round(gbs, 1), "frac_of_measured": round(gbs / peak, 4),
+            "frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4)}
+
+
+def config_lines(args, rank, peak):
+    """The capacity, integrity-stress and ragged + prefix workloads, each
+    larger than L2 (no flush), CUDA-graph replays of the checked step
+    (fused check + append, then attention) and of the attention call."""
+    import numpy as np
+    import torch
+    import workloads
+    steps = max(args.steps, 20)
+    out = {}
+
+    # capacity: the same byte budget as 64 FP8 or 32 BF16 requests of 21,440
+    # tokens; both read ~2.81 GB of KV per step
+    cap = {}
+    for kv in ("fp8", "bf16"):
+        wl = workloads.capacity(kv, seed=replica_seed(3, rank), device="cuda")
+        st = Step(wl, kv)
+        eb = 1 if kv == "fp8" else 2
+        byts = attn_algorithmic_bytes(wl.seq_lens, wl.page_size, wl.num_q_heads,
+                                      wl.num_kv_heads, wl.head_dim, eb)
+        gf = _graph(st.full)
+        ga = _graph(lambda: st.attend(True))
+        t_step, _ = time_per_call(gf.replay, steps, args.warmup)
+        t_a, _ = time_per_call(ga.replay, steps, args.warmup)
+        torch.cuda.synchronize()
+        assert pkv_status_ok(st) and not bool(st.abort.any())
+        cap[kv] = {"batch": wl.batch, "tokens_per_request": int(wl.seq_lens[0]),
+                   "cached_tokens": wl.logical_tokens(),
+                   "kv_bytes": kv_bytes_per_step(wl.seq_lens, wl.num_kv_heads, wl.head_dim, eb),
+                   "step_us": round(t_step, 2),
+                   "tokens_per_s": round(wl.batch / (t_step * 1e-6), 1),
+                   "attn_us": round(t_a, 2), **_kv_row(byts, t_a, peak)}
+        del gf, ga, st, wl
+        torch.cuda.empty_cache()
+    cap["fp8_over_bf16_tokens_per_s"] = round(cap["fp8"]["tokens_per_s"] /
+                                              cap["bf16"]["tokens_per_s"], 3)
+    out["capacity"] = cap
+
+    # integrity stress: 256 requests, L ~ U[1024, 16384], pages reallocated
+    # three times; the overhead is measured with every expected tag current
+    # (equal work), then 0.1% of the entries are made stale
+    wl = workloads.integrity_stress(seed=replica_seed(4, rank), device="cuda")
+    st = Step(wl, "fp8")
+    stale_tags = wl.expected_tags.copy()
+    clean = wl.expected_tags.copy()
+    for b, j in wl.stale_entries:
+        clean[b, j] = wl.page_tags[wl.page_table[b, j]]
+    st.expected.copy_(torch.from_numpy(clean.view(np.int32)))
+    byts = attn_algorithmic_bytes(wl.seq_lens, wl.page_size, wl.num_q_heads,
+                                  wl.num_kv_heads, wl.head_dim, 1)
+    gf = _graph(st.full)
+    gu = _graph(st.unchecked)
+    gc = _graph(lambda: (st.check(), st.attend(True)))
+    ga = _graph(lambda: st.attend(False))
+    n_pair = max(steps, 60)
+    t_full, t_unch = time_pair(gf.replay, gu.replay, n_pair, args.warmup)
+    t_ca, t_a = time_pair(gc.replay, ga.replay, n_pair, args.warmup)
+    torch.cuda.synchronize()
+    assert not bool(st.abort.any())
+    st.expected.copy_(torch.from_numpy(stale_tags.view(np.int32)))
+    t_stale, _ = time_per_call(gf.replay, steps, args.warmup)
+    torch.cuda.synchronize()
+    aborted = np.nonzero(st.abort.cpu().numpy())[0].tolist()
+    want = sorted({b for b, _ in wl.stale_entries})
+    live = [b for b in range(wl.batch) if b not in set(want)]
+    live_bytes = attn_algorithmic_bytes(wl.seq_lens[live], wl.page_size, wl.num_q_heads,
+                                        wl.num_kv_heads, wl.head_dim, 1)
+    assert pkv_status_ok(st)
+    out["integrity_stress"] = {
+        "batch": wl.batch, "kv_tokens": wl.logical_tokens(),
+        "page_table_entries": int(sum(wl.used_pages(b) for b in range(wl.batch))),
+        "step_us": round(t_full, 2), "step_unchecked_us": round(t_unch, 2),
+        "check_overhead_pct": round(100.0 * (t_full - t_unch) / t_unch, 3),
+        "tag_check_then_attn_us": round(t_ca, 2), "attn_alone_us": round(t_a, 2),
+        "separate_check_overhead_pct": round(100.0 * (t_ca - t_a) / t_a, 3),
+        "attn": _kv_row(byts, t_a, peak),
+        "stale": {"entries": len(wl.stale_entries), "requests": len(want),
+                  "aborted_match": aborted == want, "step_us": round(t_stale, 2),
+                  "bytes_of_live_requests": live_bytes,
+                  **_kv_row(live_bytes, t_stale, peak)},
+        "overhead": "graph replays alternated: (fused check + append, attention with the "
+                    "mask) vs (append, attention without it); and (kv_tag_check, attention) "
+                    "vs attention alone"}
+    assert aborted == want, "abort mask differs from the stale requests"
+    del gf, gu, gc, ga, st, wl
+    torch.cuda.empty_cache()
+
+    # ragged + prefix: 512 requests, lognormal lengths, groups of 8 sharing a
+    # 4,096-token prefix; GB/s against unique bytes (L2 serves the repeats)
+    wl = workloads.ragged_prefix(seed=replica_seed(5, rank), device="cuda")
+    st = Step(wl, "fp8")
+    logical = attn_algorithmic_bytes(wl.seq_lens, wl.page_size, wl.num_q_heads,
+                                     wl.num_kv_heads, wl.head_dim, 1)
+    kv_logical = kv_bytes_per_step(wl.seq_lens, wl.num_kv_heads, wl.head_dim, 1)
+    u_tok = unique_kv_tokens(wl.seq_lens, wl.page_table, wl.page_size)
+    unique = logical - kv_logical + u_tok * wl.num_kv_heads * wl.head_dim * 2
+    gf = _graph(st.full)
+    ga = _graph(lambda: st.attend(True))
+    t_step, _ = time_per_call(gf.replay, steps, args.warmup)
+    t_a, _ = time_per_call(ga.replay, steps, args.warmup)
+    torch.cuda.synchronize()
+    assert pkv_status_ok(st) and not bool(st.abort.any())
+    lens = wl.seq_lens.astype(np.int64)
+    out["ragged_prefix"] = {
+        "batch": wl.batch, "logical_tokens": int(lens.sum()), "unique_tokens": u_tok,
+        "min_len": int(lens.min()), "median_len": int(np.median(lens)), "max_len": int(lens.max()),
+        "requests_over_8192": int((lens > 8192).sum()),
+        "logical_bytes": logical, "unique_bytes": unique,
+        "step_us": round(t_step, 2), "tokens_per_s": round(wl.batch / (t_step * 1e-6), 1),
+        "attn_us": round(t_a, 2),
+        "attn_logical_gbs": round(logical / (t_a * 1e-6) / 1e9, 1),
+        "attn_unique": _kv_row(unique, t_a, peak)}
+    del gf, ga, st, wl
+    torch.cuda.empty_cache()
+    return out
 
 
 def int4_algorithmic_bytes(batch, n, k, group):
@@ -737,6 +901,8 @@ def main():
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-int4", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the capacity, integrity-stress and ragged + prefix workloads")
     ap.add_argument("--kernel-only", choices=["fp8", "bf16", "int4"], default=None,
                     help="profiling target: run only the decode step (fp8/bf16) on a --batch "
                          "request concurrency-sweep batch, or only the INT4 GEMV at --batch; "

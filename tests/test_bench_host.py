@@ -81,3 +81,15 @@ def test_reference_arm_line_shape(monkeypatch):
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 3
     assert line["e2e"]["h2d_bytes_per_step"] == 0
     assert bench.reference_arm(args, 1, 2) is None
+
+
+def test_unique_kv_tokens_counts_shared_pages_once():
+    # P = 4.  Request 0 (10 tokens) reads pages 5, 6, 7 with 4, 4, 2 slots;
+    # request 1 (6 tokens) reads pages 5, 8 with 4, 2; request 2 (3 tokens)
+    # reads 3 slots of page 6.  Distinct positions: page 5 -> 4, page 6 -> 4,
+    # page 7 -> 2, page 8 -> 2 = 12 of 19 logical tokens.
+    table = [[5, 6, 7], [5, 8, -1], [6, -1, -1]]
+    assert bench.unique_kv_tokens([10, 6, 3], table, 4) == 12
+    assert bench.unique_kv_tokens([10], table[:1], 4) == 10
+    # a shorter reader of a shared page never raises its count
+    assert bench.unique_kv_tokens([3, 10], [[6, -1, -1], [5, 6, 7]], 4) == 10

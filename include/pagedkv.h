@@ -339,10 +339,13 @@ PKV_API size_t paged_decode_attn_fp8_noalloc_scratch_bytes(void);
  *           4-bit codes (-8..7) in tiles of 128 rows x 256 columns: tile
  *           (r, t), rows 128r.. and columns 256t.., is 16384 bytes at byte
  *           (r * (k/256) + t) * 16384; inside it row j's 128 bytes start at
- *           (j mod 128) * 128, and byte b holds column 256t + 2b in its low
- *           nibble and 256t + 2b + 1 in its high nibble (each tile is one
- *           contiguous read; a row-major [n][k/2] matrix m is tiled by
- *           m.reshape(n/128, 128, k/256, 128).transpose(0, 2, 1, 3));
+ *           (j mod 128) * 128 and hold 32 little-endian 32-bit words, word w
+ *           covering columns 256t + 8w .. +7: column 8w + 2i sits in bits
+ *           4i .. 4i+3 and column 8w + 2i + 1 in bits 16 + 4i .. 19 + 4i
+ *           (i = 0..3: the even columns in the low half-word, the odd ones
+ *           in the high half-word; each tile is one contiguous read).
+ *           int4_tile_layout in the Python binding re-lays a row-major
+ *           matrix of codes into this format;
  *   scales  n * k / group_size bf16 (16-byte aligned): the scale of rows
  *           128r.. for columns g*group_size.. is the 128-value run starting
  *           at element (r * (k/group_size) + g) * 128, one value per row;

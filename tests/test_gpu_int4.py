@@ -112,9 +112,11 @@ def test_full_size_sampled_rows(batch):
     compare(case, y, rows=rows)
 
 
-def test_batch_slices_are_independent():
-    # batch 64 runs as two 32-row slices: each row of y must equal the same
-    # row computed alone
+def test_batch_rows_are_independent():
+    # each row of a batch-64 call (tcgen05 kernel) equals the same row
+    # computed alone (warp-level kernel): the group sums of these inputs are
+    # exact in fp32 and both kernels scale and add the groups in the same
+    # order
     case = workloads.int4_gemv_case(64, n=256, k=512, seed=10, device="cuda")
     y = run_gpu(case)
     for b in (0, 31, 32, 63):
@@ -147,3 +149,18 @@ def test_tile_layout_helper_matches_the_format():
     tiles, sc = pkv.int4_tile_layout(rowmajor, s.to(torch.bfloat16).cuda())
     assert np.array_equal(oracle.int4_unpack(tiles.cpu().numpy(), n, k), codes)
     assert np.array_equal(oracle.int4_scales(workloads.bf16_bits(sc), n, k, 128), s.double().numpy())
+
+
+@pytest.mark.parametrize("batch", [3, 16, 17, 40])
+def test_odd_numbers_of_row_blocks_and_k_tiles(batch):
+    """37 row blocks x 9 k-tiles: CTA counts and k-tile loops that are not
+    powers of two, on both kernels."""
+    case = workloads.int4_gemv_case(batch, n=128 * 37, k=256 * 9, seed=13, device="cuda")
+    compare(case, run_gpu(case))
+
+
+def test_repeated_calls_are_bit_identical():
+    case = workloads.int4_gemv_case(8, n=128 * 37, k=256 * 9, seed=14, device="cuda")
+    y1 = run_gpu(case)
+    for _ in range(3):
+        assert torch.equal(y1, run_gpu(case))

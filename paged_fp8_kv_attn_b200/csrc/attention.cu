@@ -921,7 +921,10 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
 }
 
 // ---------------------------------------------------------------------------
-// merge: one CTA per (request, KV head) item.  For each query head h of the
+// merge: per (request, KV head) item, one CTA for all of its query heads
+// (kHPC = 16) or, when the items are split over many CTAs, one CTA per group
+// of 4 query heads (kHPC = 4: each thread then owns a single output and has
+// every segment's value in flight at once).  For each query head h of the
 // item: M = max_s m_s, L = sum_s l_s 2^(m_s - M), out = sum_s O_s 2^(m_s - M) / L
 // over the item's segments s (one per CTA that worked on it).  Segment
 // weights are computed once into shared memory (in tiles of kMergeTile
@@ -936,27 +939,31 @@ __device__ __forceinline__ int64_t cta_of_unit(int64_t u, int64_t U, int N) {
     return ((u + 1) * N + U - 1) / U - 1;
 }
 
-template <int kD>
+template <int kD, int kHPC>
 __global__ void __launch_bounds__(kMergeThreads)
 attn_merge_kernel(const AttnArgs a) {
-    __shared__ float s_w[kMergeTile][16];   // m_s, then weight 2^(m_s - M), of segment s, head h
-    __shared__ float s_l[kMergeTile][16];   // l_s
-    __shared__ float s_m[16], s_sum[16], s_scale[16];
+    __shared__ float s_w[kMergeTile][kHPC];   // m_s, then weight 2^(m_s - M), of segment s, head h
+    __shared__ float s_l[kMergeTile][kHPC];   // l_s
+    __shared__ float s_m[kHPC], s_sum[kHPC], s_scale[kHPC];
     __shared__ int s_dead;
     launch_dependents();
     grid_dependency_wait();
+    constexpr int kGroups = 16 / kHPC;       // CTAs per item
     const int IPR = a.items_per_req;
-    const int item = blockIdx.x;
+    const int item = blockIdx.x / kGroups;
     const int b = item / IPR, h = item % IPR;
-    const int G = a.group * a.kv_per_item;   // query heads of one item
+    const int G = a.group * a.kv_per_item;   // query heads of one item (at most 16)
+    const int hq0 = (blockIdx.x % kGroups) * kHPC;   // this CTA's first head of the item
+    if (hq0 >= G) return;
+    const int NH = min(kHPC, G - hq0);       // this CTA's heads
     const int tid = threadIdx.x;
-    const int64_t head0 = static_cast<int64_t>(b) * a.num_q_heads + h * G;
+    const int64_t head0 = static_cast<int64_t>(b) * a.num_q_heads + h * G + hq0;
     const int32_t pre = a.ws_prefix[b];
     const int32_t nxt = a.ws_prefix[b + 1];
     const int32_t tot = a.ws_prefix[a.batch];
     const int32_t n = nxt - pre;
     if (n == 0) {
-        for (int e = tid; e < G * kD; e += kMergeThreads) {
+        for (int e = tid; e < NH * kD; e += kMergeThreads) {
             const int hq = e / kD, d = e % kD;
             a.out[(head0 + hq) * kD + d] = 0;
             if (d == 0) a.lse[head0 + hq] = kNegInf;
@@ -970,12 +977,12 @@ attn_merge_kernel(const AttnArgs a) {
     const int64_t c1 = cta_of_unit(u0 + n - 1, U, NE);
     if (c0 == c1) return;   // finished by the partial kernel
     const int nseg = static_cast<int>(c1 - c0 + 1);
-    if (tid < 16) {
+    if (tid < kHPC) {
         s_m[tid] = kNegInf;
         s_sum[tid] = 0.f;
     }
     if (tid == 0) s_dead = 0;
-    constexpr int kPer = (16 * kD + kMergeThreads - 1) / kMergeThreads;
+    constexpr int kPer = (kHPC * kD + kMergeThreads - 1) / kMergeThreads;
     float acc[kPer];
 #pragma unroll
     for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
@@ -983,17 +990,18 @@ attn_merge_kernel(const AttnArgs a) {
 
     for (int t0 = 0; t0 < nseg; t0 += kMergeTile) {
         const int tn = min(kMergeTile, nseg - t0);
-        // (1) the tile's (m, l) pairs into shared memory: one round trip
-        for (int e = tid; e < tn * G; e += kMergeThreads) {
-            const int sg = e / G, hq = e % G;
+        // (1) the tile's (m, l) pairs of this CTA's heads into shared memory:
+        // one round trip
+        for (int e = tid; e < tn * NH; e += kMergeThreads) {
+            const int sg = e / NH, hq = e % NH;
             const int64_t slot = c0 + t0 + sg + item;
-            const float2 ml = *reinterpret_cast<const float2*>(a.ws_ml + (slot * G + hq) * 2);
+            const float2 ml = *reinterpret_cast<const float2*>(a.ws_ml + (slot * G + hq0 + hq) * 2);
             s_w[sg][hq] = ml.x;
             s_l[sg][hq] = ml.y;
         }
         __syncthreads();
         // (2) per head, in shared memory: new running max, weights, sum
-        for (int hq = tid >> 5; hq < G; hq += kMergeThreads / 32) {
+        for (int hq = tid >> 5; hq < NH; hq += kMergeThreads / 32) {
             float mx = kNegInf;
             int dead = 0;
             for (int sg = (tid & 31); sg < tn; sg += 32) {
@@ -1025,19 +1033,28 @@ attn_merge_kernel(const AttnArgs a) {
             }
         }
         __syncthreads();
-        // (3) outputs: segment-major, kPer x 8 independent loads in flight
-        const float* base = a.ws_o + (c0 + t0 + item) * stride;
+        // (3) outputs: segment-major, kPer x kUnroll independent loads in flight
+        const float* base = a.ws_o + (c0 + t0 + item) * stride + static_cast<int64_t>(hq0) * kD;
 #pragma unroll
         for (int k = 0; k < kPer; ++k) {
             const int e = tid + k * kMergeThreads;
-            if (e < G * kD) acc[k] *= s_scale[e / kD];
+            if (e < NH * kD) acc[k] *= s_scale[e / kD];
         }
+        if constexpr (kPer == 1) {
+            const int e = tid;
+            if (e < NH * kD) {
+                const int hq = e / kD;
+#pragma unroll 16
+                for (int sg = 0; sg < tn; ++sg) acc[0] += s_w[sg][hq] * base[sg * stride + e];
+            }
+        } else {
 #pragma unroll 8
-        for (int sg = 0; sg < tn; ++sg) {
+            for (int sg = 0; sg < tn; ++sg) {
 #pragma unroll
-            for (int k = 0; k < kPer; ++k) {
-                const int e = tid + k * kMergeThreads;
-                if (e < G * kD) acc[k] += s_w[sg][e / kD] * base[sg * stride + e];
+                for (int k = 0; k < kPer; ++k) {
+                    const int e = tid + k * kMergeThreads;
+                    if (e < NH * kD) acc[k] += s_w[sg][e / kD] * base[sg * stride + e];
+                }
             }
         }
         __syncthreads();
@@ -1045,7 +1062,7 @@ attn_merge_kernel(const AttnArgs a) {
 #pragma unroll
     for (int k = 0; k < kPer; ++k) {
         const int e = tid + k * kMergeThreads;
-        if (e >= G * kD) break;
+        if (e >= NH * kD) break;
         const int hq = e / kD, d = e % kD;
         if (s_dead) {
             a.out[(head0 + hq) * kD + d] = 0;
@@ -1119,9 +1136,17 @@ cudaError_t launch_attn_partial(bool fp8, int head_dim, int group_pad, int kv_pe
 }
 
 cudaError_t launch_attn_merge(int head_dim, cudaStream_t stream, const AttnArgs& args) {
-    PdlLaunch l(dim3(args.batch * args.items_per_req), dim3(kMergeThreads), 0, stream);
-    if (head_dim == 64) return cudaLaunchKernelEx(&l.cfg, attn_merge_kernel<64>, args);
-    return cudaLaunchKernelEx(&l.cfg, attn_merge_kernel<128>, args);
+    // Items split over 8 or more CTAs on average (small batches on a full
+    // grid) are merged by one CTA per 4 query heads, the others by one CTA
+    // per item.
+    const int64_t items = static_cast<int64_t>(args.batch) * args.items_per_req;
+    const bool wide = args.num_ctas >= 8 * items;
+    PdlLaunch l(dim3(static_cast<unsigned>(items * (wide ? 4 : 1))), dim3(kMergeThreads), 0, stream);
+    if (head_dim == 64)
+        return wide ? cudaLaunchKernelEx(&l.cfg, attn_merge_kernel<64, 4>, args)
+                    : cudaLaunchKernelEx(&l.cfg, attn_merge_kernel<64, 16>, args);
+    return wide ? cudaLaunchKernelEx(&l.cfg, attn_merge_kernel<128, 4>, args)
+                : cudaLaunchKernelEx(&l.cfg, attn_merge_kernel<128, 16>, args);
 }
 
 }  // namespace pkv

@@ -74,6 +74,9 @@ def _load():
             lib.orc_paged_decode_attn.argtypes = [i32, P, P, P, f32, f32, P, i32, P, i32,
                                                   i32, i32, i32, i32, i32, f32, P, P, i32,
                                                   P, P]
+            lib.orc_attn_partial.argtypes = [i32, P, P, P, f32, f32, P, i32, i32, i32, i32,
+                                             i32, f32, i32, i32, i32, i32, P, P, P]
+            lib.orc_lse_merge.argtypes = [i32, i32, P, P, P, P, P]
             lib.orc_int4_code.argtypes = [P, i32, i32, i32]
             lib.orc_int4_code.restype = i32
             lib.orc_int4_scale.argtypes = [P, i32, i32, i32, i32]
@@ -282,6 +285,41 @@ def paged_decode_attn(q_bits, k_cache, v_cache, page_table, seq_lens, num_kv_hea
         with ThreadPoolExecutor(max_workers=len(chunks)) as ex:
             list(ex.map(run, chunks))
     return out, lse
+
+
+def attn_partial(q_bits, k_cache, v_cache, page_table, num_kv_heads, page_size, sm_scale,
+                 b, h, t0, t1, k_scale=1.0, v_scale=1.0):
+    """Split-K piece of query head h of request b over tokens [t0, t1):
+    (m, l, o) with m = max s_t, l = sum exp(s_t - m), o = sum exp(s_t - m) v_t
+    (unnormalised, fp64 [D])."""
+    lib = _load()
+    q_bits = _c(q_bits, np.uint16)
+    page_table = _c(page_table, np.int32)
+    kv_dtype = 0 if k_cache.dtype == np.uint8 else 1
+    k_cache = np.ascontiguousarray(k_cache)
+    v_cache = np.ascontiguousarray(v_cache)
+    B, Hq, D = q_bits.shape
+    m = np.zeros(1, dtype=np.float64)
+    l = np.zeros(1, dtype=np.float64)
+    o = np.zeros(D, dtype=np.float64)
+    lib.orc_attn_partial(kv_dtype, _ptr(q_bits), _ptr(k_cache), _ptr(v_cache),
+                         ctypes.c_float(k_scale), ctypes.c_float(v_scale), _ptr(page_table),
+                         page_table.shape[1], Hq, num_kv_heads, D, page_size,
+                         ctypes.c_float(sm_scale), b, h, t0, t1, _ptr(m), _ptr(l), _ptr(o))
+    return float(m[0]), float(l[0]), o
+
+
+def lse_merge(ms, ls, os_):
+    """Merge of split-K partials (m_s, l_s, o_s [D]): (out fp64 [D], lse)."""
+    lib = _load()
+    ms = _c(np.asarray(ms, dtype=np.float64), np.float64)
+    ls = _c(np.asarray(ls, dtype=np.float64), np.float64)
+    os_ = _c(np.asarray(os_, dtype=np.float64).reshape(ms.size, -1), np.float64)
+    D = os_.shape[1]
+    out = np.zeros(D, dtype=np.float64)
+    lse = np.zeros(1, dtype=np.float64)
+    lib.orc_lse_merge(ms.size, D, _ptr(ms), _ptr(ls), _ptr(os_), _ptr(out), _ptr(lse))
+    return out, float(lse[0])
 
 
 # --------------------------------------------------------------------------

@@ -450,6 +450,90 @@ void orc_paged_decode_attn(int32_t kv_dtype, const uint16_t* q,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Split-K pieces and their log-sum-exp merge                               */
+/* ------------------------------------------------------------------------ */
+/*
+ * The decomposition the CUDA path uses (not on the pages, which give no
+ * kernel design): attention over a token range [t0, t1) of one query head
+ * gives a partial (m, l, o) with m = max_t s_t, l = sum_t exp(s_t - m) and
+ * the unnormalised o = sum_t exp(s_t - m) v_t; partials of disjoint ranges
+ * covering the sequence merge into the head's output and LSE:
+ *   M = max_s m_s,  l = sum_s l_s exp(m_s - M),
+ *   out = sum_s o_s exp(m_s - M) / l,  LSE = M + ln l.
+ * An empty range is the partial (-inf, 0, 0); merging only empty partials
+ * gives out = 0 and LSE = -inf.  The scores s_t are those of
+ * orc_paged_decode_attn (the caller passes a live request).
+ */
+void orc_attn_partial(int32_t kv_dtype, const uint16_t* q, const void* k_cache,
+                      const void* v_cache, float k_scale, float v_scale,
+                      const int32_t* page_table, int32_t max_pages, int32_t num_q_heads,
+                      int32_t num_kv_heads, int32_t head_dim, int32_t page_size,
+                      float sm_scale, int32_t b, int32_t h, int32_t t0, int32_t t1,
+                      double* m_out, double* l_out, double* o_out)
+{
+    int32_t hk = h / (num_q_heads / num_kv_heads);
+    const uint16_t* qh = q + ((int64_t)b * num_q_heads + h) * head_dim;
+    for (int32_t d = 0; d < head_dim; ++d)
+        o_out[d] = 0.0;
+    *m_out = -INFINITY;
+    *l_out = 0.0;
+    if (t1 <= t0)
+        return;
+    double* scores = (double*)malloc(sizeof(double) * (size_t)(t1 - t0));
+    double m = -INFINITY;
+    for (int32_t t = t0; t < t1; ++t) {
+        int32_t pid = page_table[(int64_t)b * max_pages + t / page_size];
+        double dot = 0.0;
+        for (int32_t d = 0; d < head_dim; ++d)
+            dot += orc_bf16_to_double(qh[d]) *
+                   kv_element(kv_dtype, k_cache, (double)k_scale, pid, num_kv_heads, hk,
+                              page_size, t % page_size, head_dim, d);
+        scores[t - t0] = (double)sm_scale * dot;
+        if (scores[t - t0] > m)
+            m = scores[t - t0];
+    }
+    double l = 0.0;
+    for (int32_t t = t0; t < t1; ++t) {
+        int32_t pid = page_table[(int64_t)b * max_pages + t / page_size];
+        double w = exp(scores[t - t0] - m);
+        l += w;
+        for (int32_t d = 0; d < head_dim; ++d)
+            o_out[d] += w * kv_element(kv_dtype, v_cache, (double)v_scale, pid, num_kv_heads,
+                                       hk, page_size, t % page_size, head_dim, d);
+    }
+    free(scores);
+    *m_out = m;
+    *l_out = l;
+}
+
+void orc_lse_merge(int32_t n, int32_t head_dim, const double* m, const double* l,
+                   const double* o, double* out, double* lse)
+{
+    double M = -INFINITY;
+    for (int32_t s = 0; s < n; ++s)
+        if (m[s] > M)
+            M = m[s];
+    for (int32_t d = 0; d < head_dim; ++d)
+        out[d] = 0.0;
+    if (M == -INFINITY) {
+        *lse = -INFINITY;
+        return;
+    }
+    double lsum = 0.0;
+    for (int32_t s = 0; s < n; ++s) {
+        if (m[s] == -INFINITY)
+            continue;
+        double w = exp(m[s] - M);
+        lsum += l[s] * w;
+        for (int32_t d = 0; d < head_dim; ++d)
+            out[d] += o[(int64_t)s * head_dim + d] * w;
+    }
+    for (int32_t d = 0; d < head_dim; ++d)
+        out[d] /= lsum;
+    *lse = M + log(lsum);
+}
+
+/* ------------------------------------------------------------------------ */
 /* INT4 weight dequantisation GEMV (decode)                                 */
 /* ------------------------------------------------------------------------ */
 /*

@@ -40,6 +40,11 @@ MUTANTS = {
                                "int64_t at = (int64_t)j * (k / group) + i / group;"),
     "int4_group_off_by_one": ("int64_t at = ((int64_t)(j / 128) * (k / group) + i / group) * 128 + j % 128;",
                               "int64_t at = ((int64_t)(j / 128) * (k / group) + (i + 1) % k / group) * 128 + j % 128;"),
+    "merge_l_unweighted": ("lsum += l[s] * w;", "lsum += l[s];"),
+    "merge_o_unweighted": ("out[d] += o[(int64_t)s * head_dim + d] * w;",
+                           "out[d] += o[(int64_t)s * head_dim + d];"),
+    "partial_not_shifted_by_max": ("double w = exp(scores[t - t0] - m);\n        l += w;",
+                                   "double w = exp(scores[t - t0]);\n        l += w;"),
     "transposed_v_index": ("o[d] += w * kv_element(kv_dtype, v_cache, (double)v_scale, pid,\n                                           num_kv_heads, hk, page_size, t % page_size,\n                                           head_dim, d);",
                            "o[d] += w * kv_element(kv_dtype, v_cache, (double)v_scale, pid,\n                                           num_kv_heads, hk, page_size, d % page_size,\n                                           head_dim, t % head_dim);"),
 }
@@ -60,6 +65,7 @@ def test_planted_mistake_is_caught(name, tmp_path):
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                         os.path.join(ROOT, "tests", "test_oracle_codec.py"),
                         os.path.join(ROOT, "tests", "test_oracle_paths.py"),
-                        os.path.join(ROOT, "tests", "test_oracle_int4.py")],
+                        os.path.join(ROOT, "tests", "test_oracle_int4.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_merge.py")],
                        env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"planted mistake {name} passed every pin:\n{r.stdout[-2000:]}"

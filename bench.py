@@ -93,6 +93,18 @@ def replica_seed(base: int, rank: int) -> int:
     return base + 1000 * rank
 
 
+def headline_config(world):
+    """The `config` object of both arms' lines: the headline workload."""
+    kv_gb = HEADLINE_BATCH * CONTEXT * 8 * 128 * 2 / 1e9
+    return {"workload": f"concurrency sweep, batch {HEADLINE_BATCH} x context {CONTEXT}, "
+                        "page 64, 64 q heads / 8 kv heads, head_dim 128, FP8 E4M3 KV",
+            "step": "tag check + FP8 append (one fused kernel) + paged attention "
+                    "(partial + merge), one layer",
+            "global_batch": world * HEADLINE_BATCH, "seq_len": CONTEXT,
+            "kv_dtype": "fp8_e4m3", "parallelism": f"replicas x{world}",
+            "l2": f"inputs larger than L2 ({kv_gb:.2f} GB of KV per step)"}
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -374,8 +386,9 @@ def time_per_call(fn, steps, warmup, flush=None):
 
 
 def time_pair(fn_a, fn_b, steps, warmup, flush=None):
-    """Median device times (us) of two calls measured alternately (a, b, a, b,
-    ...) so that clock and thermal drift affect both alike."""
+    """Device times (us) of two calls measured alternately (a, b, a, b, ...)
+    so that clock and thermal drift affect both alike: (median a, median b,
+    samples a, samples b), sample i of a and of b forming one pair."""
     import torch
     for _ in range(warmup):
         fn_a()
@@ -392,7 +405,42 @@ def time_pair(fn_a, fn_b, steps, warmup, flush=None):
     torch.cuda.synchronize()
     ta = [e[0].elapsed_time(e[1]) * 1e3 for e in ev]
     tb = [e[2].elapsed_time(e[3]) * 1e3 for e in ev]
-    return statistics.median(ta), statistics.median(tb)
+    return statistics.median(ta), statistics.median(tb), ta, tb
+
+
+def paired_overhead(ta, tb, n_boot=4000, seed=0):
+    """Overhead of a over b in percent from alternately measured pairs
+    (a_i, b_i): the median of the paired differences 100 (a_i - b_i) / b_i,
+    and a percentile-bootstrap 95% interval of that median (pairs resampled
+    with replacement, n_boot resamples, seeded)."""
+    import numpy as np
+    a = np.asarray(ta, dtype=np.float64)
+    b = np.asarray(tb, dtype=np.float64)
+    d = 100.0 * (a - b) / b
+    rng = np.random.Generator(np.random.PCG64(seed))
+    meds = np.median(d[rng.integers(0, d.size, (n_boot, d.size))], axis=1)
+    lo, hi = np.percentile(meds, [2.5, 97.5])
+    return float(np.median(d)), float(lo), float(hi)
+
+
+def measure_overhead(fn_a, fn_b, warmup, flush=None, pairs=200, max_pairs=1600, bound=1.0):
+    """Paired overhead of fn_a over fn_b with its 95% interval.  While the
+    interval straddles `bound` percent, more pairs are measured (doubling, up
+    to max_pairs), so the figure says on which side of the bound it lies
+    whenever the noise allows."""
+    ta, tb = [], []
+    n = pairs
+    while True:
+        _, _, a, b = time_pair(fn_a, fn_b, n - len(ta), warmup, flush)
+        ta += a
+        tb += b
+        med, lo, hi = paired_overhead(ta, tb)
+        if not (lo < bound < hi) or len(ta) >= max_pairs:
+            break
+        n = min(2 * n, max_pairs)
+    return {"median_pct": round(med, 3), "ci95_pct": [round(lo, 3), round(hi, 3)],
+            "pairs": len(ta), "t_a_us": round(statistics.median(ta), 2),
+            "t_b_us": round(statistics.median(tb), 2)}
 
 
 def gpu_arm(args, rank, world):
@@ -457,9 +505,7 @@ def gpu_arm(args, rank, world):
     traffic = ncu_traffic_per_launch(wl.logical_tokens() * wl.num_kv_heads)
 
     # ---- tag-check overhead: full step vs step without the check ---------
-    t_full, t_unch = time_pair(g_full.replay, g_unchecked.replay, max(args.steps, 100),
-                               args.warmup)
-    overhead_pct = 100.0 * (t_full - t_unch) / t_unch
+    overhead = measure_overhead(g_full.replay, g_unchecked.replay, args.warmup)
 
     # ---- end to end through the public API with host buffers -------------
     B = HEADLINE_BATCH
@@ -524,36 +570,45 @@ def gpu_arm(args, rank, world):
     torch.cuda.empty_cache()
 
     # ---- concurrency sweep, FP8 and BF16 side by side ---------------------
-    sweep = []
+    rows = []
     if not args.no_sweep:
         for b in SWEEP:
             wlb = workloads.concurrency_sweep(b, seed=replica_seed(2, rank), device="cuda")
-            row = {"batch": b}
+            row = [b]
             for kv in ("fp8", "bf16"):
                 sb = Step(wlb, kv)
                 eb = 1 if kv == "fp8" else 2
                 byts = attn_algorithmic_bytes(wlb.seq_lens, wlb.page_size, wlb.num_q_heads,
                                               wlb.num_kv_heads, wlb.head_dim, eb)
-                small = byts < 2 * L2_BYTES
+                fl = flush if byts < 2 * L2_BYTES else None
                 gf = _graph(sb.full)
                 gu = _graph(sb.unchecked)
                 ga = _graph(lambda: sb.attend(True))
-                steps = max(args.steps, 20)
-                fl = flush if small else None
-                t_step, t_u = time_pair(gf.replay, gu.replay, max(steps, 60), args.warmup, fl)
-                t_a, _ = time_per_call(ga.replay, steps, args.warmup, fl)
-                row[kv] = {"step_us": round(t_step, 2), "tokens_per_s": round(b / (t_step * 1e-6), 1),
-                           "attn_us": round(t_a, 2),
-                           "attn_gbs": round(byts / (t_a * 1e-6) / 1e9, 1),
-                           "attn_frac_of_measured": round(byts / (t_a * 1e-6) / 1e9 / peak, 4),
-                           "attn_frac_of_8tbs": round(byts / (t_a * 1e-6) / 1e9 / NOMINAL_HBM_GBS, 4),
-                           "check_overhead_pct": round(100.0 * (t_step - t_u) / t_u, 3),
-                           "l2": L2Flush.describe if small else "inputs larger than L2"}
+                ov = measure_overhead(gf.replay, gu.replay, args.warmup, fl)
+                t_a, _ = time_per_call(ga.replay, max(args.steps, 50), args.warmup, fl)
+                gbs = byts / (t_a * 1e-6) / 1e9
+                row += [round(t_a, 2), round(gbs / peak, 4), round(gbs / NOMINAL_HBM_GBS, 4),
+                        round(b / (ov["t_a_us"] * 1e-6), 1), ov["median_pct"], *ov["ci95_pct"]]
+                assert pkv_status_ok(sb)
                 del gf, gu, ga, sb
                 torch.cuda.empty_cache()
-            sweep.append(row)
+            rows.append(row)
             del wlb
             torch.cuda.empty_cache()
+    sweep = {
+        "cols": ["B"] + [f"{kv}_{c}" for kv in ("fp8", "bf16")
+                         for c in ("attn_us", "frac_meas", "frac_8tbs", "step_tok_s",
+                                   "chk_pct", "chk_ci_lo", "chk_ci_hi")],
+        "rows": rows,
+        "how": "attn: CUDA-graph replays of the attention call; step: check+append then "
+               "attention; chk: paired median overhead of the checked step over the unchecked "
+               "one, bootstrap 95% CI; L2 flushed between calls when KV < 2x L2 (B=1, 8 FP8; "
+               "B=1 BF16)"}
+    by_b = {r[0]: r for r in rows}
+    target = {"goal_frac_of_8tbs": 0.70,
+              "fp8_attn_frac_of_8tbs": {str(b): by_b[b][3] for b in (32, 64) if b in by_b}}
+    target["met_at_32_and_64"] = (len(target["fp8_attn_frac_of_8tbs"]) == 2 and
+                                  all(v >= 0.70 for v in target["fp8_attn_frac_of_8tbs"].values()))
 
     # ---- INT4 weight dequantisation GEMV (decode), against concurrency ----
     int4 = [] if args.no_int4 else int4_gemv_lines(args, rank, peak)
@@ -574,17 +629,12 @@ def gpu_arm(args, rank, world):
         "vs_baseline": None,
         "dtype": "e4m3 cache; f16 tensor-core products, f32 accumulate",
         "data": "synthetic (seeded; Q~N(0,1), K/V~N(0,1) with 1% x20 outliers, bf16 -> e4m3 at amax/448)",
-        "config": {"workload": f"concurrency sweep, batch {HEADLINE_BATCH} x context {CONTEXT}, "
-                               "page 64, 64 q heads / 8 kv heads, head_dim 128, FP8 E4M3 KV",
-                   "step": "tag check + FP8 append (one fused kernel) + paged attention "
-                           "(partial + merge), one layer",
-                   "global_batch": world * HEADLINE_BATCH, "seq_len": CONTEXT,
-                   "kv_dtype": "fp8_e4m3", "parallelism": f"replicas x{world}",
-                   "launch": "CUDA graph of the step (programmatic dependent launch)",
-                   "l2": f"inputs larger than L2 ({kv_bytes / 1e9:.2f} GB of KV per step)"},
+        "config": headline_config(world),
+        "launch": "CUDA graph of the step (programmatic dependent launch)",
         "step_kv_gbs": round(kv_bytes / (ms_per_step * 1e-3) / 1e9, 1),
         "step_kv_frac_of_8tbs": round(kv_bytes / (ms_per_step * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 4),
-        "check_overhead_pct": round(overhead_pct, 3),
+        "check_overhead_pct": overhead["median_pct"],
+        "check_overhead_ci95_pct": overhead["ci95_pct"],
         "roofline": {"kernel": "paged_decode_attn_fp8 (split-K partial + LSE merge)",
                      "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
@@ -601,9 +651,11 @@ def gpu_arm(args, rank, world):
                        "while step i computes)"},
         "gpu_launches": 3 * args.steps,
         "clocks": clk,
-        "sweep": sweep,
         "int4_gemv": int4,
         "configs": configs,
+        # kept last so that a reader of the line's tail sees them
+        "sweep": sweep,
+        "target": target,
     }
     return line
 
@@ -667,9 +719,10 @@ def config_lines(args, rank, peak):
     gu = _graph(st.unchecked)
     gc = _graph(lambda: (st.check(), st.attend(True)))
     ga = _graph(lambda: st.attend(False))
-    n_pair = max(steps, 60)
-    t_full, t_unch = time_pair(gf.replay, gu.replay, n_pair, args.warmup)
-    t_ca, t_a = time_pair(gc.replay, ga.replay, n_pair, args.warmup)
+    ov_fused = measure_overhead(gf.replay, gu.replay, args.warmup)
+    ov_sep = measure_overhead(gc.replay, ga.replay, args.warmup)
+    t_full, t_unch = ov_fused["t_a_us"], ov_fused["t_b_us"]
+    t_ca, t_a = ov_sep["t_a_us"], ov_sep["t_b_us"]
     torch.cuda.synchronize()
     assert not bool(st.abort.any())
     st.expected.copy_(torch.from_numpy(stale_tags.view(np.int32)))
@@ -684,10 +737,12 @@ def config_lines(args, rank, peak):
     out["integrity_stress"] = {
         "batch": wl.batch, "kv_tokens": wl.logical_tokens(),
         "page_table_entries": int(sum(wl.used_pages(b) for b in range(wl.batch))),
-        "step_us": round(t_full, 2), "step_unchecked_us": round(t_unch, 2),
-        "check_overhead_pct": round(100.0 * (t_full - t_unch) / t_unch, 3),
-        "tag_check_then_attn_us": round(t_ca, 2), "attn_alone_us": round(t_a, 2),
-        "separate_check_overhead_pct": round(100.0 * (t_ca - t_a) / t_a, 3),
+        "step_us": t_full, "step_unchecked_us": t_unch,
+        "check_overhead_pct": ov_fused["median_pct"],
+        "check_overhead_ci95_pct": ov_fused["ci95_pct"],
+        "tag_check_then_attn_us": t_ca, "attn_alone_us": t_a,
+        "separate_check_overhead_pct": ov_sep["median_pct"],
+        "separate_check_overhead_ci95_pct": ov_sep["ci95_pct"],
         "attn": _kv_row(byts, t_a, peak),
         "stale": {"entries": len(wl.stale_entries), "requests": len(want),
                   "aborted_match": aborted == want, "step_us": round(t_stale, 2),
@@ -695,7 +750,7 @@ def config_lines(args, rank, peak):
                   **_kv_row(live_bytes, t_stale, peak)},
         "overhead": "graph replays alternated: (fused check + append, attention with the "
                     "mask) vs (append, attention without it); and (kv_tag_check, attention) "
-                    "vs attention alone"}
+                    "vs attention alone; median of paired differences, bootstrap 95% CI"}
     assert aborted == want, "abort mask differs from the stale requests"
     del gf, gu, gc, ga, st, wl
     torch.cuda.empty_cache()
@@ -782,10 +837,9 @@ def pkv_status_ok(st) -> bool:
 class OracleSampler:
     """The CPU oracle, as it stands, on a bounded sample of the headline
     workload: R requests with the headline's per-request shape (8,192 tokens,
-    64 q heads / 8 KV heads, D=128, P=64, FP8).  One timed oracle step is the
-    tag check and the append of those requests plus attention over their
-    (request, KV head) items, run on all host cores; the time per item is
-    scaled to the 512 items of the batch-64 step."""
+    64 q heads / 8 KV heads, D=128, P=64, FP8).  One oracle step is the tag
+    check and the append of those requests plus attention over all their
+    (request, KV head) items, spread over the host cores."""
 
     def __init__(self, requests: int, seed: int = 2):
         import numpy as np
@@ -795,6 +849,7 @@ class OracleSampler:
         self.oracle = oracle
         self.np = np
         self.threads = os.cpu_count() or 1
+        self.requests = requests
         wl = workloads.concurrency_sweep(requests, seed=seed, device="cpu", context=CONTEXT)
         self.wl = wl
         self.kbits, self.vbits = bf16_bits(wl.k_pool), bf16_bits(wl.v_pool)
@@ -816,8 +871,9 @@ class OracleSampler:
             list(ex.map(job, [p for p in parts if p.size]))
         return out.reshape(bits.shape)
 
-    def step(self, n_items=None):
-        """Seconds of one oracle step over the first n_items items."""
+    def step(self, n_items=None, threads=None):
+        """Seconds of one oracle step over the first n_items items (all by
+        default) on `threads` threads (all host cores by default)."""
         wl, o = self.wl, self.oracle
         total = wl.batch * wl.num_kv_heads
         items = self.np.arange(total if n_items is None else min(n_items, total),
@@ -829,63 +885,76 @@ class OracleSampler:
                         wl.v_scale, self.kc, self.vc, abort)
         o.paged_decode_attn(self.q, self.kc, self.vc, wl.page_table, wl.seq_lens,
                             wl.num_kv_heads, wl.page_size, wl.sm_scale, wl.k_scale, wl.v_scale,
-                            abort=abort, items=items, threads=self.threads)
+                            abort=abort, items=items, threads=threads or self.threads)
         return time.perf_counter() - t0, int(items.size)
 
-    def tokens_per_s(self, seconds, n_items):
-        step_s = seconds / n_items * (HEADLINE_BATCH * self.wl.num_kv_heads)
-        return HEADLINE_BATCH / step_s
+
+def oracle_requests_per_step(threads=None):
+    """Requests per oracle step: enough (request, KV head) items, 8 per
+    request, to give every host core one."""
+    threads = threads or os.cpu_count() or 1
+    return max(1, -(-threads // 8))
+
+
+def oracle_run(steps, warmup, seed=2):
+    """The oracle timed over whole steps of R requests (R from
+    oracle_requests_per_step) on all host cores, plus one item on a single
+    thread.  tokens/s = R requests per step / measured step time (each request
+    yields one token per decode step)."""
+    requests = oracle_requests_per_step()
+    sampler = OracleSampler(requests=requests, seed=seed)
+    for _ in range(warmup):
+        sampler.step()
+    times = [sampler.step()[0] for _ in range(steps)]
+    step_s = sum(times) / len(times)
+    t1, _ = sampler.step(n_items=1, threads=1)
+    items_per_request = sampler.wl.num_kv_heads
+    return {"requests": requests, "items": requests * items_per_request,
+            "threads": sampler.threads, "steps": steps, "step_s": step_s,
+            "tokens_per_s": requests / step_s,
+            "single_thread_item_s": t1,
+            "single_thread_tokens_per_s": 1.0 / (t1 * items_per_request)}
+
+
+def _cpu_baseline_entry(r):
+    return {"value": round(r["tokens_per_s"], 4), "unit": UNIT, "cores": r["threads"],
+            "kind": "oracle",
+            "sample": f"{r['steps']} oracle steps, each the tag check, append and attention of "
+                      f"{r['requests']} request(s) ({r['items']} (request, KV head) items) of "
+                      f"the batch-64 step's shape (8,192 tokens, P=64, 64/8 heads, D=128, FP8) "
+                      f"on {r['threads']} threads; {r['step_s'] * 1e3:.1f} ms per step",
+            "single_thread": {"value": round(r["single_thread_tokens_per_s"], 4), "unit": UNIT,
+                              "cores": 1,
+                              "sample": f"one item on one thread ({r['single_thread_item_s']:.3f} "
+                                        f"s), times the 8 items of a request"}}
 
 
 def oracle_sample(target_s: float = 10.0, seed: int = 2):
-    """cpu_baseline entry of the JSON line: the oracle timed for about
-    target_s seconds of wall time on all host cores."""
-    threads = os.cpu_count() or 1
-    probe = OracleSampler(requests=1, seed=seed)
-    t1, n1 = probe.step(n_items=min(threads, 8))
-    per_round = t1                      # one item per thread, all threads busy
-    rounds = max(1, int(target_s / max(per_round, 1e-6)))
-    n_items = min(threads * rounds, 8 * 16)
-    requests = max(1, (n_items + 7) // 8)
-    sampler = OracleSampler(requests=requests, seed=seed)
-    t, n = sampler.step(n_items=n_items)
-    return {"value": round(sampler.tokens_per_s(t, n), 4), "unit": UNIT, "cores": threads,
-            "kind": "oracle",
-            "sample": f"{n} (request, KV head) items of {requests} request(s) with the batch-64 "
-                      f"step's shape (8,192 tokens, P=64, 64/8 heads, D=128, FP8) plus their tag "
-                      f"check and append, {t:.1f} s wall on {threads} threads; scaled to the "
-                      f"512 items of the batch-64 step"}
+    """cpu_baseline entry of the GPU arm's line: the same measurement as the
+    reference arm, with as many steps as fit in about target_s seconds."""
+    probe = OracleSampler(requests=oracle_requests_per_step(), seed=seed)
+    t, _ = probe.step()
+    del probe
+    steps = int(min(50, max(3, target_s / max(t, 1e-6))))
+    return _cpu_baseline_entry(oracle_run(steps, 1, seed))
 
 
-def reference_arm(args, rank, world):
-    """The oracle as the reference arm: each step is one oracle step over the
-    items of one request of the headline shape (a bounded sample), scaled to
-    the batch-64 step."""
+def reference_arm(args, rank, world, gpu_config=None):
+    """The oracle as the reference arm: each step is one oracle step over R
+    requests of the headline shape (enough items for every host core);
+    ms_per_step is that step's measured wall time and tokens/s = R / step
+    time.  Rank 0 only."""
     if rank != 0:
         return None
-    sampler = OracleSampler(requests=1)
-    for _ in range(args.warmup):
-        sampler.step()
-    secs, items = 0.0, 0
-    for _ in range(args.steps):
-        t, n = sampler.step()
-        secs += t
-        items += n
-    value = sampler.tokens_per_s(secs, items)
-    step_s = HEADLINE_BATCH / value
-    cpu = {"value": round(value, 4), "unit": UNIT, "cores": sampler.threads, "kind": "oracle",
-           "sample": f"per step: the 8 (request, KV head) items of one request of the batch-64 "
-                     f"step's shape plus its tag check and append, on {sampler.threads} "
-                     f"threads; scaled to the 512 items of the batch-64 step"}
+    r = oracle_run(args.steps, args.warmup)
+    value = r["tokens_per_s"]
     return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(step_s * 1e3, 3), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic (seeded)",
-            "config": {"workload": f"concurrency sweep, batch {HEADLINE_BATCH} x context {CONTEXT}, "
-                                   "page 64, 64 q heads / 8 kv heads, head_dim 128, FP8 E4M3 KV",
-                       "global_batch": HEADLINE_BATCH, "seq_len": CONTEXT,
-                       "parallelism": "host cores"},
-            "cpu_baseline": cpu,
+            "ms_per_step": round(r["step_s"] * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+            "data": "synthetic (seeded)",
+            "config": gpu_config if gpu_config is not None else headline_config(world),
+            "cpu_baseline": _cpu_baseline_entry(r),
             "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
@@ -951,6 +1020,8 @@ def main():
         if rank == 0 and not args.no_cpu_baseline:
             line["cpu_baseline"] = oracle_sample()
         if rank == 0:
+            for k in ("sweep", "target"):      # keep the sweep at the end of the line
+                line[k] = line.pop(k)
             print(json.dumps(line), flush=True)
     finally:
         if world > 1:

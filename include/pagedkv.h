@@ -224,9 +224,10 @@ PKV_API pkv_status kv_requant_pages_fp8(const uint16_t* src_pool, int32_t src_nu
  * call (0 = the default, one full wave of resident CTAs on the current
  * device).  Returns 0 on invalid arguments (see pkv_last_error).  The
  * workspace holds a status word, the per-request chunk offsets and the
- * split-K partial results; its first 4 bytes are a status word that the
- * kernels set nonzero only if an internal bounded wait expires (never
- * expected); the caller may read it after the stream has finished.
+ * split-K partial results.  Its first 4 bytes are a status word that every
+ * attention call writes: 0, or 1 if an internal bounded wait expired in that
+ * call (never expected; the outputs are then unreliable).  The caller may
+ * read it once the stream has finished the call.
  */
 PKV_API size_t paged_decode_attn_workspace_size(int32_t kv_dtype, int32_t batch, int32_t num_q_heads,
                                         int32_t num_kv_heads, int32_t head_dim,
@@ -255,8 +256,11 @@ PKV_API size_t paged_decode_attn_workspace_size(int32_t kv_dtype, int32_t batch,
  * [batch][num_q_heads] fp32.  workspace: device memory of at least
  * paged_decode_attn_workspace_size(PKV_KV_FP8, ...) bytes, 256-byte
  * aligned, not shared with a concurrently running attention call; its
- * contents need no initialisation.  num_ctas: split-K grid size (0 =
- * default); any value >= 1 gives the same result up to rounding.
+ * contents need no initialisation.  Calls issued back to back on one stream
+ * may share a workspace, with no synchronisation between them: a call's
+ * kernels write the workspace only after the previous kernel on the stream
+ * has finished.  num_ctas: split-K grid size (0 = default); any value >= 1
+ * gives the same result up to rounding.
  *
  * Work split: the (request, KV head, 64-token chunk) units are divided
  * evenly over the CTAs of one persistent wave; a request split over several
@@ -307,9 +311,10 @@ PKV_API pkv_status paged_decode_attn_bf16(const uint16_t* q, const uint16_t* k_c
  *     at head_dim 128 and a GQA group of 8;
  *   - the first call on a device looks up the array's device address for that
  *     device (make that first call before any stream capture);
- *   - the call allocates and frees nothing; it clears the array's status word
- *     on the stream and otherwise relies on the kernels writing every scratch
- *     value before reading it (the array keeps the previous call's contents);
+ *   - the call allocates and frees nothing; the kernels write every scratch
+ *     value before reading it (the array keeps the previous call's contents),
+ *     including the status word, which paged_decode_attn_fp8_noalloc_status
+ *     copies out;
  *   - all calls on a device share the one array, so two calls whose work
  *     overlaps on the GPU (different streams, or different host threads
  *     without ordering) race and corrupt each other's results.
@@ -325,6 +330,18 @@ PKV_API pkv_status paged_decode_attn_fp8_noalloc(const uint16_t* q, const uint8_
 
 /* Bytes of the built-in scratch used by paged_decode_attn_fp8_noalloc. */
 PKV_API size_t paged_decode_attn_fp8_noalloc_scratch_bytes(void);
+
+/*
+ * paged_decode_attn_fp8_noalloc_status -- enqueues on `stream` a copy of the
+ * current device's built-in scratch status word (4 bytes) to status_out,
+ * host or device memory.  The word is the one paged_decode_attn_fp8 reports
+ * in its workspace: 0, or 1 if an internal bounded wait expired in the last
+ * no-allocation call on that device.  The copy is stream-ordered: issue it
+ * after the call on the same stream and read status_out once the stream has
+ * finished (a pageable host destination makes the copy synchronous).
+ * Allocates nothing.  Returns PKV_ERR_INVALID_ARG if status_out is NULL.
+ */
+PKV_API pkv_status paged_decode_attn_fp8_noalloc_status(uint32_t* status_out, void* stream);
 
 /*
  * int4_dequant_gemv -- y = x W^T with W stored as 4-bit integer codes and

@@ -84,6 +84,8 @@ def _load():
         lib.paged_decode_attn_fp8_noalloc.restype = i32
         lib.paged_decode_attn_fp8_noalloc_scratch_bytes.argtypes = []
         lib.paged_decode_attn_fp8_noalloc_scratch_bytes.restype = sz
+        lib.paged_decode_attn_fp8_noalloc_status.argtypes = [P, P]
+        lib.paged_decode_attn_fp8_noalloc_status.restype = i32
         lib.paged_decode_attn_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
         lib.paged_decode_attn_workspace_size.restype = sz
         lib.pkv_last_error.argtypes = []
@@ -354,6 +356,18 @@ def paged_decode_attn_fp8_noalloc(q, k_cache, v_cache, k_scale, v_scale, page_ta
 
 def noalloc_scratch_bytes() -> int:
     return int(_load().paged_decode_attn_fp8_noalloc_scratch_bytes())
+
+
+def noalloc_status(stream=None) -> int:
+    """The built-in scratch's status word after the last no-allocation call
+    on the current device (0 = no internal wait expired).  Copies 4 bytes to
+    host memory on `stream` and waits for that copy."""
+    import numpy as np
+    word = np.zeros(1, dtype=np.uint32)
+    _check("paged_decode_attn_fp8_noalloc_status", _load().paged_decode_attn_fp8_noalloc_status(
+        ctypes.c_void_p(word.ctypes.data), _stream(stream)))
+    (torch.cuda.current_stream() if stream is None else stream).synchronize()
+    return int(word[0])
 
 
 def version() -> int:

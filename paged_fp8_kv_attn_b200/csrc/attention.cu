@@ -169,18 +169,17 @@ struct Walker {
     }
 };
 
-__device__ __forceinline__ void record_timeout(const AttnArgs& a, volatile int* cta_failed) {
-    *cta_failed = 1;
-    atomicOr(a.ws_status, 1u);
-}
 // Bounded mbarrier wait.  After a timeout in this CTA every later wait
 // returns at once, so the kernel always runs to completion; the workspace
-// status word reports the failure.
-__device__ __forceinline__ void wait_or_give_up(uint64_t* bar, uint32_t parity, const AttnArgs& a,
-                                                volatile int* cta_failed) {
+// status word (cleared by CTA 0 when the kernel starts) reports the failure.
+__device__ __forceinline__ void wait_or_give_up(uint64_t* bar, uint32_t parity,
+                                                volatile int* cta_failed, uint32_t* status) {
     if (mbar_try_wait(bar, parity)) return;   // the common case: already complete
     if (*cta_failed) return;
-    if (!mbar_wait(bar, parity)) record_timeout(a, cta_failed);
+    if (!mbar_wait(bar, parity)) {
+        *cta_failed = 1;
+        atomicOr(status, 1u);
+    }
 }
 
 // Page id of entry j of a row, read through a 32-entry window held across
@@ -239,6 +238,11 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int64_t max_tokens = static_cast<int64_t>(a.max_pages) * a.page_size;
 
     launch_dependents();
+    // The call's status word starts at zero.  Clearing it before the grid
+    // dependency wait is safe: no kernel reads it (the caller reads it in
+    // stream order, after the call), and a bounded wait of this call can only
+    // expire seconds after CTA 0, the first to be scheduled, has run this.
+    if (blockIdx.x == 0 && tid == 0) *a.ws_status = 0u;
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full_bar[s], 1);
@@ -282,11 +286,11 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int64_t NE = U < a.num_ctas ? U : a.num_ctas;
     const int64_t u_lo = (blockIdx.x < NE) ? static_cast<int64_t>(blockIdx.x) * U / NE : U;
     const int64_t u_hi = (blockIdx.x < NE) ? static_cast<int64_t>(blockIdx.x + 1) * U / NE : U;
+    const int run0 = warp_base + incl - local;   // chunks of the requests before b_lo
     {
-        int run = warp_base + incl - local;
+        int run = run0;
         for (int b = b_lo; b < b_hi; ++b) {
             const int n = walk.chunks_of(a.seq_lens[b]);
-            if (blockIdx.x == 0) a.ws_prefix[b] = run;
             if (n > 0 && u_lo < u_hi && static_cast<int64_t>(IPR) * run <= u_lo &&
                 u_lo < static_cast<int64_t>(IPR) * (run + n)) {
                 scratch[8] = b;
@@ -294,10 +298,25 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
             run += n;
         }
-        if (blockIdx.x == 0 && tid == 0) a.ws_prefix[B] = total;
     }
+    // Block 0 publishes the chunk offsets for the merge kernel only after the
+    // grid-dependency wait: until then the previous call's merge kernel (same
+    // workspace, same stream) may still be reading them.
+    auto publish_prefix = [&]() {
+        if (blockIdx.x != 0) return;
+        int run = run0;
+        for (int b = b_lo; b < b_hi; ++b) {
+            a.ws_prefix[b] = run;
+            run += walk.chunks_of(a.seq_lens[b]);
+        }
+        if (tid == 0) a.ws_prefix[B] = total;
+    };
     __syncthreads();
-    if (u_lo >= u_hi) return;
+    if (u_lo >= u_hi) {
+        grid_dependency_wait();
+        publish_prefix();
+        return;
+    }
     walk.init(scratch[8], scratch[9], u_lo, u_hi);
 
     const int P = a.page_size;
@@ -341,6 +360,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
         }
         grid_dependency_wait();
+        publish_prefix();
         // A segment's abort flag and first page-table window are loaded one
         // segment ahead, so the first TMA of a segment waits on no load.
         auto load_meta = [&](const Segment& sg, PageWindow& w) {
@@ -375,7 +395,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
             for (int ch = s.c0; ch < s.c1; ++ch, ++it) {
                 const int stage = it % S;
                 if (it >= static_cast<uint32_t>(S)) {
-                    if (lane == 0) wait_or_give_up(&empty_bar[stage], ((it / S) + 1) & 1, a, cta_failed);
+                    if (lane == 0) wait_or_give_up(&empty_bar[stage], ((it / S) + 1) & 1, cta_failed, a.ws_status);
                     __syncwarp();
                 }
                 const uint32_t kdst = smem_addr(smem + stage * C::kStageBytes);
@@ -435,6 +455,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
     // the GQA group (kNB n-blocks of 8).  P is moved from the S accumulator
     // layout into the PV B-operand layout with an in-register 8x8 transpose.
     grid_dependency_wait();
+    publish_prefix();
     const int g = lane >> 2;   // MMA group id
     const int c = lane & 3;    // thread in group
     const int G = a.group;
@@ -604,7 +625,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
         for (int ch = s.c0; ch < s.c1; ++ch, ++it) {
             const int stage = it % S;
-            wait_or_give_up(&full_bar[stage], (it / S) & 1, a, cta_failed);
+            wait_or_give_up(&full_bar[stage], (it / S) & 1, cta_failed, a.ws_status);
             poisoned |= stage_bad_rd[stage];
             const int n_valid = min(kChunkTokens, s.L - ch * kChunkTokens);
             const bool tail = n_valid < kChunkTokens;
@@ -948,6 +969,7 @@ attn_merge_kernel(const AttnArgs a) {
     __shared__ int s_dead;
     launch_dependents();
     grid_dependency_wait();
+    const int tid = threadIdx.x;
     constexpr int kGroups = 16 / kHPC;       // CTAs per item
     const int IPR = a.items_per_req;
     const int item = blockIdx.x / kGroups;
@@ -956,7 +978,6 @@ attn_merge_kernel(const AttnArgs a) {
     const int hq0 = (blockIdx.x % kGroups) * kHPC;   // this CTA's first head of the item
     if (hq0 >= G) return;
     const int NH = min(kHPC, G - hq0);       // this CTA's heads
-    const int tid = threadIdx.x;
     const int64_t head0 = static_cast<int64_t>(b) * a.num_q_heads + h * G + hq0;
     const int32_t pre = a.ws_prefix[b];
     const int32_t nxt = a.ws_prefix[b + 1];

@@ -249,6 +249,15 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 }
 
 // bf16x2 (q_even, q_odd) of the two codes at bits 0-3 and 16-19 of v.
+// Method: the exponent-bias ("magic number") integer-to-float conversion.
+// A small integer placed in the low mantissa bits of a float whose exponent
+// makes one mantissa unit worth 1 reads as (magic + integer); subtracting
+// the magic leaves the integer exactly.  Its use for 4-bit weight codes is
+// described by Kim et al., "Who Says Elephants Can't Run: Bringing Large
+// Scale MoE Models into Cloud Scale Production" (2022).  Here the magic is
+// 128 in bf16 (one mantissa unit = 1 at exponent 7); flipping bit 3 of the
+// signed nibble maps q in [-8, 7] to q + 8 in [0, 15], so the float reads
+// 128 + 8 + q and one FMA subtracts 136.
 __device__ __forceinline__ uint32_t int4_pair_to_bf16x2(uint32_t v) {
     uint32_t t;   // (v & 0x000F000F) ^ 0x43084308: mantissa = nibble ^ 8 = q + 8 under 2^7
     asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(t) : "r"(v), "r"(0x000F000Fu), "r"(0x43084308u));

@@ -19,7 +19,7 @@ struct AttnArgs {
     const uint8_t* abort;       // [B] or null
     uint16_t* out;              // [B][Hq][D] bf16
     float* lse;                 // [B][Hq]
-    uint32_t* ws_status;        // workspace word 0
+    uint32_t* ws_status;        // workspace word 0 (cleared by CTA 0 of each call)
     int32_t* ws_prefix;         // [B + 1] chunk offsets (written by CTA 0)
     float* ws_ml;               // [slots][G][2]  (running max in log2 units, sum)
     float* ws_o;                // [slots][G][D]  (unnormalised, V scale applied)

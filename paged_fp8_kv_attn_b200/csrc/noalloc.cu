@@ -91,15 +91,32 @@ extern "C" PKV_API pkv_status paged_decode_attn_fp8_noalloc(
     void* scratch = nullptr;
     pkv_status st = scratch_for_current_device(&scratch);
     if (st != PKV_OK) return st;
-    // The array keeps the previous call's contents; only the status word has
-    // to start at zero (the kernels write everything else before reading it).
-    cudaError_t e = cudaMemsetAsync(scratch, 0, sizeof(uint32_t), static_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) {
-        pkv::set_last_error("paged_decode_attn_fp8_noalloc: clearing the status word failed");
-        return PKV_ERR_CUDA;
-    }
+    // The array keeps the previous call's contents; the kernels write every
+    // word they read, the status word included, before reading it.
     return paged_decode_attn_fp8(q, k_cache, v_cache, k_scale, v_scale, page_table, max_pages,
                                  seq_lens, batch, num_q_heads, num_kv_heads, head_dim, page_size,
                                  num_pages, sm_scale, abort, out, lse, scratch,
                                  kNoAllocScratchBytes, num_ctas, stream);
+}
+
+extern "C" PKV_API pkv_status paged_decode_attn_fp8_noalloc_status(uint32_t* status_out,
+                                                                  void* stream) {
+    if (status_out == nullptr) {
+        pkv::set_last_error("paged_decode_attn_fp8_noalloc_status: status_out is NULL");
+        return PKV_ERR_INVALID_ARG;
+    }
+    void* scratch = nullptr;
+    pkv_status st = scratch_for_current_device(&scratch);
+    if (st != PKV_OK) return st;
+    // word 0 of the scratch is the status word of the attention workspace
+    cudaError_t e = cudaMemcpyAsync(status_out, scratch, sizeof(uint32_t), cudaMemcpyDefault,
+                                    static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        char buf[256];
+        snprintf(buf, sizeof buf, "paged_decode_attn_fp8_noalloc_status: cudaMemcpyAsync: %s",
+                 cudaGetErrorString(e));
+        pkv::set_last_error(buf);
+        return PKV_ERR_CUDA;
+    }
+    return PKV_OK;
 }

@@ -72,6 +72,10 @@ def test_host_validation_without_a_gpu(lib):
     assert lib.paged_decode_attn_workspace_size(0, 4, 6, 4, 64, 10) == 0
     # explicit grid: size is computable without a device
     assert lib.paged_decode_attn_workspace_size(0, 4, 64, 8, 128, 296) > 0
+    # the no-allocation status copy needs a destination
+    assert lib.paged_decode_attn_fp8_noalloc_status(None, None) == 1
+    assert b"status_out" in lib.pkv_last_error()
+
 
 
 def test_int4_gemv_host_validation_without_a_gpu(lib):

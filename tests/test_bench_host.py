@@ -66,21 +66,68 @@ def test_reference_arm_line_shape(monkeypatch):
         threads = 3
 
         def __init__(self, requests, seed=2):
+            self.requests = requests
             self.wl = type("W", (), {"num_kv_heads": 8})()
 
-        def step(self, n_items=None):
-            return 0.5, 8
-
-        def tokens_per_s(self, seconds, n):
-            return bench.HEADLINE_BATCH / (seconds / n * 512)
+        def step(self, n_items=None, threads=None):
+            return (0.05, 1) if n_items == 1 else (0.5, 8 * self.requests)
 
     monkeypatch.setattr(bench, "OracleSampler", FakeSampler)
+    monkeypatch.setattr(bench.os, "cpu_count", lambda: 16)
     args = type("A", (), {"warmup": 3, "steps": 2})()
     line = bench.reference_arm(args, 0, 1)
     assert line["impl"] == "reference"
+    # 16 cores -> 2 requests (16 items) per step; a step of 0.5 s -> 4 tokens/s
+    assert line["value"] == 4.0 and line["ms_per_step"] == 500.0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 3
+    assert line["cpu_baseline"]["value"] == line["value"]
+    # one item on one thread in 0.05 s -> a request (8 items) in 0.4 s
+    assert line["cpu_baseline"]["single_thread"]["value"] == 2.5
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+    # the same workload description as the GPU arm
+    assert line["config"] == bench.headline_config(1)
     assert bench.reference_arm(args, 1, 2) is None
+
+
+def test_oracle_requests_cover_every_core():
+    assert bench.oracle_requests_per_step(1) == 1
+    assert bench.oracle_requests_per_step(8) == 1
+    assert bench.oracle_requests_per_step(9) == 2
+    assert bench.oracle_requests_per_step(16) == 2
+    assert bench.oracle_requests_per_step(96) == 12
+
+
+def test_paired_overhead_median_and_interval():
+    import numpy as np
+    rng = np.random.Generator(np.random.PCG64(1))
+    b = 100.0 + rng.normal(0, 1.0, 400)
+    a = b * 1.02 + rng.normal(0, 0.2, 400)          # +2% with paired noise
+    med, lo, hi = bench.paired_overhead(a, b)
+    assert lo <= med <= hi
+    assert 1.9 < med < 2.1 and lo > 1.8 and hi < 2.2
+    # identical timings: zero with a zero-width interval
+    med, lo, hi = bench.paired_overhead(b, b)
+    assert med == lo == hi == 0.0
+    # seeded: repeatable
+    assert bench.paired_overhead(a, b) == bench.paired_overhead(a, b)
+
+
+def test_measure_overhead_adds_pairs_while_the_interval_straddles_the_bound(monkeypatch):
+    import numpy as np
+    rng = np.random.Generator(np.random.PCG64(2))
+    calls = []
+
+    def fake_time_pair(fa, fb, steps, warmup, flush=None):
+        calls.append(steps)
+        b = list(100.0 + rng.normal(0, 3.0, steps))
+        a = [x * 1.01 for x in b]                      # exactly +1%: always straddles
+        a = [x + rng.normal(0, 3.0) for x in a]
+        return 0.0, 0.0, a, b
+
+    monkeypatch.setattr(bench, "time_pair", fake_time_pair)
+    r = bench.measure_overhead(None, None, 3, pairs=100, max_pairs=400)
+    assert r["pairs"] == 400 and sum(calls) == 400
+    assert r["ci95_pct"][0] <= r["median_pct"] <= r["ci95_pct"][1]
 
 
 def test_unique_kv_tokens_counts_shared_pages_once():

@@ -251,8 +251,9 @@ def test_attention_small_all_items(cuda_device, case, kv):
 @pytest.mark.parametrize("kv", ["fp8", "bf16"])
 def test_attention_workspace_reused_across_calls(cuda_device, kv):
     """One workspace serves consecutive calls with different grids and a
-    different batch: the per-item arrival counters that pick the CTA merging
-    a split item must be back at zero after every call."""
+    different batch.  The workspace holds the status word, the per-request
+    chunk offsets and the partial (m, l) and O slots; every call rewrites what
+    it reads, so no clearing is needed."""
     wl1 = workloads.custom([3000, 70, 9000, 1, 640], page_size=64, num_q_heads=64, num_kv_heads=8,
                            head_dim=128, seed=41, spare_pages=2)
     wl2 = workloads.custom([129] * 9 + [2000], page_size=64, num_q_heads=64, num_kv_heads=8,
@@ -276,6 +277,47 @@ def test_attention_workspace_reused_across_calls(cuda_device, kv):
         out, lse = db.outputs()
         compare(wl, items, out, lse, ref[0], ref[1], label=f"{kv} B={wl.batch} ctas={ctas}")
         assert pkv.workspace_status(ws) == 0
+
+
+@pytest.mark.parametrize("kv", ["fp8", "bf16"])
+def test_attention_workspace_back_to_back_without_sync(cuda_device, kv):
+    """Calls on one stream that share a workspace, with different lengths and
+    batches and no synchronisation between them (each call's kernels may be
+    scheduled while the previous call's merge still runs): every output must
+    match the oracle.  The workspace starts filled with 0xFF, which the calls
+    must not need cleared, and the status word must read 0 afterwards."""
+    shapes = ([3000, 70, 9000, 1, 640], [129] * 9 + [2000], [64, 65, 8192, 300, 4097, 1, 2, 33],
+              [5000, 17])
+    wls = [workloads.custom(lens, page_size=64, num_q_heads=64, num_kv_heads=8, head_dim=128,
+                            seed=70 + i, spare_pages=2) for i, lens in enumerate(shapes)]
+    dbs = [DeviceBatch(wl, kv_dtype=kv) for wl in wls]
+    n = max(pkv.paged_decode_attn_workspace_size(db.kv_code, wl.batch, 64, 8, 128, 0)
+            for db, wl in zip(dbs, wls))
+    ws = torch.full((n,), 0xFF, dtype=torch.uint8, device=dbs[0].q.device)
+    for db in dbs:
+        db.ws = ws
+        db.append(use_abort=False)
+    torch.cuda.synchronize()
+    outs = []
+    for rnd in range(2):
+        for db in dbs:
+            out = torch.full_like(db.out, float("nan"))
+            lse = torch.full_like(db.lse, float("nan"))
+            db.out, db.lse = out, lse
+            db.attend(use_abort=False)       # no synchronisation between calls
+            outs.append((db, out, lse))
+    torch.cuda.synchronize()
+    assert pkv.workspace_status(ws) == 0
+    refs = {}
+    for db, out, lse in outs:
+        wl = db.wl
+        items = list(range(wl.batch * 8))
+        if id(db) not in refs:
+            refs[id(db)] = oracle_step(wl, items, kv_dtype=kv, check=False, append=True)
+        ref = refs[id(db)]
+        o = out.float().cpu().numpy().astype(np.float64)
+        l = lse.cpu().numpy().astype(np.float64)
+        compare(wl, items, o, l, ref[0], ref[1], label=f"{kv} B={wl.batch} back-to-back")
 
 
 @pytest.mark.parametrize("kv", ["fp8", "bf16"])

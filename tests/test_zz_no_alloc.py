@@ -13,7 +13,7 @@ import torch
 import paged_fp8_kv_attn_b200 as pkv
 import workloads
 
-from _pkv_helpers import LSE_RTOL, OUT_ATOL, OUT_RTOL, DeviceBatch
+from _pkv_helpers import LSE_RTOL, OUT_ATOL, OUT_RTOL, DeviceBatch, compare, oracle_step
 
 pytestmark = pytest.mark.gpu
 
@@ -53,6 +53,27 @@ def test_noalloc_matches_workspace_call_twice(cuda_device):
         db = DeviceBatch(wl, kv_dtype="fp8")
         out_ref, lse_ref, out_na, lse_na = _run_pair(db)
         _close(out_na, lse_na, out_ref, lse_ref)
+        assert pkv.noalloc_status() == 0
+
+
+def test_noalloc_matches_the_oracle(cuda_device):
+    """The no-allocation call against the CPU oracle directly, on every item
+    of a ragged batch that splits requests over several CTAs."""
+    wl = workloads.custom([3000, 70, 9000, 1, 640, 64, 65], page_size=64, num_q_heads=64,
+                          num_kv_heads=8, head_dim=128, seed=31, device="cuda")
+    db = DeviceBatch(wl, kv_dtype="fp8")
+    items = list(range(wl.batch * wl.num_kv_heads))
+    ref_o, ref_l, _ = oracle_step(wl, items, kv_dtype="fp8", check=False, append=False)
+    for ctas in (0, 37):
+        out = torch.full_like(db.out, float("nan"))
+        lse = torch.full_like(db.lse, float("nan"))
+        pkv.paged_decode_attn_fp8_noalloc(db.q, db.k_cache, db.v_cache, wl.k_scale, wl.v_scale,
+                                          db.page_table, db.seq_lens, wl.sm_scale, out, lse,
+                                          num_ctas=ctas)
+        torch.cuda.synchronize()
+        compare(wl, items, out.float().cpu().numpy().astype(np.float64),
+                lse.cpu().numpy().astype(np.float64), ref_o, ref_l, label=f"noalloc ctas={ctas}")
+        assert pkv.noalloc_status() == 0
 
 
 def test_noalloc_with_aborted_requests(cuda_device):

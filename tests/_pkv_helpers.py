@@ -188,9 +188,18 @@ def heads_of(wl, items):
             for i in items for g in range(G)]
 
 
+# Worst tolerance margin seen by compare() per label in this process:
+# max over elements of |out - ref| / (OUT_ATOL + OUT_RTOL |ref|) (1.0 = at the
+# tolerance) and of the LSE error over its bound.  Printed in the pytest
+# terminal summary.
+MARGINS = {}
+
+
 def compare(wl, items, gpu_out, gpu_lse, ref_out, ref_lse, label=""):
-    """Element-wise comparison of the listed items; returns the max errors."""
-    worst_o = worst_l = 0.0
+    """Element-wise comparison of the listed items; returns (max |out error|,
+    max relative LSE error, worst margin), the margin being the largest
+    |out - ref| / (OUT_ATOL + OUT_RTOL |ref|) over the compared outputs."""
+    worst_o = worst_l = worst_m = worst_lm = 0.0
     for b, h in heads_of(wl, items):
         go, ro = gpu_out[b, h], ref_out[b, h]
         gl, rl = gpu_lse[b, h], ref_lse[b, h]
@@ -209,7 +218,12 @@ def compare(wl, items, gpu_out, gpu_lse, ref_out, ref_lse, label=""):
         assert lerr <= LSE_RTOL, f"{label} b={b} h={h}: lse {gl} vs {rl} (rel {lerr:.3g})"
         worst_o = max(worst_o, float(err.max()))
         worst_l = max(worst_l, lerr)
-    return worst_o, worst_l
+        worst_m = max(worst_m, float((err / (OUT_ATOL + OUT_RTOL * np.abs(ro))).max()))
+        worst_lm = max(worst_lm, lerr / LSE_RTOL)
+    key = label.split(" ")[0] if label else "unlabelled"
+    prev = MARGINS.get(key, (0.0, 0.0))
+    MARGINS[key] = (max(prev[0], worst_m), max(prev[1], worst_lm))
+    return worst_o, worst_l, worst_m
 
 
 def sample_items(wl, n, seed=0, must=()):

@@ -19,3 +19,15 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.fail("GPU test collected on a machine without CUDA")
     return torch.device("cuda:0")
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Worst tolerance margins of the GPU parity comparisons (1.0 = at the
+    tolerance: atol 1e-2 + rtol 1e-2 |ref| for outputs, 1e-4 max(1, |lse|) for
+    LSE), grouped by the first word of each comparison's label."""
+    helpers = sys.modules.get("_pkv_helpers")
+    if helpers is None or not getattr(helpers, "MARGINS", None):
+        return
+    terminalreporter.write_sep("-", "worst tolerance margins (error / tolerance)")
+    for key, (mo, ml) in sorted(helpers.MARGINS.items()):
+        terminalreporter.write_line(f"{key:>24}: out {mo:.3f}  lse {ml:.3f}")

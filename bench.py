@@ -98,8 +98,7 @@ def headline_config(world):
     kv_gb = HEADLINE_BATCH * CONTEXT * 8 * 128 * 2 / 1e9
     return {"workload": f"concurrency sweep, batch {HEADLINE_BATCH} x context {CONTEXT}, "
                         "page 64, 64 q heads / 8 kv heads, head_dim 128, FP8 E4M3 KV",
-            "step": "tag check + FP8 append (one fused kernel) + paged attention "
-                    "(partial + merge), one layer",
+            "step": "tag check + FP8 append (one fused kernel) + paged attention, one layer",
             "global_batch": world * HEADLINE_BATCH, "seq_len": CONTEXT,
             "kv_dtype": "fp8_e4m3", "parallelism": f"replicas x{world}",
             "l2": f"inputs larger than L2 ({kv_gb:.2f} GB of KV per step)"}
@@ -496,6 +495,12 @@ def gpu_arm(args, rank, world):
     # ---- roofline of the dominant kernel: the FP8 attention call ------------
     attn_bytes = attn_algorithmic_bytes(wl.seq_lens, wl.page_size, wl.num_q_heads,
                                         wl.num_kv_heads, wl.head_dim, 1)
+    import paged_fp8_kv_attn_b200 as pkv
+    clu, ctas, attn_launches = pkv.paged_decode_attn_plan(
+        pkv.PKV_KV_FP8, HEADLINE_BATCH, wl.num_q_heads, wl.num_kv_heads, wl.head_dim,
+        wl.page_table.shape[1], wl.page_size)
+    split = (f"cluster mode, {ctas} CTAs in clusters of {clu}, one launch" if clu
+             else f"split-K over {ctas} CTAs + LSE merge")
     # the call's device duration: CUDA-graph replays (no host launch gaps inside
     # the events), one event pair per replay, mean over the timed replays
     g_attn = _graph(lambda: st.attend(True))
@@ -635,7 +640,7 @@ def gpu_arm(args, rank, world):
         "step_kv_frac_of_8tbs": round(kv_bytes / (ms_per_step * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 4),
         "check_overhead_pct": overhead["median_pct"],
         "check_overhead_ci95_pct": overhead["ci95_pct"],
-        "roofline": {"kernel": "paged_decode_attn_fp8 (split-K partial + LSE merge)",
+        "roofline": {"kernel": f"paged_decode_attn_fp8 ({split})",
                      "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "peak_kind": f"{peak_kind} (copy bandwidth)",
@@ -649,7 +654,7 @@ def gpu_arm(args, rank, world):
                        "packed inputs and one D2H copy of the packed results per step, "
                        "double-buffered on two copy streams (step i+1 in and step i-1 out "
                        "while step i computes)"},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": (1 + attn_launches) * args.steps,   # check+append, then attention
         "clocks": clk,
         "int4_gemv": int4,
         "configs": configs,

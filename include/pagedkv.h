@@ -40,13 +40,14 @@
  *  - Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).
  *    Every call only enqueues work: it returns before the GPU runs it, and
  *    never synchronises.
- *  - Launch chaining: every kernel is launched with programmatic dependent
- *    launch, so it may be scheduled while the previous kernel on the stream
- *    is still running.  Each kernel waits for that kernel to finish before it
- *    touches memory that kernel may write, with one exception documented at
- *    paged_decode_attn_fp8: before waiting, attention reads q, seq_lens and
- *    page_table and prefetches K/V pages into L2 (nothing it reads before
- *    the wait reaches its outputs).
+ *  - Launch chaining: every kernel except the cluster-mode attention kernel
+ *    is launched with programmatic dependent launch, so it may be scheduled
+ *    while the previous kernel on the stream is still running.  Each kernel
+ *    waits for that kernel to finish before it touches memory that kernel
+ *    may write, with one exception documented at paged_decode_attn_fp8:
+ *    before waiting, attention reads q, seq_lens and page_table and
+ *    prefetches K/V pages into L2 (nothing it reads before the wait reaches
+ *    its outputs).
  *  - Errors: a status code is returned.  Invalid arguments are detected on
  *    the host before anything is enqueued (PKV_ERR_INVALID_ARG,
  *    PKV_ERR_WORKSPACE, PKV_ERR_UNSUPPORTED); a failed launch returns
@@ -220,11 +221,12 @@ PKV_API pkv_status kv_requant_pages_fp8(const uint16_t* src_pool, int32_t src_nu
 /*
  * paged_decode_attn_workspace_size -- bytes of device workspace the
  * attention calls need for these sizes.  kv_dtype is PKV_KV_FP8 or
- * PKV_KV_BF16; num_ctas is the split-K grid size passed to the attention
- * call (0 = the default, one full wave of resident CTAs on the current
- * device).  Returns 0 on invalid arguments (see pkv_last_error).  The
- * workspace holds a status word, the per-request chunk offsets and the
- * split-K partial results.  Its first 4 bytes are a status word that every
+ * PKV_KV_BF16; num_ctas is the value passed to the attention call (0 = the
+ * default; > 0 a split-K grid of that many CTAs; -C, C in 1..16, cluster
+ * mode, which needs no more than the default).  Returns 0 on invalid
+ * arguments (see pkv_last_error).  The
+ * workspace holds a status word and the split-K partial results.  Its
+ * first 4 bytes are a status word that every
  * attention call writes: 0, or 1 if an internal bounded wait expired in that
  * call (never expected; the outputs are then unreliable).  The caller may
  * read it once the stream has finished the call.
@@ -232,6 +234,23 @@ PKV_API pkv_status kv_requant_pages_fp8(const uint16_t* src_pool, int32_t src_nu
 PKV_API size_t paged_decode_attn_workspace_size(int32_t kv_dtype, int32_t batch, int32_t num_q_heads,
                                         int32_t num_kv_heads, int32_t head_dim,
                                         int32_t num_ctas);
+
+/*
+ * paged_decode_attn_plan -- the work split that paged_decode_attn_fp8
+ * (kv_dtype PKV_KV_FP8) or paged_decode_attn_bf16 (PKV_KV_BF16) chooses for
+ * these sizes and this num_ctas on the current device, without launching
+ * anything: *cluster_size = 0 for split-K (a partial kernel and a merge
+ * kernel), C > 0 for cluster mode (one kernel of clusters of C CTAs);
+ * *ctas = CTAs of the partial kernel; *launches = kernels one call launches
+ * (2 or 1).  The choice depends only on these arguments and the device, never
+ * on the device-side lengths.  Returns PKV_ERR_INVALID_ARG /
+ * PKV_ERR_UNSUPPORTED for arguments the attention call would reject.
+ */
+PKV_API pkv_status paged_decode_attn_plan(int32_t kv_dtype, int32_t batch, int32_t num_q_heads,
+                                          int32_t num_kv_heads, int32_t head_dim,
+                                          int32_t max_pages, int32_t page_size, int32_t num_ctas,
+                                          int32_t* cluster_size, int32_t* ctas,
+                                          int32_t* launches);
 
 /*
  * paged_decode_attn_fp8 -- decode attention of one new query token per
@@ -257,17 +276,29 @@ PKV_API size_t paged_decode_attn_workspace_size(int32_t kv_dtype, int32_t batch,
  * paged_decode_attn_workspace_size(PKV_KV_FP8, ...) bytes, 256-byte
  * aligned, not shared with a concurrently running attention call; its
  * contents need no initialisation.  Calls issued back to back on one stream
- * may share a workspace, with no synchronisation between them: a call's
- * kernels write the workspace only after the previous kernel on the stream
- * has finished.  num_ctas: split-K grid size (0 = default); any value >= 1
- * gives the same result up to rounding.
+ * may share a workspace, with no synchronisation between them: apart from
+ * clearing the status word (which no kernel reads), a call's kernels write
+ * the workspace only after the previous kernel on the stream has finished.
+ * num_ctas selects the work split (every choice gives the
+ * same result up to rounding):
+ *   0     the library chooses (cluster mode when the batch has no more
+ *         (request, KV-head) items than the GPU holds resident CTAs, split-K
+ *         over one wave otherwise);
+ *   N > 0 split-K over N CTAs;
+ *   -C    cluster mode with clusters of C CTAs, 1 <= C <= 16
+ *         (PKV_ERR_UNSUPPORTED if the device cannot run that cluster size).
  *
- * Work split: the (request, KV head, 64-token chunk) units are divided
- * evenly over the CTAs of one persistent wave; a request split over several
- * CTAs is combined by a log-sum-exp merge kernel.  Before its grid
- * dependency wait the kernel reads q, seq_lens and page_table and prefetches
- * its first K/V tiles into L2; everything else (abort, the cache contents)
- * is read after the preceding kernel on the stream has finished.
+ * Work split.  Split-K: the (request, KV head, 64-token chunk) units are
+ * divided evenly over the CTAs of one persistent wave, and a request split
+ * over several CTAs is combined by a log-sum-exp merge kernel (a second
+ * launch).  Cluster mode: one launch of K thread-block clusters of C CTAs;
+ * cluster k owns whole items, whose units its C CTAs divide evenly, and the
+ * CTAs of a cluster combine the partial results of the items they share in
+ * distributed shared memory; no merge kernel runs and the workspace is used
+ * only for its status word.  Before its grid dependency wait the kernel
+ * reads q, seq_lens and page_table and prefetches its first K/V tiles into
+ * L2; everything else (abort, the cache contents) is read after the
+ * preceding kernel on the stream has finished.
  */
 PKV_API pkv_status paged_decode_attn_fp8(const uint16_t* q, const uint8_t* k_cache,
                                  const uint8_t* v_cache, float k_scale, float v_scale,

@@ -86,6 +86,10 @@ def _load():
         lib.paged_decode_attn_fp8_noalloc_scratch_bytes.restype = sz
         lib.paged_decode_attn_fp8_noalloc_status.argtypes = [P, P]
         lib.paged_decode_attn_fp8_noalloc_status.restype = i32
+        pi32 = ctypes.POINTER(i32)
+        lib.paged_decode_attn_plan.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, pi32,
+                                               pi32, pi32]
+        lib.paged_decode_attn_plan.restype = i32
         lib.paged_decode_attn_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
         lib.paged_decode_attn_workspace_size.restype = sz
         lib.pkv_last_error.argtypes = []
@@ -282,6 +286,17 @@ def alloc_workspace(kv_dtype, batch, num_q_heads, num_kv_heads, head_dim, num_ct
     n = paged_decode_attn_workspace_size(kv_dtype, batch, num_q_heads, num_kv_heads, head_dim,
                                          num_ctas)
     return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def paged_decode_attn_plan(kv_dtype, batch, num_q_heads, num_kv_heads, head_dim, max_pages,
+                           page_size, num_ctas=0):
+    """The attention call's work split on the current device:
+    (cluster_size, ctas, launches); cluster_size 0 means split-K + merge."""
+    out = [ctypes.c_int32(0) for _ in range(3)]
+    _check("paged_decode_attn_plan", _load().paged_decode_attn_plan(
+        int(kv_dtype), int(batch), int(num_q_heads), int(num_kv_heads), int(head_dim),
+        int(max_pages), int(page_size), int(num_ctas), *[ctypes.byref(o) for o in out]))
+    return tuple(int(o.value) for o in out)
 
 
 def workspace_status(workspace) -> int:

@@ -47,6 +47,8 @@ struct DeviceInfo {
     bool ready = false;
     int sms = 0;
     int occupancy[2][2][2][2] = {};   // [fp8][d128][gp16][two KV heads per item]
+    // resident clusters of each size (index = cluster size; -1 = not queried)
+    int clusters[2][2][2][2][pkv::kMaxCluster + 1];
 };
 std::mutex g_dev_mutex;
 DeviceInfo g_dev[kMaxDevices];
@@ -74,6 +76,7 @@ pkv_status device_info(const DeviceInfo** out) {
                         e = pkv::attn_occupancy(fp8, hd, gpad, kvh, &blocks);
                         if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
                         info.occupancy[f][d][gp][h2] = blocks < 1 ? 1 : blocks;
+                        for (int c = 0; c <= pkv::kMaxCluster; ++c) info.clusters[f][d][gp][h2][c] = -1;
                     }
         info.ready = true;
     }
@@ -82,6 +85,60 @@ pkv_status device_info(const DeviceInfo** out) {
 }
 
 int group_pad_of(int group) { return group <= 8 ? 8 : 16; }
+
+// Clusters of `size` CTAs of this attention variant that fit on the device at
+// once (queried once per device, variant and size).
+pkv_status max_clusters(bool fp8, int head_dim, int group, int kv_per_item, int size, int* out) {
+    const DeviceInfo* cinfo = nullptr;
+    pkv_status st = device_info(&cinfo);
+    if (st != PKV_OK) return st;
+    DeviceInfo& info = const_cast<DeviceInfo&>(*cinfo);
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    int& slot = info.clusters[fp8 ? 1 : 0][head_dim == 128][group > 8][kv_per_item == 2][size];
+    if (slot < 0) {
+        int n = 0;
+        cudaError_t e = pkv::attn_max_clusters(fp8, head_dim, group_pad_of(group), kv_per_item,
+                                               size, &n);
+        if (e != cudaSuccess) {
+            cudaGetLastError();   // a refused shape is an answer, not a sticky error
+            n = 0;
+        }
+        slot = n;
+    }
+    *out = slot;
+    return PKV_OK;
+}
+
+// Cluster mode for `items` work items: cluster size C and K clusters, each
+// owning ceil(items / K) or fewer whole items.  With `forced` > 0 the size is
+// given; otherwise the size maximising C * items / (items per cluster) -- the
+// CTAs kept busy, discounted by the imbalance of whole items per cluster --
+// over 2..kMaxCluster.  Among sizes that tie, the largest portable one (at
+// most 8) wins: more CTAs share each cluster's items, which evens out
+// requests of unequal length.  Returns C = 0 when no cluster shape fits.
+pkv_status choose_clusters(bool fp8, int head_dim, int group, int kv_per_item, int64_t items,
+                           int forced, int* size, int* count) {
+    *size = 0;
+    *count = 0;
+    double best = 0.0;
+    const int c_lo = forced > 0 ? forced : 2;
+    const int c_hi = forced > 0 ? forced : pkv::kMaxCluster;
+    for (int c = c_lo; c <= c_hi; ++c) {
+        int kmax = 0;
+        pkv_status st = max_clusters(fp8, head_dim, group, kv_per_item, c, &kmax);
+        if (st != PKV_OK) return st;
+        if (kmax <= 0) continue;
+        const int64_t k = std::min<int64_t>(items, kmax);
+        const int64_t per = (items + k - 1) / k;            // items of the fullest cluster
+        const double score = static_cast<double>(c) * static_cast<double>(items) / per;
+        if (score > best || (score == best && c <= 8)) {
+            best = score;
+            *size = c;
+            *count = static_cast<int>((items + per - 1) / per);
+        }
+    }
+    return PKV_OK;
+}
 
 pkv_status default_ctas(bool fp8, int head_dim, int group, int kv_per_item, int* ctas) {
     const DeviceInfo* info = nullptr;
@@ -173,36 +230,22 @@ pkv_status check_common_kv(int32_t batch, int32_t num_kv_heads, int32_t head_dim
     return PKV_OK;
 }
 
-pkv_status attn_impl(bool fp8, const uint16_t* q, const void* k_cache, const void* v_cache,
-                     float k_scale, float v_scale, const int32_t* page_table, int32_t max_pages,
-                     const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
-                     int32_t num_kv_heads, int32_t head_dim, int32_t page_size, int32_t num_pages,
-                     float sm_scale, const uint8_t* abort, uint16_t* out, float* lse,
-                     void* workspace, size_t workspace_bytes, int32_t num_ctas, void* stream) {
-    pkv_status st = check_common_kv(batch, num_kv_heads, head_dim, page_size, num_pages, max_pages);
-    if (st != PKV_OK) return st;
-    if (num_q_heads < 1 || num_q_heads % num_kv_heads != 0)
-        return fail(PKV_ERR_INVALID_ARG, "num_q_heads (%d) must be a positive multiple of "
-                    "num_kv_heads (%d)", num_q_heads, num_kv_heads);
-    const int group = num_q_heads / num_kv_heads;
-    if (group > 16) return fail(PKV_ERR_UNSUPPORTED, "GQA group %d > 16 not supported", group);
-    if (!(std::isfinite(sm_scale)))
-        return fail(PKV_ERR_INVALID_ARG, "sm_scale must be finite");
-    if (fp8 && (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) ||
-                !std::isfinite(v_scale)))
-        return fail(PKV_ERR_INVALID_ARG, "k_scale and v_scale must be finite and > 0");
-    if (num_ctas < 0) return fail(PKV_ERR_INVALID_ARG, "num_ctas must be >= 0");
-    if (batch == 0) return PKV_OK;
-    if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !out || !lse)
-        return fail(PKV_ERR_INVALID_ARG, "null pointer argument");
-    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 4) ||
-        !aligned(lse, 4) || !aligned(page_table, 4) || !aligned(seq_lens, 4))
-        return fail(PKV_ERR_INVALID_ARG, "misaligned pointer (q and caches need 16 bytes)");
-    if (!workspace || !aligned(workspace, 256))
-        return fail(PKV_ERR_WORKSPACE, "workspace must be non-null and 256-byte aligned");
+// The work split of one attention call (see paged_decode_attn_plan).
+struct AttnPlan {
+    int kv_per_item;      // KV heads per work item the kernel uses
+    int ws_kv_per_item;   // the one the workspace is sized for
+    int grid;             // split-K grid (also sizes the workspace)
+    int cluster;          // 0: split-K + merge; C > 0: clusters of C CTAs
+    int nclusters;
+};
 
-    const int kv_per_item = pkv::kv_heads_per_item(fp8, num_kv_heads, group);
-    int grid = num_ctas;
+pkv_status plan_attention(bool fp8, int32_t batch, int32_t num_kv_heads, int32_t group,
+                          int32_t head_dim, int32_t max_pages, int32_t page_size,
+                          int32_t num_ctas, AttnPlan* plan) {
+    pkv_status st = PKV_OK;
+    int kv_per_item = pkv::kv_heads_per_item(fp8, num_kv_heads, group);
+    plan->ws_kv_per_item = kv_per_item;
+    int grid = num_ctas > 0 ? num_ctas : 0;
     if (grid == 0) {
         // one wave of resident CTAs, but no more than leaves each CTA about
         // eight 64-token chunks of the largest batch the page table allows
@@ -223,8 +266,81 @@ pkv_status attn_impl(bool fp8, const uint16_t* q, const void* k_cache, const voi
         st = device_info(&info);  // sets the shared-memory attribute
         if (st != PKV_OK) return st;
     }
+    plan->grid = grid;
+    // Cluster mode (no merge kernel): the library's choice (num_ctas == 0)
+    // when the batch has no more items than one wave of CTAs (measured on
+    // B200: faster than split-K plus merge at every such size of the
+    // concurrency sweep; larger batches, which can be ragged, keep the
+    // balanced split-K partition), or requested with num_ctas = -C.  When
+    // even clusters of the largest size
+    // would leave SMs idle with two KV heads per item (a handful of
+    // requests), the library's choice takes one KV head per item, which
+    // doubles the CTAs (cluster mode needs the workspace for its status word
+    // only, so the workspace size does not depend on this).
+    int64_t items = static_cast<int64_t>(batch) * (num_kv_heads / kv_per_item);
+    int cluster = 0, nclusters = 0;
+    if (num_ctas < 0 || (num_ctas == 0 && items <= grid)) {
+        if (num_ctas == 0 && kv_per_item == 2) {
+            const DeviceInfo* info = nullptr;
+            st = device_info(&info);
+            if (st != PKV_OK) return st;
+            if (items * pkv::kMaxCluster <= info->sms) {
+                kv_per_item = 1;
+                items *= 2;
+            }
+        }
+        st = choose_clusters(fp8, head_dim, group, kv_per_item, items,
+                             num_ctas < 0 ? -num_ctas : 0, &cluster, &nclusters);
+        if (st != PKV_OK) return st;
+        if (cluster == 0 && num_ctas < 0)
+            return fail(PKV_ERR_UNSUPPORTED, "clusters of %d CTAs do not fit on this device",
+                        -num_ctas);
+    }
+    plan->kv_per_item = kv_per_item;
+    plan->cluster = cluster;
+    plan->nclusters = nclusters;
+    return PKV_OK;
+}
+
+pkv_status attn_impl(bool fp8, const uint16_t* q, const void* k_cache, const void* v_cache,
+                     float k_scale, float v_scale, const int32_t* page_table, int32_t max_pages,
+                     const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
+                     int32_t num_kv_heads, int32_t head_dim, int32_t page_size, int32_t num_pages,
+                     float sm_scale, const uint8_t* abort, uint16_t* out, float* lse,
+                     void* workspace, size_t workspace_bytes, int32_t num_ctas, void* stream) {
+    pkv_status st = check_common_kv(batch, num_kv_heads, head_dim, page_size, num_pages, max_pages);
+    if (st != PKV_OK) return st;
+    if (num_q_heads < 1 || num_q_heads % num_kv_heads != 0)
+        return fail(PKV_ERR_INVALID_ARG, "num_q_heads (%d) must be a positive multiple of "
+                    "num_kv_heads (%d)", num_q_heads, num_kv_heads);
+    const int group = num_q_heads / num_kv_heads;
+    if (group > 16) return fail(PKV_ERR_UNSUPPORTED, "GQA group %d > 16 not supported", group);
+    if (!(std::isfinite(sm_scale)))
+        return fail(PKV_ERR_INVALID_ARG, "sm_scale must be finite");
+    if (fp8 && (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) ||
+                !std::isfinite(v_scale)))
+        return fail(PKV_ERR_INVALID_ARG, "k_scale and v_scale must be finite and > 0");
+    if (num_ctas < -pkv::kMaxCluster)
+        return fail(PKV_ERR_INVALID_ARG, "num_ctas must be >= %d (got %d)", -pkv::kMaxCluster,
+                    num_ctas);
+    if (batch == 0) return PKV_OK;
+    if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !out || !lse)
+        return fail(PKV_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 4) ||
+        !aligned(lse, 4) || !aligned(page_table, 4) || !aligned(seq_lens, 4))
+        return fail(PKV_ERR_INVALID_ARG, "misaligned pointer (q and caches need 16 bytes)");
+    if (!workspace || !aligned(workspace, 256))
+        return fail(PKV_ERR_WORKSPACE, "workspace must be non-null and 256-byte aligned");
+
+    AttnPlan plan;
+    st = plan_attention(fp8, batch, num_kv_heads, group, head_dim, max_pages, page_size, num_ctas,
+                        &plan);
+    if (st != PKV_OK) return st;
+    const int kv_per_item = plan.kv_per_item;
+    const int grid = plan.grid;
+    const int cluster = plan.cluster, nclusters = plan.nclusters;
     const pkv::WorkspaceLayout wl =
-        pkv::workspace_layout(batch, group, num_kv_heads, kv_per_item, head_dim, grid);
+        pkv::workspace_layout(batch, group, num_kv_heads, plan.ws_kv_per_item, head_dim, grid);
     if (workspace_bytes < wl.total)
         return fail(PKV_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes,
                     wl.total);
@@ -251,7 +367,6 @@ pkv_status attn_impl(bool fp8, const uint16_t* q, const void* k_cache, const voi
     a.out = out;
     a.lse = lse;
     a.ws_status = reinterpret_cast<uint32_t*>(ws);
-    a.ws_prefix = reinterpret_cast<int32_t*>(ws + wl.prefix_off);
     a.ws_ml = reinterpret_cast<float*>(ws + wl.ml_off);
     a.ws_o = reinterpret_cast<float*>(ws + wl.o_off);
     a.batch = batch;
@@ -263,16 +378,20 @@ pkv_status attn_impl(bool fp8, const uint16_t* q, const void* k_cache, const voi
     a.group = group;
     a.page_size = page_size;
     a.num_pages = num_pages;
-    a.num_ctas = grid;
+    a.num_ctas = cluster > 0 ? cluster * nclusters : grid;
     a.box_rows = box_rows;
+    a.cluster_size = cluster;
+    a.num_clusters = nclusters;
     a.qk_scale = sm_scale * (fp8 ? k_scale : 1.f) * 1.4426950408889634f;
     a.v_scale = fp8 ? v_scale : 1.f;
 
-    cudaError_t e = pkv::launch_attn_partial(fp8, head_dim, group_pad_of(group), kv_per_item, grid,
-                                             as_stream(stream), tk, tv, a);
+    cudaError_t e = pkv::launch_attn_partial(fp8, head_dim, group_pad_of(group), kv_per_item,
+                                             a.num_ctas, as_stream(stream), tk, tv, a);
     if (e != cudaSuccess) return cuda_fail(e, "attention partial launch");
-    e = pkv::launch_attn_merge(head_dim, as_stream(stream), a);
-    if (e != cudaSuccess) return cuda_fail(e, "attention merge launch");
+    if (cluster == 0) {
+        e = pkv::launch_attn_merge(head_dim, as_stream(stream), a);
+        if (e != cudaSuccess) return cuda_fail(e, "attention merge launch");
+    }
     return PKV_OK;
 }
 
@@ -284,12 +403,11 @@ void set_last_error(const char* message) { g_last_error = message; }
 WorkspaceLayout workspace_layout(int32_t batch, int32_t group, int32_t num_kv_heads,
                                  int32_t kv_per_item, int32_t head_dim, int32_t num_ctas) {
     WorkspaceLayout l{};
-    l.prefix_off = 256;
     const size_t items = static_cast<size_t>(batch) * (num_kv_heads / kv_per_item);
     const size_t heads_per_slot = static_cast<size_t>(group) * kv_per_item;
     const size_t slots = static_cast<size_t>(num_ctas) + items;
-    l.ml_off = round_up(l.prefix_off + (static_cast<size_t>(batch) + 1) * 4, 256);
-    l.o_off = round_up(l.ml_off + slots * heads_per_slot * 2 * 4, 256);
+    l.ml_off = 256;   // after the status word
+    l.o_off = round_up(l.ml_off + slots * heads_per_slot * 4 * 4, 256);
     l.total = round_up(l.o_off + slots * heads_per_slot * head_dim * 4, 256);
     return l;
 }
@@ -477,6 +595,33 @@ pkv_status kv_requant_pages_fp8(const uint16_t* src_pool, int32_t src_num_pages,
     return PKV_OK;
 }
 
+pkv_status paged_decode_attn_plan(int32_t kv_dtype, int32_t batch, int32_t num_q_heads,
+                                  int32_t num_kv_heads, int32_t head_dim, int32_t max_pages,
+                                  int32_t page_size, int32_t num_ctas, int32_t* cluster_size,
+                                  int32_t* ctas, int32_t* launches) {
+    if (kv_dtype != PKV_KV_FP8 && kv_dtype != PKV_KV_BF16)
+        return fail(PKV_ERR_INVALID_ARG, "kv_dtype must be PKV_KV_FP8 or PKV_KV_BF16");
+    if (!cluster_size || !ctas || !launches)
+        return fail(PKV_ERR_INVALID_ARG, "null output pointer");
+    if (batch < 1) return fail(PKV_ERR_INVALID_ARG, "batch must be >= 1");
+    pkv_status st = check_common_kv(batch, num_kv_heads, head_dim, page_size, 1, max_pages);
+    if (st != PKV_OK) return st;
+    if (num_q_heads < 1 || num_q_heads % num_kv_heads != 0)
+        return fail(PKV_ERR_INVALID_ARG, "num_q_heads must be a positive multiple of num_kv_heads");
+    const int group = num_q_heads / num_kv_heads;
+    if (group > 16) return fail(PKV_ERR_UNSUPPORTED, "GQA group %d > 16 not supported", group);
+    if (num_ctas < -pkv::kMaxCluster)
+        return fail(PKV_ERR_INVALID_ARG, "num_ctas must be >= %d", -pkv::kMaxCluster);
+    AttnPlan plan;
+    st = plan_attention(kv_dtype == PKV_KV_FP8, batch, num_kv_heads, group, head_dim, max_pages,
+                        page_size, num_ctas, &plan);
+    if (st != PKV_OK) return st;
+    *cluster_size = plan.cluster;
+    *ctas = plan.cluster > 0 ? plan.cluster * plan.nclusters : plan.grid;
+    *launches = plan.cluster > 0 ? 1 : 2;
+    return PKV_OK;
+}
+
 size_t paged_decode_attn_workspace_size(int32_t kv_dtype, int32_t batch, int32_t num_q_heads,
                                         int32_t num_kv_heads, int32_t head_dim,
                                         int32_t num_ctas) {
@@ -485,7 +630,7 @@ size_t paged_decode_attn_workspace_size(int32_t kv_dtype, int32_t batch, int32_t
         return 0;
     }
     if (batch < 0 || num_kv_heads < 1 || num_q_heads < 1 || num_q_heads % num_kv_heads != 0 ||
-        !supported_head_dim(head_dim) || num_ctas < 0) {
+        !supported_head_dim(head_dim) || num_ctas < -pkv::kMaxCluster) {
         fail(PKV_ERR_INVALID_ARG, "invalid sizes for the workspace query");
         return 0;
     }
@@ -494,7 +639,7 @@ size_t paged_decode_attn_workspace_size(int32_t kv_dtype, int32_t batch, int32_t
         fail(PKV_ERR_UNSUPPORTED, "GQA group %d > 16 not supported", group);
         return 0;
     }
-    int grid = num_ctas;
+    int grid = num_ctas > 0 ? num_ctas : 0;   // cluster mode (< 0) needs no more than the default
     const bool fp8 = kv_dtype == PKV_KV_FP8;
     const int kv_per_item = pkv::kv_heads_per_item(fp8, num_kv_heads, group);
     if (grid == 0 && default_ctas(fp8, head_dim, group, kv_per_item, &grid) != PKV_OK) return 0;

@@ -75,11 +75,22 @@ struct AttnCfg {
     // only after the epilogue; otherwise it has its own buffer.
     static constexpr bool kRedInStage = kConsumerWarps * kGP * kD * 4 <= kStageBytes;
     static constexpr int kRedOff = kStages * kStageBytes;
-    static constexpr int kRedFloats = kConsumerWarps * kGP * ((kRedInStage ? 0 : kD) + 2);
+    static constexpr int kRedFloats = kConsumerWarps * kGP * ((kRedInStage ? 0 : kD) + 3);
     static constexpr int kBarOff = kRedOff + kRedFloats * 4;
     static constexpr int kFlagOff = kBarOff + 2 * kStages * 8;
     static constexpr int kScratchOff = kFlagOff + kStages * 4;
-    static constexpr int kSmemBytes = kScratchOff + 16 * 4 + 1024;  // + alignment slack
+    // Cluster mode: the partial result of one item (O[kRecHeads][kD], then
+    // (m, l, lr, 0) per head, fp32) kept in shared memory for the cluster's
+    // reduction.  A CTA's first segment uses the dedicated buffer at kRecOff;
+    // its last one a pipeline stage (all free by then).  The cluster table
+    // holds, per (rank, record), the item and the record's address.
+    static constexpr int kRecHeads = kH * kGP;
+    static constexpr int kRecBytes = kRecHeads * kD * 4 + 4 * kRecHeads * 4;
+    static constexpr int kCluOff = kScratchOff + 16 * 4;
+    static constexpr int kCluInts = 4 * kMaxCluster + 2 * kMaxCluster * kMaxCluster + 1;
+    static constexpr int kRecOff = (kCluOff + kCluInts * 4 + 15) / 16 * 16;
+    static constexpr int kSmemBytes = kRecOff + kRecBytes + 1024;  // + alignment slack
+    static_assert(kRecBytes <= kStageBytes, "a record must fit in one stage");
     // Registers per thread holding a segment's raw query words.  They are
     // loaded before the previous segment's epilogue when that adds at most
     // 16 live registers to a variant with the 2-CTA register budget (168);
@@ -207,12 +218,160 @@ struct PageWindow {
 };
 
 // ---------------------------------------------------------------------------
+// cluster mode: combine the split items inside the cluster
+// ---------------------------------------------------------------------------
+// Every CTA of the cluster, all threads, after its walk.  The records of one
+// item sit in consecutive ranks (the ranges are contiguous and increasing), so
+// in (rank, record) order each split item's records form one run; the runs'
+// outputs are spread over all threads of the cluster.  Kept out of line so
+// that nothing it needs stays live through the partial kernel's main loop.
+template <bool kFp8, int kD, int kGP, int kH>
+__device__ __noinline__ void attn_cluster_reduce(const AttnArgs& a, uint8_t* smem) {
+    using C = AttnCfg<kFp8, kD, kGP, kH>;
+    constexpr int K = kMaxCluster;
+    constexpr int kWarps = kAttnThreads / 32;
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    int* const scratch = reinterpret_cast<int*>(smem + C::kScratchOff);
+    float* const rec0 = reinterpret_cast<float*>(smem + C::kRecOff);
+    // per split item: its id, its records' cluster-window addresses (at most
+    // one per rank and record slot) and their count
+    int* const s_item = reinterpret_cast<int*>(smem + C::kCluOff);        // [2K]
+    int* const s_count = s_item + 2 * K;                                    // [2K]
+    uint32_t* const s_list = reinterpret_cast<uint32_t*>(s_count + 2 * K);  // [2K][K]
+    int* const n_split = reinterpret_cast<int*>(s_list + 2 * K * K);
+    // the arguments used below, in registers
+    const int B = a.batch, IPR = a.items_per_req, CS = a.cluster_size, NCL = a.num_clusters;
+    const int IQ = kH * a.group, Hq = a.num_q_heads;
+    const int32_t* const seq_lens = a.seq_lens;
+    uint16_t* const out = a.out;
+    float* const lse = a.lse;
+    const int64_t max_tokens = static_cast<int64_t>(a.max_pages) * a.page_size;
+    const int crank = static_cast<int>(blockIdx.x % CS);
+
+    // Requests with no chunks (invalid length) among the cluster's items
+    // produce no record: rank 0 writes their dead outputs, one warp per item,
+    // while the other CTAs of the cluster are still arriving.
+    if (crank == 0) {
+        const int cid = static_cast<int>(blockIdx.x) / CS, I = B * IPR;
+        const int i0 = static_cast<int>(static_cast<int64_t>(cid) * I / NCL);
+        const int i1 = static_cast<int>(static_cast<int64_t>(cid + 1) * I / NCL);
+        for (int item = i0 + warp; item < i1; item += kWarps) {
+            const int b = item / IPR, h = item - b * IPR;
+            const int32_t len = seq_lens[b];
+            if (len >= 1 && static_cast<int64_t>(len) <= max_tokens) continue;
+            const int64_t row0 = static_cast<int64_t>(b) * Hq + static_cast<int64_t>(h) * IQ;
+            for (int e = lane; e < IQ * kD; e += 32) out[row0 * kD + e] = 0;
+            if (lane < IQ) lse[row0 + lane] = kNegInf;
+        }
+    }
+
+    cluster_sync_all();   // every record of the cluster is written
+    if (warp == 0) {
+        // Lane e < 2 CS reads record e (rank e / 2, slot e % 2): its item and,
+        // for slot 1, the address of the rank's stage-resident record.  In
+        // this order the records of one item are consecutive (empty records
+        // aside), so the split items and their record lists follow from masks.
+        int item = -1;
+        uint32_t addr = 0;
+        if (lane < 2 * CS) {
+            const uint32_t r = static_cast<uint32_t>(lane >> 1), slot = static_cast<uint32_t>(lane & 1);
+            item = ld_cluster_s32(cluster_map(smem_addr(&scratch[5 + slot]), r));
+            const uint32_t rec1 =
+                static_cast<uint32_t>(ld_cluster_s32(cluster_map(smem_addr(&scratch[7]), r)));
+            addr = cluster_map(slot == 0 ? smem_addr(rec0) : rec1, r);
+        }
+        const uint32_t valid = __ballot_sync(0xffffffffu, item >= 0);
+        const uint32_t below = (1u << lane) - 1u;
+        // the nearest valid record before this one, and its item
+        const uint32_t vb = valid & below;
+        const int prev_lane = vb ? 31 - __clz(vb) : 0;
+        const int prev_item = __shfl_sync(0xffffffffu, item, prev_lane);
+        const bool starts = item >= 0 && (vb == 0 || prev_item != item);
+        const uint32_t starts_mask = __ballot_sync(0xffffffffu, starts);
+        if (item >= 0) {
+            const uint32_t sb = starts_mask & (below | (1u << lane));
+            const int first = 31 - __clz(sb);                  // this item's first record
+            const int j = __popc(sb) - 1;                      // its split-item index
+            const int k = __popc(valid & below & ~((1u << first) - 1u));   // position in its list
+            s_list[j * K + k] = addr;
+            if (starts) {
+                const uint32_t later = starts_mask & ~(below | (1u << lane));
+                const int next = later ? __ffs(later) - 1 : 32;
+                const uint32_t span = (next == 32 ? 0xffffffffu : ((1u << next) - 1u)) & ~below;
+                s_item[j] = item;
+                s_count[j] = __popc(valid & span);
+            }
+        }
+        if (lane == 0) *n_split = __popc(starts_mask);
+    }
+    __syncthreads();
+
+    // One warp per (split item, query head), spread over the cluster's ranks:
+    // lane k < n loads record k's (m, l, lr) (one round trip), the weights are
+    // shared by shuffles, then lane q sums output quad q over the n records
+    // with all n loads in flight (a second round trip).
+    constexpr uint32_t kMlOff = C::kRecHeads * kD * 4;   // byte offset of (m, l, lr, 0) per head
+    constexpr int kQuads = kD / 4;                       // 32 (D = 128) or 16 (D = 64)
+    const int pairs = *n_split * IQ;
+    for (int pr = crank + CS * warp; pr < pairs; pr += CS * kWarps) {
+        const int j = pr / IQ, hq = pr - j * IQ;
+        const int n = s_count[j];
+        const uint32_t* const list = s_list + j * K;
+        float4 ml = make_float4(kNegInf, 0.f, 0.f, 0.f);
+        if (lane < n) ml = ld_cluster_f32x4(list[lane] + kMlOff + 16 * hq);
+        float M = ml.x;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        const float wt = (lane < n && ml.x != kNegInf) ? exp2f(ml.x - M) : 0.f;
+        float Lsum = wt * ml.y, Lr = wt * ml.z;
+        int dead = lane < n && ml.y < 0.f;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            Lsum += __shfl_xor_sync(0xffffffffu, Lsum, off);
+            Lr += __shfl_xor_sync(0xffffffffu, Lr, off);
+        }
+        dead = __any_sync(0xffffffffu, dead);
+        const int item = s_item[j];
+        const int b = item / IPR, h = item - b * IPR;
+        const int64_t hrow = static_cast<int64_t>(b) * Hq + static_cast<int64_t>(h) * IQ + hq;
+        if (lane < kQuads) {
+            float4 x[K];
+#pragma unroll
+            for (int k = 0; k < K; ++k)
+                if (k < n) x[k] = ld_cluster_f32x4(list[k] + (hq * kD + 4 * lane) * 4);
+            float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int k = 0; k < K; ++k) {
+                const float w = __shfl_sync(0xffffffffu >> (32 - kQuads), wt, k);
+                if (k < n) {
+                    O.x += w * x[k].x;
+                    O.y += w * x[k].y;
+                    O.z += w * x[k].z;
+                    O.w += w * x[k].w;
+                }
+            }
+            uint32_t* dst = reinterpret_cast<uint32_t*>(out + hrow * kD + 4 * lane);
+            if (dead) {
+                dst[0] = 0u;
+                dst[1] = 0u;
+            } else {
+                dst[0] = pack_bf16x2(O.x / Lr, O.y / Lr);
+                dst[1] = pack_bf16x2(O.z / Lr, O.w / Lr);
+            }
+        }
+        if (lane == 0) lse[hrow] = dead ? kNegInf : (M + log2f(Lsum)) * kLn2;
+    }
+    cluster_sync_all();   // no CTA leaves while another may read its records
+}
+
+// ---------------------------------------------------------------------------
 // the split-K partial kernel
 // ---------------------------------------------------------------------------
 template <bool kFp8, int kD, int kGP, int kH>
 __global__ void __launch_bounds__(kAttnThreads, (AttnCfg<kFp8, kD, kGP, kH>::kMinBlocks))
 attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
-                    const __grid_constant__ CUtensorMap tmap_v, const AttnArgs a) {
+                    const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ AttnArgs a) {
     using C = AttnCfg<kFp8, kD, kGP, kH>;
     constexpr int S = C::kStages;
     extern __shared__ uint8_t smem_raw[];
@@ -220,7 +379,8 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     float* red_m = reinterpret_cast<float*>(smem + C::kRedOff);
     float* red_l = red_m + kConsumerWarps * kGP;
-    float* const red_o_own = red_l + kConsumerWarps * kGP;   // used when !kRedInStage
+    float* red_lr = red_l + kConsumerWarps * kGP;
+    float* const red_o_own = red_lr + kConsumerWarps * kGP;   // used when !kRedInStage
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
     uint64_t* empty_bar = full_bar + S;
     volatile int* stage_bad = reinterpret_cast<volatile int*>(smem + C::kFlagOff);
@@ -228,6 +388,10 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int* stage_bad_rd = reinterpret_cast<const int*>(smem + C::kFlagOff);
     int* scratch = reinterpret_cast<int*>(smem + C::kScratchOff);
     volatile int* cta_failed = scratch + 10;
+    // cluster mode: scratch[5], scratch[6] = item of this CTA's first / last
+    // partial record (-1: none); scratch[7] = shared address of the last one
+    float* const rec0 = reinterpret_cast<float*>(smem + C::kRecOff);
+    const bool clu = a.cluster_size > 0;
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -249,6 +413,9 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
             mbar_init(&empty_bar[s], kConsumerWarps);
         }
         *cta_failed = 0;
+        scratch[5] = -1;
+        scratch[6] = -1;
+        scratch[7] = 0;
         fence_barrier_init();
     }
 
@@ -279,14 +446,42 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
         total += t;
     }
     const int64_t U = static_cast<int64_t>(IPR) * total;
-    // The units are cut over NE = min(grid, U) CTAs, so that every CTA of the
-    // partition holds at least one unit and therefore writes the partial of
-    // every item it touches: the merge reads only slots written by this call
-    // (the rest of the grid, if any, has nothing to do).
-    const int64_t NE = U < a.num_ctas ? U : a.num_ctas;
-    const int64_t u_lo = (blockIdx.x < NE) ? static_cast<int64_t>(blockIdx.x) * U / NE : U;
-    const int64_t u_hi = (blockIdx.x < NE) ? static_cast<int64_t>(blockIdx.x + 1) * U / NE : U;
     const int run0 = warp_base + incl - local;   // chunks of the requests before b_lo
+    int64_t u_lo, u_hi;
+    if (!clu) {
+        // The units are cut over NE = min(grid, U) CTAs, so that every CTA of
+        // the partition holds at least one unit and therefore writes the
+        // partial of every item it touches: the merge reads only slots written
+        // by this call (the rest of the grid, if any, has nothing to do).
+        const int64_t NE = U < a.num_ctas ? U : a.num_ctas;
+        u_lo = (blockIdx.x < NE) ? static_cast<int64_t>(blockIdx.x) * U / NE : U;
+        u_hi = (blockIdx.x < NE) ? static_cast<int64_t>(blockIdx.x + 1) * U / NE : U;
+    } else {
+        // Cluster mode: cluster k owns the items [k I / K, (k+1) I / K) (I
+        // items, K clusters), so no item crosses a cluster; its units are cut
+        // evenly over the cluster's CTAs.  Unit offset of item i = b IPR + h:
+        // IPR * (chunks of the requests before b) + h * (chunks of b).
+        const int CS = a.cluster_size;
+        const int cid = blockIdx.x / CS;
+        const int crank = blockIdx.x % CS;
+        const int I = B * IPR;
+        const int i0 = static_cast<int>(static_cast<int64_t>(cid) * I / a.num_clusters);
+        const int i1 = static_cast<int>(static_cast<int64_t>(cid + 1) * I / a.num_clusters);
+        int run = run0;
+        for (int b = b_lo; b < b_hi; ++b) {
+            const int n = walk.chunks_of(a.seq_lens[b]);
+            if (b == i0 / IPR) { scratch[11] = run; scratch[12] = n; }
+            if (b == i1 / IPR) { scratch[13] = run; scratch[14] = n; }
+            run += n;
+        }
+        __syncthreads();
+        const int64_t c_lo = (i0 >= I) ? U : static_cast<int64_t>(IPR) * scratch[11] +
+                                                 static_cast<int64_t>(i0 % IPR) * scratch[12];
+        const int64_t c_hi = (i1 >= I) ? U : static_cast<int64_t>(IPR) * scratch[13] +
+                                                 static_cast<int64_t>(i1 % IPR) * scratch[14];
+        u_lo = c_lo + static_cast<int64_t>(crank) * (c_hi - c_lo) / CS;
+        u_hi = c_lo + static_cast<int64_t>(crank + 1) * (c_hi - c_lo) / CS;
+    }
     {
         int run = run0;
         for (int b = b_lo; b < b_hi; ++b) {
@@ -299,25 +494,12 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
             run += n;
         }
     }
-    // Block 0 publishes the chunk offsets for the merge kernel only after the
-    // grid-dependency wait: until then the previous call's merge kernel (same
-    // workspace, same stream) may still be reading them.
-    auto publish_prefix = [&]() {
-        if (blockIdx.x != 0) return;
-        int run = run0;
-        for (int b = b_lo; b < b_hi; ++b) {
-            a.ws_prefix[b] = run;
-            run += walk.chunks_of(a.seq_lens[b]);
-        }
-        if (tid == 0) a.ws_prefix[B] = total;
-    };
     __syncthreads();
-    if (u_lo >= u_hi) {
-        grid_dependency_wait();
-        publish_prefix();
-        return;
-    }
-    walk.init(scratch[8], scratch[9], u_lo, u_hi);
+    if (u_lo >= u_hi && !clu) return;   // nothing to do (the merge reads no slot of this CTA)
+    // (an empty range in cluster mode: the walk yields nothing and the CTA
+    // only takes part in its cluster's reduction)
+    walk.init(u_lo < u_hi ? scratch[8] : 0, u_lo < u_hi ? scratch[9] : 0, u_lo, u_hi);
+
 
     const int P = a.page_size;
     const int box_rows = a.box_rows;
@@ -332,6 +514,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
         prefetch_tensormap(&tmap_k);
         prefetch_tensormap(&tmap_v);
         PageWindow win;
+        win.reset(nullptr);
         // L2 prefetch of the first S chunks, before the dependency wait.
         {
             Walker w2 = walk;
@@ -360,12 +543,17 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
         }
         grid_dependency_wait();
-        publish_prefix();
         // A segment's abort flag and first page-table window are loaded one
         // segment ahead, so the first TMA of a segment waits on no load.
+        // (the page table is not written by the preceding kernels, so a window
+        // the L2 prefetch above already loaded for this row is kept)
         auto load_meta = [&](const Segment& sg, PageWindow& w) {
-            w.reset(a.page_table + static_cast<int64_t>(sg.b) * a.max_pages);
-            w.preload(sg.c0 * kChunkTokens / P, (sg.L + P - 1) / P, lane);
+            const int32_t* row = a.page_table + static_cast<int64_t>(sg.b) * a.max_pages;
+            const int j0 = sg.c0 * kChunkTokens / P;
+            if (w.row != row || w.base != j0) {
+                w.reset(row);
+                w.preload(j0, (sg.L + P - 1) / P, lane);
+            }
             return (a.abort != nullptr) ? static_cast<int>(a.abort[sg.b]) : 0;
         };
         uint32_t it = 0;
@@ -445,6 +633,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
             s = sn;
             have = have_next;
         }
+        if (a.cluster_size > 0) attn_cluster_reduce<kFp8, kD, kGP, kH>(a, smem);
         return;
     }
 
@@ -455,7 +644,6 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
     // the GQA group (kNB n-blocks of 8).  P is moved from the S accumulator
     // layout into the PV B-operand layout with an in-register 8x8 transpose.
     grid_dependency_wait();
-    publish_prefix();
     const int g = lane >> 2;   // MMA group id
     const int c = lane & 3;    // thread in group
     const int G = a.group;
@@ -533,24 +721,55 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
         Segment sn;
         const bool have_next = walk.next(sn);
         if constexpr (!C::kEarlyQ) aborted = load_q(s, qw);
-        const int item = s.b * IPR + s.h;
-        const bool whole = (s.c0 == 0 && s.c1 == s.n);
-        const int64_t slot = static_cast<int64_t>(blockIdx.x) + item;
-        const int64_t head0 = static_cast<int64_t>(s.b) * a.num_q_heads + s.h * IQ;  // item
-        const int64_t head0_w = head0 + kvh_w * G;                                    // this warp
+        // (the item's indices are recomputed where they are used, after the
+        // chunk loop, rather than held in registers through it)
+        auto item_of = [&]() { return s.b * IPR + s.h; };
+        auto whole_of = [&]() { return s.c0 == 0 && s.c1 == s.n; };
+        auto slot_of = [&]() { return static_cast<int64_t>(blockIdx.x) + item_of(); };
+        auto head0_of = [&]() {   // the item's first query-head row
+            return static_cast<int64_t>(s.b) * a.num_q_heads + s.h * IQ;
+        };
+        // Cluster mode: a partial segment goes to a shared-memory record.  Of
+        // a contiguous range only the first segment can start inside its item
+        // (c0 > 0), and a partial segment that starts at its item's beginning
+        // ends inside it and is the range's last: the former uses the
+        // dedicated buffer (record 0), the latter the stage after its last
+        // chunk (record 1; no stage is in use any more).  `it` must be the
+        // chunk count after the segment.
+        auto record = [&]() -> float* {
+            const bool first = s.c0 > 0;
+            float* r = first ? rec0 : reinterpret_cast<float*>(smem + (it % S) * C::kStageBytes);
+            if (tid == 0) {
+                scratch[first ? 5 : 6] = item_of();
+                if (!first) scratch[7] = static_cast<int>(smem_addr(r));
+            }
+            return r;
+        };
 
         if (aborted) {
+            const bool whole = whole_of();
+            const int64_t head0 = head0_of();
+            // partial O and (m, l, lr) of the item: workspace slot or record
+            float* o_dst = nullptr;
+            float* ml_dst = nullptr;
+            if (!whole) {
+                if (a.cluster_size > 0) {
+                    o_dst = record();
+                    ml_dst = o_dst + C::kRecHeads * kD;
+                } else {
+                    o_dst = a.ws_o + slot_of() * IQ * kD;
+                    ml_dst = a.ws_ml + slot_of() * IQ * 4;
+                }
+            }
             for (int e = tid; e < IQ * kD; e += kConsumerThreads) {
                 const int hq = e / kD, d = e % kD;
                 if (whole) {
                     a.out[(head0 + hq) * kD + d] = 0;
                     if (d == 0) a.lse[head0 + hq] = kNegInf;
                 } else {
-                    a.ws_o[(slot * IQ + hq) * kD + d] = 0.f;
-                    if (d == 0) {
-                        a.ws_ml[(slot * IQ + hq) * 2 + 0] = kNegInf;
-                        a.ws_ml[(slot * IQ + hq) * 2 + 1] = -1.f;
-                    }
+                    o_dst[hq * kD + d] = 0.f;
+                    if (d == 0)
+                        *reinterpret_cast<float4*>(ml_dst + 4 * hq) = make_float4(kNegInf, -1.f, -1.f, 0.f);
                 }
             }
             if constexpr (C::kEarlyQ) aborted = have_next ? load_q(sn, qw) : 0;
@@ -615,11 +834,15 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
         for (int nb = 0; nb < kNB; ++nb)
 #pragma unroll
             for (int mb = 0; mb < kMB; ++mb) o[nb][mb][0] = o[nb][mb][1] = o[nb][mb][2] = o[nb][mb][3] = 0.f;
-        float m[kNB][2], l[kNB][2];
+        // l: sum of the fp32 weights (for the LSE); lr: sum of the weights as
+        // rounded for the PV product (the output's normaliser, so that the
+        // output is a weighted mean with exactly the weights the MMA used)
+        float m[kNB][2], l[kNB][2], lr[kNB][2];
 #pragma unroll
         for (int nb = 0; nb < kNB; ++nb) {
             m[nb][0] = m[nb][1] = kNegInf;
             l[nb][0] = l[nb][1] = 0.f;
+            lr[nb][0] = lr[nb][1] = 0.f;
         }
         int poisoned = 0;
 
@@ -719,6 +942,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         alpha[col] = (nm == kNegInf) ? 1.f : exp2f(m[nb][col] - nm);
                         m[nb][col] = nm;
                         l[nb][col] *= alpha[col];
+                        lr[nb][col] *= alpha[col];
                     }
 #pragma unroll
                     for (int mb = 0; mb < kMB; ++mb) {
@@ -740,13 +964,23 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 }
                 l[nb][0] += p[nb][0] + p[nb][2];
                 l[nb][1] += p[nb][1] + p[nb][3];
+                uint32_t h01, h23;
+                float r0, r1, r2, r3;
                 if constexpr (kFp8) {
-                    pb[nb][0] = movmatrix_trans(pack_f16x2(p[nb][0], p[nb][1]));
-                    pb[nb][1] = movmatrix_trans(pack_f16x2(p[nb][2], p[nb][3]));
+                    h01 = pack_f16x2(p[nb][0], p[nb][1]);
+                    h23 = pack_f16x2(p[nb][2], p[nb][3]);
+                    f16x2_to_f32x2(h01, r0, r1);
+                    f16x2_to_f32x2(h23, r2, r3);
                 } else {
-                    pb[nb][0] = movmatrix_trans(pack_bf16x2(p[nb][0], p[nb][1]));
-                    pb[nb][1] = movmatrix_trans(pack_bf16x2(p[nb][2], p[nb][3]));
+                    h01 = pack_bf16x2(p[nb][0], p[nb][1]);
+                    h23 = pack_bf16x2(p[nb][2], p[nb][3]);
+                    bf16x2_to_f32x2(h01, r0, r1);
+                    bf16x2_to_f32x2(h23, r2, r3);
                 }
+                lr[nb][0] += r0 + r2;
+                lr[nb][1] += r1 + r3;
+                pb[nb][0] = movmatrix_trans(h01);
+                pb[nb][1] = movmatrix_trans(h23);
             }
 
             // ---- O^T[16 dims][8 heads] += V^T P^T per m-block of dims --------
@@ -815,9 +1049,12 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
             __syncwarp();
             if (lane == 0 && !(C::kRedInStage && ch + 1 == s.c1)) mbar_arrive(&empty_bar[stage]);
         }
-        // the next segment's query words and abort flag, consumed after the epilogue
+        // the next segment's query words and abort flag, consumed after the
+        // epilogue
         int next_aborted = 0;
         if constexpr (C::kEarlyQ) next_aborted = have_next ? load_q(sn, qw) : 0;
+        const bool whole = whole_of();
+        const int64_t head0 = head0_of();
 
         const int last_stage = (it + S - 1) % S;   // stage of the segment's last chunk
         float* red_o = C::kRedInStage ? reinterpret_cast<float*>(smem + last_stage * C::kStageBytes)
@@ -832,11 +1069,15 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
         for (int nb = 0; nb < kNB; ++nb)
 #pragma unroll
             for (int col = 0; col < 2; ++col) {
-                float v = l[nb][col];
+                float v = l[nb][col], vr = lr[nb][col];
                 v += __shfl_xor_sync(0xffffffffu, v, 4);
+                vr += __shfl_xor_sync(0xffffffffu, vr, 4);
                 v += __shfl_xor_sync(0xffffffffu, v, 8);
+                vr += __shfl_xor_sync(0xffffffffu, vr, 8);
                 v += __shfl_xor_sync(0xffffffffu, v, 16);
+                vr += __shfl_xor_sync(0xffffffffu, vr, 16);
                 l[nb][col] = v;
+                lr[nb][col] = vr;
             }
         if (g == 0) {
 #pragma unroll
@@ -845,6 +1086,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 for (int col = 0; col < 2; ++col) {
                     red_m[warp * kGP + 8 * nb + 2 * c + col] = m[nb][col];
                     red_l[warp * kGP + 8 * nb + 2 * c + col] = l[nb][col];
+                    red_lr[warp * kGP + 8 * nb + 2 * c + col] = lr[nb][col];
                 }
         }
         // O into red_o[warp][head][kD] (fp32); the 16-byte units of a row are
@@ -882,6 +1124,17 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
         // Thread -> (head, 16-byte unit of dims): per pass the consumer
         // threads cover kConsumerThreads / (kD/4) heads.
         {
+            float* o_dst = nullptr;    // partial O and (m, l, lr): workspace slot or record
+            float* ml_dst = nullptr;
+            if (!whole) {
+                if (a.cluster_size > 0) {
+                    o_dst = record();
+                    ml_dst = o_dst + C::kRecHeads * kD;
+                } else {
+                    o_dst = a.ws_o + slot_of() * IQ * kD;
+                    ml_dst = a.ws_ml + slot_of() * IQ * 4;
+                }
+            }
             constexpr int kUnits = kD / 4;
             constexpr int kHeadsPerPass = kConsumerThreads / kUnits;
             const int u = tid % kUnits;
@@ -893,13 +1146,14 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 float M = kNegInf;
 #pragma unroll
                 for (int w = 0; w < kWarpsPerHead; ++w) M = fmaxf(M, red_m[r0 + w * kGP]);
-                float Lsum = 0.f;
+                float Lsum = 0.f, Lr = 0.f;
                 float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                 for (int w = 0; w < kWarpsPerHead; ++w) {
                     const float mw = red_m[r0 + w * kGP];
                     const float wt = (mw == kNegInf) ? 0.f : exp2f(mw - M);
                     Lsum += wt * red_l[r0 + w * kGP];
+                    Lr += wt * red_lr[r0 + w * kGP];
                     const float4 x = *reinterpret_cast<const float4*>(red_o + (r0 + w * kGP) * kD + 4 * su);
                     O.x += wt * x.x;
                     O.y += wt * x.y;
@@ -914,19 +1168,20 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         dst[1] = 0u;
                         if (u == 0) a.lse[hrow] = kNegInf;
                     } else {
-                        dst[0] = pack_bf16x2(O.x * a.v_scale / Lsum, O.y * a.v_scale / Lsum);
-                        dst[1] = pack_bf16x2(O.z * a.v_scale / Lsum, O.w * a.v_scale / Lsum);
+                        const float k = a.v_scale / Lr;
+                        dst[0] = pack_bf16x2(O.x * k, O.y * k);
+                        dst[1] = pack_bf16x2(O.z * k, O.w * k);
                         if (u == 0) a.lse[hrow] = (M + log2f(Lsum)) * kLn2;
                     }
                 } else {
-                    const int64_t r = slot * IQ + hq;
                     const float4 val = poisoned ? make_float4(0.f, 0.f, 0.f, 0.f)
                                                 : make_float4(O.x * a.v_scale, O.y * a.v_scale,
                                                               O.z * a.v_scale, O.w * a.v_scale);
-                    *reinterpret_cast<float4*>(a.ws_o + r * kD + 4 * u) = val;
+                    *reinterpret_cast<float4*>(o_dst + hq * kD + 4 * u) = val;
                     if (u == 0)
-                        *reinterpret_cast<float2*>(a.ws_ml + r * 2) =
-                            poisoned ? make_float2(kNegInf, -1.f) : make_float2(M, Lsum);
+                        *reinterpret_cast<float4*>(ml_dst + 4 * hq) =
+                            poisoned ? make_float4(kNegInf, -1.f, -1.f, 0.f)
+                                     : make_float4(M, Lsum, Lr, 0.f);
                 }
             }
         }
@@ -939,6 +1194,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
         s = sn;
         have = have_next;
     }
+    if (a.cluster_size > 0) attn_cluster_reduce<kFp8, kD, kGP, kH>(a, smem);
 }
 
 // ---------------------------------------------------------------------------
@@ -946,14 +1202,17 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
 // (kHPC = 16) or, when the items are split over many CTAs, one CTA per group
 // of 4 query heads (kHPC = 4: each thread then owns a single output and has
 // every segment's value in flight at once).  For each query head h of the
-// item: M = max_s m_s, L = sum_s l_s 2^(m_s - M), out = sum_s O_s 2^(m_s - M) / L
-// over the item's segments s (one per CTA that worked on it).  Segment
+// item: M = max_s m_s, L = sum_s l_s 2^(m_s - M), Lr = sum_s lr_s 2^(m_s - M),
+// out = sum_s O_s 2^(m_s - M) / Lr and lse = M + log2 L (natural units) over the
+// item's segments s (one per CTA that worked on it); lr is the sum of the
+// weights as rounded for the PV product, l of the fp32 weights.  Segment
 // weights are computed once into shared memory (in tiles of kMergeTile
 // segments, merged online), then every thread sums its (head, dim) outputs
 // with independent loads.
 // ---------------------------------------------------------------------------
 constexpr int kMergeThreads = 512;
-constexpr int kMergeTile = 256;
+constexpr int kMergeTile = 128;
+constexpr int kMergeFastSegs = 8;   // items split over at most this many CTAs: one round trip
 
 __device__ __forceinline__ int64_t cta_of_unit(int64_t u, int64_t U, int N) {
     // largest c with floor(c * U / N) <= u
@@ -964,11 +1223,12 @@ template <int kD, int kHPC>
 __global__ void __launch_bounds__(kMergeThreads)
 attn_merge_kernel(const AttnArgs a) {
     __shared__ float s_w[kMergeTile][kHPC];   // m_s, then weight 2^(m_s - M), of segment s, head h
-    __shared__ float s_l[kMergeTile][kHPC];   // l_s
-    __shared__ float s_m[kHPC], s_sum[kHPC], s_scale[kHPC];
+    __shared__ float s_l[kMergeTile][kHPC];   // l_s (fp32 weights)
+    __shared__ float s_lr[kMergeTile][kHPC];  // lr_s (weights as rounded for the PV product)
+    __shared__ float s_m[kHPC], s_sum[kHPC], s_sumr[kHPC], s_scale[kHPC];
     __shared__ int s_dead;
+    __shared__ int s_red[2][kMergeThreads / 32], s_nb;
     launch_dependents();
-    grid_dependency_wait();
     const int tid = threadIdx.x;
     constexpr int kGroups = 16 / kHPC;       // CTAs per item
     const int IPR = a.items_per_req;
@@ -979,10 +1239,40 @@ attn_merge_kernel(const AttnArgs a) {
     if (hq0 >= G) return;
     const int NH = min(kHPC, G - hq0);       // this CTA's heads
     const int64_t head0 = static_cast<int64_t>(b) * a.num_q_heads + h * G + hq0;
-    const int32_t pre = a.ws_prefix[b];
-    const int32_t nxt = a.ws_prefix[b + 1];
-    const int32_t tot = a.ws_prefix[a.batch];
-    const int32_t n = nxt - pre;
+    // Chunk counts of the requests before b, of b and of the batch, from the
+    // lengths (an input no kernel writes), before the grid-dependency wait:
+    // this overlaps the partial kernel's tail.
+    {
+        const int64_t max_tokens = static_cast<int64_t>(a.max_pages) * a.page_size;
+        int pre_part = 0, tot_part = 0;
+        for (int bb = tid; bb < a.batch; bb += kMergeThreads) {
+            const int32_t len = a.seq_lens[bb];
+            const int nb = (len >= 1 && static_cast<int64_t>(len) <= max_tokens)
+                               ? (len + kChunkTokens - 1) / kChunkTokens
+                               : 0;
+            tot_part += nb;
+            if (bb < b) pre_part += nb;
+            if (bb == b) s_nb = nb;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            pre_part += __shfl_xor_sync(0xffffffffu, pre_part, off);
+            tot_part += __shfl_xor_sync(0xffffffffu, tot_part, off);
+        }
+        if ((tid & 31) == 0) {
+            s_red[0][tid >> 5] = pre_part;
+            s_red[1][tid >> 5] = tot_part;
+        }
+        __syncthreads();
+    }
+    int32_t pre = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < kMergeThreads / 32; ++w) {
+        pre += s_red[0][w];
+        tot += s_red[1][w];
+    }
+    const int32_t n = s_nb;
+    grid_dependency_wait();
     if (n == 0) {
         for (int e = tid; e < NH * kD; e += kMergeThreads) {
             const int hq = e / kD, d = e % kD;
@@ -998,27 +1288,79 @@ attn_merge_kernel(const AttnArgs a) {
     const int64_t c1 = cta_of_unit(u0 + n - 1, U, NE);
     if (c0 == c1) return;   // finished by the partial kernel
     const int nseg = static_cast<int>(c1 - c0 + 1);
+    const int64_t stride = static_cast<int64_t>(G) * kD;
+    if (nseg <= kMergeFastSegs) {
+        // Few segments: thread -> (head, 4 dims); every segment's (m, l, lr)
+        // and output quad are requested at once (one round trip).
+        constexpr int kQuads = kD / 4;
+        const int hq = tid / kQuads, q = tid - hq * kQuads;
+        if (hq >= NH) return;
+        float4 ml[kMergeFastSegs], x[kMergeFastSegs];
+#pragma unroll
+        for (int k = 0; k < kMergeFastSegs; ++k) {
+            if (k < nseg) {
+                const int64_t slot = c0 + k + item;
+                ml[k] = *reinterpret_cast<const float4*>(a.ws_ml + (slot * G + hq0 + hq) * 4);
+                x[k] = *reinterpret_cast<const float4*>(a.ws_o + slot * stride +
+                                                        static_cast<int64_t>(hq0 + hq) * kD + 4 * q);
+            }
+        }
+        float M = kNegInf;
+        int dead = 0;
+#pragma unroll
+        for (int k = 0; k < kMergeFastSegs; ++k) {
+            if (k < nseg) {
+                M = fmaxf(M, ml[k].x);
+                dead |= ml[k].y < 0.f;
+            }
+        }
+        float Lsum = 0.f, Lr = 0.f;
+        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < kMergeFastSegs; ++k) {
+            if (k < nseg) {
+                const float wt = (ml[k].x == kNegInf) ? 0.f : exp2f(ml[k].x - M);
+                Lsum += wt * ml[k].y;
+                Lr += wt * ml[k].z;
+                O.x += wt * x[k].x;
+                O.y += wt * x[k].y;
+                O.z += wt * x[k].z;
+                O.w += wt * x[k].w;
+            }
+        }
+        uint32_t* dst = reinterpret_cast<uint32_t*>(a.out + (head0 + hq) * kD + 4 * q);
+        if (dead) {
+            dst[0] = 0u;
+            dst[1] = 0u;
+        } else {
+            dst[0] = pack_bf16x2(O.x / Lr, O.y / Lr);
+            dst[1] = pack_bf16x2(O.z / Lr, O.w / Lr);
+        }
+        if (q == 0) a.lse[head0 + hq] = dead ? kNegInf : (M + log2f(Lsum)) * kLn2;
+        return;
+    }
     if (tid < kHPC) {
         s_m[tid] = kNegInf;
         s_sum[tid] = 0.f;
+        s_sumr[tid] = 0.f;
     }
     if (tid == 0) s_dead = 0;
     constexpr int kPer = (kHPC * kD + kMergeThreads - 1) / kMergeThreads;
     float acc[kPer];
 #pragma unroll
     for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
-    const int64_t stride = static_cast<int64_t>(G) * kD;
 
     for (int t0 = 0; t0 < nseg; t0 += kMergeTile) {
         const int tn = min(kMergeTile, nseg - t0);
-        // (1) the tile's (m, l) pairs of this CTA's heads into shared memory:
+        // (1) the tile's (m, l, lr) of this CTA's heads into shared memory:
         // one round trip
         for (int e = tid; e < tn * NH; e += kMergeThreads) {
             const int sg = e / NH, hq = e % NH;
             const int64_t slot = c0 + t0 + sg + item;
-            const float2 ml = *reinterpret_cast<const float2*>(a.ws_ml + (slot * G + hq0 + hq) * 2);
+            const float4 ml = *reinterpret_cast<const float4*>(a.ws_ml + (slot * G + hq0 + hq) * 4);
             s_w[sg][hq] = ml.x;
             s_l[sg][hq] = ml.y;
+            s_lr[sg][hq] = ml.z;
         }
         __syncthreads();
         // (2) per head, in shared memory: new running max, weights, sum
@@ -1036,20 +1378,25 @@ attn_merge_kernel(const AttnArgs a) {
             }
             const float m_old = s_m[hq];
             const float m_new = fmaxf(m_old, mx);
-            float lsum = 0.f;
+            float lsum = 0.f, lrsum = 0.f;
             for (int sg = (tid & 31); sg < tn; sg += 32) {
                 const float ms = s_w[sg][hq];
                 const float wt = (ms == kNegInf) ? 0.f : exp2f(ms - m_new);
                 s_w[sg][hq] = wt;
                 lsum += wt * s_l[sg][hq];
+                lrsum += wt * s_lr[sg][hq];
             }
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+            for (int off = 16; off > 0; off >>= 1) {
+                lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+                lrsum += __shfl_xor_sync(0xffffffffu, lrsum, off);
+            }
             if ((tid & 31) == 0) {
                 const float r = (m_old == kNegInf) ? 0.f : exp2f(m_old - m_new);
                 if (dead) s_dead = 1;
                 s_scale[hq] = r;
                 s_sum[hq] = s_sum[hq] * r + lsum;
+                s_sumr[hq] = s_sumr[hq] * r + lrsum;
                 s_m[hq] = m_new;
             }
         }
@@ -1089,7 +1436,7 @@ attn_merge_kernel(const AttnArgs a) {
             a.out[(head0 + hq) * kD + d] = 0;
             if (d == 0) a.lse[head0 + hq] = kNegInf;
         } else {
-            a.out[(head0 + hq) * kD + d] = f32_to_bf16_bits(acc[k] / s_sum[hq]);
+            a.out[(head0 + hq) * kD + d] = f32_to_bf16_bits(acc[k] / s_sumr[hq]);
             if (d == 0) a.lse[head0 + hq] = (s_m[hq] + log2f(s_sum[hq])) * kLn2;
         }
     }
@@ -1103,7 +1450,42 @@ static cudaError_t launch_variant(int grid, cudaStream_t stream, const CUtensorM
                                   const CUtensorMap& tv, const AttnArgs& args) {
     using C = AttnCfg<kFp8, kD, kGP, kH>;
     PdlLaunch l(dim3(grid), dim3(kAttnThreads), C::kSmemBytes, stream);
+    if (args.cluster_size > 0) {
+        // Cluster launches go without programmatic dependent launch.  Measured
+        // on B200: launched early, beside the resident CTAs of the preceding
+        // kernel (the check + append kernel, with 256 or with 128 threads),
+        // a grid sized to every cluster the device holds could not place one
+        // or two of its clusters, and those started only when other clusters
+        // of the grid exited, about 1.6x the call's time.  Launched after the
+        // preceding kernel, every cluster starts at once.
+        l.set_cluster(args.cluster_size);
+        l.cfg.attrs = &l.attr[1];
+        l.cfg.numAttrs = 1;
+    }
     return cudaLaunchKernelEx(&l.cfg, attn_partial_kernel<kFp8, kD, kGP, kH>, tk, tv, args);
+}
+
+template <bool kFp8, int kD, int kGP, int kH>
+static cudaError_t max_clusters_variant(int cluster_size, int* clusters) {
+    using C = AttnCfg<kFp8, kD, kGP, kH>;
+    auto* fn = attn_partial_kernel<kFp8, kD, kGP, kH>;
+    cudaError_t e = cudaSuccess;
+    if (cluster_size > 8) {
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(cluster_size);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(cluster_size));
+    cfg.blockDim = dim3(kAttnThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaOccupancyMaxActiveClusters(clusters, fn, &cfg);
 }
 
 // (fp8, head_dim, group pad, KV heads per item)
@@ -1141,6 +1523,15 @@ cudaError_t attn_occupancy(bool fp8, int head_dim, int group_pad, int kv_per_ite
         return cudaOccupancyMaxActiveBlocksPerMultiprocessor(                         \
             blocks_per_sm, attn_partial_kernel<F, D, GP, H>, kAttnThreads,            \
             AttnCfg<F, D, GP, H>::kSmemBytes);
+    PKV_FOR_EACH_VARIANT(X)
+#undef X
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t attn_max_clusters(bool fp8, int head_dim, int group_pad, int kv_per_item,
+                              int cluster_size, int* clusters) {
+#define X(F, D, GP, H) \
+    if (PKV_MATCH(F, D, GP, H)) return max_clusters_variant<F, D, GP, H>(cluster_size, clusters);
     PKV_FOR_EACH_VARIANT(X)
 #undef X
     return cudaErrorInvalidValue;

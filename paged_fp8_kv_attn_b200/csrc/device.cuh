@@ -233,6 +233,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
+// The two f16 halves of x as binary32 (low half -> lo); exact.
+__device__ __forceinline__ void f16x2_to_f32x2(uint32_t x, float& lo, float& hi) {
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+        "cvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+        : "=f"(lo), "=f"(hi)
+        : "r"(x));
+}
+// The two bf16 halves of x as binary32 (low half -> lo); exact.
+__device__ __forceinline__ void bf16x2_to_f32x2(uint32_t x, float& lo, float& hi) {
+    lo = __uint_as_float(x << 16);
+    hi = __uint_as_float(x & 0xFFFF0000u);
+}
 // binary32 -> bf16 bit pattern, round to nearest even.
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float x) {
     uint16_t r;
@@ -276,6 +288,46 @@ __device__ __forceinline__ bool gemv_wait(uint64_t* bar, uint32_t parity, volati
     *failed = 1;
     if (status != nullptr) atomicOr(status, 1u);
     return false;
+}
+
+// ---------------------------------------------------------------------------
+// thread-block clusters: rank, barrier, distributed shared memory
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Every thread of every CTA of the cluster arrives and waits: shared-memory
+// writes before the barrier are visible to loads from any CTA of the
+// cluster after it.
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+// Address, in the cluster's shared window, of the variable at the local
+// shared address `addr` in the CTA of rank `rank`.
+__device__ __forceinline__ uint32_t cluster_map(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ int32_t ld_cluster_s32(uint32_t addr) {
+    int32_t v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
 }
 
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {

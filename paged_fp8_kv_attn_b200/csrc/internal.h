@@ -10,6 +10,9 @@ namespace pkv {
 
 // Tokens per pipeline stage of the attention kernels (one "chunk").
 constexpr int kChunkTokens = 64;
+// Largest thread-block cluster of the attention kernel's cluster mode (16 is
+// the non-portable maximum on sm_100).
+constexpr int kMaxCluster = 16;
 
 // Arguments of the split-K partial and merge kernels (passed by value).
 struct AttnArgs {
@@ -20,8 +23,8 @@ struct AttnArgs {
     uint16_t* out;              // [B][Hq][D] bf16
     float* lse;                 // [B][Hq]
     uint32_t* ws_status;        // workspace word 0 (cleared by CTA 0 of each call)
-    int32_t* ws_prefix;         // [B + 1] chunk offsets (written by CTA 0)
-    float* ws_ml;               // [slots][G][2]  (running max in log2 units, sum)
+    float* ws_ml;               // [slots][G][4]  (running max in log2 units, sum of the
+                                //  fp32 weights, sum of the rounded weights, unused)
     float* ws_o;                // [slots][G][D]  (unnormalised, V scale applied)
     int32_t batch;
     int32_t max_pages;
@@ -34,6 +37,9 @@ struct AttnArgs {
     int32_t num_pages;
     int32_t num_ctas;
     int32_t box_rows;           // rows per TMA box = min(page_size, 64)
+    int32_t cluster_size;       // 0: split-K over the grid + merge kernel;
+                                // C > 0: clusters of C CTAs, no merge kernel
+    int32_t num_clusters;       // cluster mode: clusters in the grid
     float qk_scale;             // sm_scale * k_scale * log2(e)
     float v_scale;              // per-tensor V scale (1 for BF16)
 };
@@ -50,7 +56,7 @@ inline int kv_heads_per_item(bool fp8, int num_kv_heads, int group) {
 
 // Workspace layout for given sizes and grid (slots = grid + work items).
 struct WorkspaceLayout {
-    size_t prefix_off, ml_off, o_off, total;
+    size_t ml_off, o_off, total;
 };
 WorkspaceLayout workspace_layout(int32_t batch, int32_t group, int32_t num_kv_heads,
                                  int32_t kv_per_item, int32_t head_dim, int32_t num_ctas);
@@ -63,6 +69,10 @@ cudaError_t attn_occupancy(bool fp8, int head_dim, int group_pad, int kv_per_ite
                            int* blocks_per_sm);
 constexpr int kAttnThreads = 160;   // 4 consumer warps + 1 producer warp
 
+// Clusters of `cluster_size` CTAs that can be resident at once (0 if none).
+cudaError_t attn_max_clusters(bool fp8, int head_dim, int group_pad, int kv_per_item,
+                              int cluster_size, int* clusters);
+// grid CTAs; with args.cluster_size > 0 launched as clusters of that size.
 cudaError_t launch_attn_partial(bool fp8, int head_dim, int group_pad, int kv_per_item, int grid,
                                 cudaStream_t stream, const CUtensorMap& tmap_k,
                                 const CUtensorMap& tmap_v, const AttnArgs& args);
@@ -133,10 +143,11 @@ cudaError_t launch_int4_gemv(int ncols, cudaStream_t stream, const CUtensorMap& 
                              const CUtensorMap& tmap_x, const CUtensorMap& tmap_s,
                              const GemvArgs& args);
 
-// Launch configuration with the programmatic-stream-serialisation attribute.
+// Launch configuration with the programmatic-stream-serialisation attribute
+// (and, optionally, a 1-D thread-block cluster shape).
 struct PdlLaunch {
     cudaLaunchConfig_t cfg;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     PdlLaunch(dim3 grid, dim3 block, size_t smem, cudaStream_t stream) {
         cfg = cudaLaunchConfig_t{};
         cfg.gridDim = grid;
@@ -147,6 +158,13 @@ struct PdlLaunch {
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
+    }
+    void set_cluster(int size) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = static_cast<unsigned>(size);
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
     }
 };
 

@@ -72,6 +72,13 @@ def test_host_validation_without_a_gpu(lib):
     assert lib.paged_decode_attn_workspace_size(0, 4, 6, 4, 64, 10) == 0
     # explicit grid: size is computable without a device
     assert lib.paged_decode_attn_workspace_size(0, 4, 64, 8, 128, 296) > 0
+    # the work-split query validates like the attention call, before any device query
+    out = [ctypes.c_int32(0) for _ in range(3)]
+    refs = [ctypes.byref(o) for o in out]
+    assert lib.paged_decode_attn_plan(7, 4, 64, 8, 128, 128, 64, 0, *refs) == 1
+    assert lib.paged_decode_attn_plan(0, 4, 64, 8, 128, 128, 64, 0, None, None, None) == 1
+    assert lib.paged_decode_attn_plan(0, 4, 64, 8, 96, 128, 64, 0, *refs) == 3
+    assert lib.paged_decode_attn_plan(0, 4, 64, 8, 128, 128, 64, -17, *refs) == 1
     # the no-allocation status copy needs a destination
     assert lib.paged_decode_attn_fp8_noalloc_status(None, None) == 1
     assert b"status_out" in lib.pkv_last_error()

@@ -14,7 +14,7 @@ from _pkv_helpers import DeviceBatch, compare, oracle_step, sample_items
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("batch", [1, 8, 32, 64])
+@pytest.mark.parametrize("batch", [1, 8, 16, 32, 64])
 @pytest.mark.parametrize("kv", ["fp8", "bf16"])
 def test_concurrency_sweep_sampled(cuda_device, batch, kv):
     wl = workloads.concurrency_sweep(batch, device="cuda")
@@ -66,4 +66,47 @@ def test_ragged_prefix_sampled(cuda_device):
     items = sample_items(wl, 8, seed=5, must=[shortest, 8 * wl.num_kv_heads + 3])
     ref_o, ref_l, _ = oracle_step(wl, items, kv_dtype="fp8")
     compare(wl, items, out, lse, ref_o, ref_l, label="ragged prefix")
+    assert pkv.workspace_status(db.ws) == 0
+
+
+def test_checked_step_costs_about_one_attention_call(cuda_device):
+    """Performance guard for the launch chaining of the cluster-mode kernel:
+    the checked step (check + append kernel, then attention) must stay close
+    to the attention call alone.  A cluster grid launched early beside the
+    preceding kernel's CTAs once left two clusters unplaced until others
+    exited (about 1.6x the call); the bound here is 1.25x, medians of 30
+    CUDA-graph replays, batch 32 x 8,192 tokens (larger than L2)."""
+    import statistics
+    wl = workloads.concurrency_sweep(32, device="cuda")
+    db = DeviceBatch(wl, kv_dtype="fp8")
+    db.workspace()
+
+    def graph(fn):
+        fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g):
+                fn()
+        torch.cuda.synchronize()
+        return g
+
+    g_step = graph(lambda: (db.check_append(), db.attend(use_abort=True)))
+    g_attn = graph(lambda: db.attend(use_abort=True))
+
+    def med(g):
+        ts = []
+        for _ in range(30):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    med(g_step)
+    t_step, t_attn = med(g_step), med(g_attn)
+    assert t_step < 1.25 * t_attn, (t_step, t_attn)
     assert pkv.workspace_status(db.ws) == 0

@@ -248,12 +248,94 @@ def test_attention_small_all_items(cuda_device, case, kv):
         assert pkv.workspace_status(db2.ws) == 0
 
 
+def _cluster_sizes_that_fit(db):
+    """Cluster sizes 1..16 the device can run for this batch's variant: every
+    size up to 8 must fit; above 8 (non-portable sizes) the device may refuse."""
+    sizes = []
+    for c in range(1, 17):
+        try:
+            db.attend(use_abort=False, num_ctas=-c)
+        except pkv.PagedKVError as err:
+            assert c > 8 and "do not fit" in str(err), err
+            continue
+        sizes.append(c)
+    torch.cuda.synchronize()
+    return sizes
+
+
+@pytest.mark.parametrize("kv", ["fp8", "bf16"])
+@pytest.mark.parametrize("case", SMALL, ids=[f"c{i}" for i in range(len(SMALL))])
+def test_attention_cluster_mode_every_size(cuda_device, case, kv):
+    """The single-launch cluster mode (each request's CTAs form a thread-block
+    cluster and combine their split-K partials in distributed shared memory,
+    no merge kernel), forced at every cluster size: every item against the
+    oracle."""
+    lens, P, Hq, Hkv, D = case
+    wl = workloads.custom(lens, page_size=P, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D,
+                          seed=sum(lens) * 7 + P, spare_pages=3)
+    items = list(range(wl.batch * Hkv))
+    ref_o, ref_l, _ = oracle_step(wl, items, kv_dtype=kv, check=True, append=True)
+    db = DeviceBatch(wl, kv_dtype=kv)
+    db.step(check=True, append=True)
+    sizes = _cluster_sizes_that_fit(db)
+    assert sizes[:8] == list(range(1, 9))
+    for c in sizes:
+        db.out.fill_(float("nan"))
+        db.lse.fill_(float("nan"))
+        db.attend(use_abort=True, num_ctas=-c)
+        torch.cuda.synchronize()
+        out, lse = db.outputs()
+        compare(wl, items, out, lse, ref_o, ref_l, label=f"{kv} cluster={c}")
+        assert pkv.workspace_status(db.ws) == 0
+
+
+@pytest.mark.parametrize("kv", ["fp8", "bf16"])
+def test_attention_cluster_mode_long_requests(cuda_device, kv):
+    """Cluster mode where each cluster owns several long requests, cut into
+    many CTA ranges (items split over up to 16 CTAs, records in both the
+    dedicated buffer and a pipeline stage), plus an aborted request."""
+    wl = workloads.custom([9000, 64, 4097, 1, 12000, 640, 3000], page_size=64, num_q_heads=64,
+                          num_kv_heads=8, head_dim=128, seed=57, spare_pages=2)
+    items = list(range(wl.batch * 8))
+    wl.expected_tags[3, 0] ^= np.uint32(1)      # request 3 fails its check
+    ref_o, ref_l, ref_abort = oracle_step(wl, items, kv_dtype=kv, check=True, append=True)
+    assert ref_abort.tolist() == [0, 0, 0, 1, 0, 0, 0]
+    db = DeviceBatch(wl, kv_dtype=kv)
+    db.step(check=True, append=True)
+    for c in _cluster_sizes_that_fit(db):
+        db.out.fill_(float("nan"))
+        db.attend(use_abort=True, num_ctas=-c)
+        torch.cuda.synchronize()
+        out, lse = db.outputs()
+        compare(wl, items, out, lse, ref_o, ref_l, label=f"{kv} cluster={c}")
+        assert np.all(np.isneginf(lse[3])) and not out[3].any()
+
+
+def test_attention_plan_matches_the_documented_choice(cuda_device):
+    """The library's default work split: cluster mode (one launch) while the
+    batch's items fit in one wave of CTAs, split-K plus merge beyond; an
+    explicit cluster size or grid is honoured."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    for kv, ipr in ((pkv.PKV_KV_FP8, 4), (pkv.PKV_KV_BF16, 8)):
+        for b in (1, 8, 16, 32, 64, 256):
+            clu, ctas, launches = pkv.paged_decode_attn_plan(kv, b, 64, 8, 128, 128, 64)
+            assert launches == (1 if clu else 2)
+            if b * ipr <= sms:
+                assert clu > 0, (kv, b)
+            if b == 256:
+                assert clu == 0 and ctas >= sms
+            if clu:
+                assert ctas % clu == 0 and clu <= 16
+        assert pkv.paged_decode_attn_plan(kv, 8, 64, 8, 128, 128, 64, -3)[0] == 3
+        assert pkv.paged_decode_attn_plan(kv, 8, 64, 8, 128, 128, 64, 37) == (0, 37, 2)
+
+
 @pytest.mark.parametrize("kv", ["fp8", "bf16"])
 def test_attention_workspace_reused_across_calls(cuda_device, kv):
     """One workspace serves consecutive calls with different grids and a
-    different batch.  The workspace holds the status word, the per-request
-    chunk offsets and the partial (m, l) and O slots; every call rewrites what
-    it reads, so no clearing is needed."""
+    different batch.  The workspace holds the status word and the partial
+    (m, l, lr) and O slots; every call rewrites what it reads, so no clearing
+    is needed."""
     wl1 = workloads.custom([3000, 70, 9000, 1, 640], page_size=64, num_q_heads=64, num_kv_heads=8,
                            head_dim=128, seed=41, spare_pages=2)
     wl2 = workloads.custom([129] * 9 + [2000], page_size=64, num_q_heads=64, num_kv_heads=8,
@@ -271,6 +353,7 @@ def test_attention_workspace_reused_across_calls(cuda_device, kv):
     ref2 = oracle_step(wl2, items2, kv_dtype=kv, check=False, append=True)
     for db, wl, items, ref, ctas in ((db1, wl1, items1, ref1, 37), (db2, wl2, items2, ref2, 5),
                                      (db1, wl1, items1, ref1, 0), (db2, wl2, items2, ref2, 0),
+                                     (db1, wl1, items1, ref1, -6), (db2, wl2, items2, ref2, -2),
                                      (db1, wl1, items1, ref1, 3)):
         db.out.fill_(float("nan"))
         db.step(check=False, append=True, num_ctas=ctas)
@@ -355,7 +438,7 @@ def test_attention_dead_requests(cuda_device, kv):
     wl.seq_lens = lens_bad
     db = DeviceBatch(wl, kv_dtype=kv)
     items = list(range(wl.batch * 2))
-    for ctas in (0, 2, 5):
+    for ctas in (0, 2, 5, -1, -3, -8):
         db.step(check=False, append=True, num_ctas=ctas)
         out, lse = db.outputs()
         ref_o, ref_l, _ = oracle_step(wl, items, kv_dtype=kv, check=False)

@@ -310,6 +310,61 @@ PKV_API pkv_status paged_decode_attn_fp8(const uint16_t* q, const uint8_t* k_cac
                                  size_t workspace_bytes, int32_t num_ctas, void* stream);
 
 /*
+ * paged_decode_attn_fp8_prefix -- paged_decode_attn_fp8 for batches whose
+ * requests share leading cache pages (a common prompt beginning whose pages
+ * several requests' page tables name: [T] "保护共享 KV cache", where cache
+ * reuse puts many requests on the same physical pages; [R], the prefix
+ * caching remark in "为什么 Cloudflare 的小型缓存胜过单纯的速度").  Same
+ * arguments, same outputs (up to rounding) and same abort / invalid-input
+ * behaviour as paged_decode_attn_fp8; the shared pages are read once per
+ * group instead of once per request.
+ *
+ * Nothing about the sharing is passed in: the call finds it on the device.
+ * Request b joins request b - 1's group when their page tables name the same
+ * valid pages for at least 4 leading 64-token chunks that lie entirely before
+ * both requests' newest tokens (only consecutive requests form groups).  A
+ * group's reference row is its member with the most chunks before its newest
+ * token (the first on a tie); each member shares with the group the leading
+ * chunks it has in common with the reference row (same rule).  Runs of up to
+ * 64 / G consecutive members from the group's first request
+ * (G = num_q_heads / num_kv_heads) form tensor-core tiles of two KV heads,
+ * if a run has 2 members and one of them other than the reference shares at
+ * least 4 chunks; the tile covers the run's largest share, which the
+ * reference, if in the run, takes as its own.  Those chunks are attended for
+ * all members of the tile together, each member's remaining chunks by the
+ * split-K kernel, and a merge kernel combines the two.  Supported: head_dim 128, an even num_kv_heads and G <= 8;
+ * other shapes run paged_decode_attn_fp8 unchanged (nothing shared).
+ *
+ * workspace: at least paged_decode_attn_fp8_prefix_workspace_size(...)
+ * bytes (the split-K workspace plus one partial record per (request, pair of
+ * KV heads) and the group plan), 256-byte aligned, no initialisation needed;
+ * word 0 is the status word as for paged_decode_attn_fp8.  num_ctas: 0 (the
+ * library's split-K grid) or N > 0 (split-K over N CTAs); cluster mode is
+ * not used (PKV_ERR_INVALID_ARG for num_ctas < 0).  chunk_begin_out: NULL,
+ * or a device [batch] int32 array that receives, per request, the number of
+ * leading chunks the shared pass covered (0 = none), in stream order.
+ * Kernels: four plan kernels, the shared-prefix kernel, the split-K partial
+ * kernel and the merge kernel, all chained with programmatic dependent
+ * launch; none of them reads the cache, the page table or abort before the
+ * preceding kernel has finished except the first, which reads seq_lens and
+ * page_table (inputs no kernel writes).
+ */
+PKV_API size_t paged_decode_attn_fp8_prefix_workspace_size(int32_t batch, int32_t num_q_heads,
+                                                           int32_t num_kv_heads,
+                                                           int32_t head_dim, int32_t num_ctas);
+PKV_API pkv_status paged_decode_attn_fp8_prefix(const uint16_t* q, const uint8_t* k_cache,
+                                                const uint8_t* v_cache, float k_scale,
+                                                float v_scale, const int32_t* page_table,
+                                                int32_t max_pages, const int32_t* seq_lens,
+                                                int32_t batch, int32_t num_q_heads,
+                                                int32_t num_kv_heads, int32_t head_dim,
+                                                int32_t page_size, int32_t num_pages,
+                                                float sm_scale, const uint8_t* abort,
+                                                uint16_t* out, float* lse, void* workspace,
+                                                size_t workspace_bytes, int32_t num_ctas,
+                                                int32_t* chunk_begin_out, void* stream);
+
+/*
  * paged_decode_attn_bf16 -- the same attention over a BF16 cache (no
  * scales), the comparison kernel of [S] Table 1.  Workspace from
  * paged_decode_attn_workspace_size(PKV_KV_BF16, ...).

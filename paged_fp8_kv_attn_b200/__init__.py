@@ -73,6 +73,8 @@ def _load():
                                       f32, P, P, P, P, sz, i32, P],
             "paged_decode_attn_bf16": [P, P, P, P, i32, P, i32, i32, i32, i32, i32, i32, f32, P,
                                        P, P, P, sz, i32, P],
+            "paged_decode_attn_fp8_prefix": [P, P, P, f32, f32, P, i32, P, i32, i32, i32, i32, i32,
+                                             i32, f32, P, P, P, P, sz, i32, P, P],
             "int4_dequant_gemv": [P, P, P, i32, i32, i32, i32, P, P, P],
         }
         for name, args in sig.items():
@@ -92,6 +94,8 @@ def _load():
         lib.paged_decode_attn_plan.restype = i32
         lib.paged_decode_attn_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
         lib.paged_decode_attn_workspace_size.restype = sz
+        lib.paged_decode_attn_fp8_prefix_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+        lib.paged_decode_attn_fp8_prefix_workspace_size.restype = sz
         lib.pkv_last_error.argtypes = []
         lib.pkv_last_error.restype = ctypes.c_char_p
         lib.pkv_version.argtypes = []
@@ -288,6 +292,24 @@ def alloc_workspace(kv_dtype, batch, num_q_heads, num_kv_heads, head_dim, num_ct
     return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
 
 
+def paged_decode_attn_fp8_prefix_workspace_size(batch, num_q_heads, num_kv_heads, head_dim,
+                                                num_ctas=0):
+    n = _load().paged_decode_attn_fp8_prefix_workspace_size(int(batch), int(num_q_heads),
+                                                            int(num_kv_heads), int(head_dim),
+                                                            int(num_ctas))
+    if n == 0:
+        raise PagedKVError("paged_decode_attn_fp8_prefix_workspace_size", 1,
+                           _load().pkv_last_error().decode())
+    return int(n)
+
+
+def alloc_prefix_workspace(batch, num_q_heads, num_kv_heads, head_dim, num_ctas=0, device=None):
+    """A uint8 CUDA tensor large enough for paged_decode_attn_fp8_prefix."""
+    n = paged_decode_attn_fp8_prefix_workspace_size(batch, num_q_heads, num_kv_heads, head_dim,
+                                                    num_ctas)
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
 def paged_decode_attn_plan(kv_dtype, batch, num_q_heads, num_kv_heads, head_dim, max_pages,
                            page_size, num_ctas=0):
     """The attention call's work split on the current device:
@@ -331,6 +353,28 @@ def paged_decode_attn_fp8(q, k_cache, v_cache, k_scale, v_scale, page_table, seq
         _ptr(q), _ptr(k_cache), _ptr(v_cache), float(k_scale), float(v_scale), _ptr(page_table),
         page_table.shape[1], _ptr(seq_lens), B, Hq, Hkv, D, P, NP, float(sm_scale), _ptr(abort),
         _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), num_ctas, _stream(stream)))
+
+
+def paged_decode_attn_fp8_prefix(q, k_cache, v_cache, k_scale, v_scale, page_table, seq_lens,
+                                 sm_scale, out, lse, workspace, abort=None, num_ctas=0,
+                                 chunk_begin_out=None, stream=None):
+    """paged_decode_attn_fp8 for batches whose consecutive requests share leading
+    pages: the shared chunks are attended once per group.  chunk_begin_out
+    (optional int32 [batch] CUDA tensor) receives the chunks the shared pass
+    covered per request."""
+    _need(k_cache, torch.uint8, 4, "k_cache")
+    _need(v_cache, torch.uint8, 4, "v_cache")
+    B, Hq, D, NP, Hkv, P = _attn_common(q, k_cache, page_table, seq_lens, out, lse, workspace,
+                                        abort)
+    if chunk_begin_out is not None:
+        _need(chunk_begin_out, torch.int32, 1, "chunk_begin_out")
+        if chunk_begin_out.numel() < B:
+            raise ValueError("chunk_begin_out needs batch entries")
+    _check("paged_decode_attn_fp8_prefix", _load().paged_decode_attn_fp8_prefix(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), float(k_scale), float(v_scale), _ptr(page_table),
+        page_table.shape[1], _ptr(seq_lens), B, Hq, Hkv, D, P, NP, float(sm_scale), _ptr(abort),
+        _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), num_ctas,
+        _ptr(chunk_begin_out), _stream(stream)))
 
 
 def paged_decode_attn_bf16(q, k_cache, v_cache, page_table, seq_lens, sm_scale, out, lse,

@@ -241,7 +241,7 @@ struct AttnPlan {
 
 pkv_status plan_attention(bool fp8, int32_t batch, int32_t num_kv_heads, int32_t group,
                           int32_t head_dim, int32_t max_pages, int32_t page_size,
-                          int32_t num_ctas, AttnPlan* plan) {
+                          int32_t num_ctas, AttnPlan* plan, bool allow_cluster = true) {
     pkv_status st = PKV_OK;
     int kv_per_item = pkv::kv_heads_per_item(fp8, num_kv_heads, group);
     plan->ws_kv_per_item = kv_per_item;
@@ -279,7 +279,7 @@ pkv_status plan_attention(bool fp8, int32_t batch, int32_t num_kv_heads, int32_t
     // only, so the workspace size does not depend on this).
     int64_t items = static_cast<int64_t>(batch) * (num_kv_heads / kv_per_item);
     int cluster = 0, nclusters = 0;
-    if (num_ctas < 0 || (num_ctas == 0 && items <= grid)) {
+    if (allow_cluster && (num_ctas < 0 || (num_ctas == 0 && items <= grid))) {
         if (num_ctas == 0 && kv_per_item == 2) {
             const DeviceInfo* info = nullptr;
             st = device_info(&info);
@@ -391,6 +391,197 @@ pkv_status attn_impl(bool fp8, const uint16_t* q, const void* k_cache, const voi
     if (cluster == 0) {
         e = pkv::launch_attn_merge(head_dim, as_stream(stream), a);
         if (e != cudaSuccess) return cuda_fail(e, "attention merge launch");
+    }
+    return PKV_OK;
+}
+
+// Shared-prefix mode: the split-K workspace, then the prefix records and the
+// plan arrays.
+struct PrefixLayout {
+    size_t pml_off, po_off, link_off, leader_off, refkey_off, ref_off, share_off, cbeg_off, tiles_off,
+        ntiles_off, total;
+};
+
+bool prefix_supported(int32_t num_kv_heads, int32_t group, int32_t head_dim) {
+    return head_dim == 128 && pkv::kv_heads_per_item(true, num_kv_heads, group) == 2;
+}
+
+PrefixLayout prefix_layout(size_t base, int32_t batch, int32_t num_kv_heads, int32_t group) {
+    PrefixLayout l{};
+    const size_t items = static_cast<size_t>(batch) * (num_kv_heads / 2);
+    const size_t heads = 2 * static_cast<size_t>(group);
+    const size_t B = static_cast<size_t>(batch);
+    l.pml_off = round_up(base, 256);
+    l.po_off = round_up(l.pml_off + items * heads * 4 * 4, 256);
+    l.link_off = round_up(l.po_off + items * heads * 128 * 4, 256);
+    l.leader_off = round_up(l.link_off + B * 4, 256);
+    l.refkey_off = round_up(l.leader_off + B * 4, 256);
+    l.ref_off = round_up(l.refkey_off + B * 8, 256);
+    l.share_off = round_up(l.ref_off + B * 4, 256);
+    l.cbeg_off = round_up(l.share_off + B * 4, 256);
+    l.tiles_off = round_up(l.cbeg_off + B * 4, 256);
+    l.ntiles_off = round_up(l.tiles_off + (B / 2 + 1) * 4 * 4, 256);
+    l.total = round_up(l.ntiles_off + 4, 256);
+    return l;
+}
+
+pkv_status prefix_impl(const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
+                       float k_scale, float v_scale, const int32_t* page_table, int32_t max_pages,
+                       const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
+                       int32_t num_kv_heads, int32_t head_dim, int32_t page_size,
+                       int32_t num_pages, float sm_scale, const uint8_t* abort, uint16_t* out,
+                       float* lse, void* workspace, size_t workspace_bytes, int32_t num_ctas,
+                       int32_t* chunk_begin_out, void* stream) {
+    pkv_status st = check_common_kv(batch, num_kv_heads, head_dim, page_size, num_pages, max_pages);
+    if (st != PKV_OK) return st;
+    if (num_q_heads < 1 || num_q_heads % num_kv_heads != 0)
+        return fail(PKV_ERR_INVALID_ARG, "num_q_heads (%d) must be a positive multiple of "
+                    "num_kv_heads (%d)", num_q_heads, num_kv_heads);
+    const int group = num_q_heads / num_kv_heads;
+    if (num_ctas < 0)
+        return fail(PKV_ERR_INVALID_ARG, "num_ctas must be >= 0 in shared-prefix mode (got %d)",
+                    num_ctas);
+    if (!prefix_supported(num_kv_heads, group, head_dim)) {
+        // no shared-prefix tile for this shape: the plain call, no chunk shared
+        st = attn_impl(true, q, k_cache, v_cache, k_scale, v_scale, page_table, max_pages,
+                       seq_lens, batch, num_q_heads, num_kv_heads, head_dim, page_size, num_pages,
+                       sm_scale, abort, out, lse, workspace, workspace_bytes, num_ctas, stream);
+        if (st != PKV_OK || chunk_begin_out == nullptr || batch == 0) return st;
+        cudaError_t e = cudaMemsetAsync(chunk_begin_out, 0, static_cast<size_t>(batch) * 4,
+                                        as_stream(stream));
+        return e == cudaSuccess ? PKV_OK : cuda_fail(e, "cudaMemsetAsync");
+    }
+    if (!(std::isfinite(sm_scale)))
+        return fail(PKV_ERR_INVALID_ARG, "sm_scale must be finite");
+    if (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
+        return fail(PKV_ERR_INVALID_ARG, "k_scale and v_scale must be finite and > 0");
+    if (batch == 0) return PKV_OK;
+    if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !out || !lse)
+        return fail(PKV_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 4) ||
+        !aligned(lse, 4) || !aligned(page_table, 4) || !aligned(seq_lens, 4) ||
+        (chunk_begin_out && !aligned(chunk_begin_out, 4)))
+        return fail(PKV_ERR_INVALID_ARG, "misaligned pointer (q and caches need 16 bytes)");
+    if (!workspace || !aligned(workspace, 256))
+        return fail(PKV_ERR_WORKSPACE, "workspace must be non-null and 256-byte aligned");
+
+    AttnPlan plan;
+    st = plan_attention(true, batch, num_kv_heads, group, head_dim, max_pages, page_size, num_ctas,
+                        &plan, /*allow_cluster=*/false);
+    if (st != PKV_OK) return st;
+    const pkv::WorkspaceLayout wl =
+        pkv::workspace_layout(batch, group, num_kv_heads, 2, head_dim, plan.grid);
+    const PrefixLayout pl = prefix_layout(wl.total, batch, num_kv_heads, group);
+    if (workspace_bytes < pl.total)
+        return fail(PKV_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes,
+                    pl.total);
+    const DeviceInfo* info = nullptr;
+    st = device_info(&info);
+    if (st != PKV_OK) return st;
+    {
+        static std::mutex m;
+        static bool ready[kMaxDevices] = {};
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+        std::lock_guard<std::mutex> lock(m);
+        if (!ready[dev]) {
+            e = pkv::prefix_set_smem_attr();
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+            ready[dev] = true;
+        }
+    }
+
+    const int box_rows = page_size < pkv::kChunkTokens ? page_size : pkv::kChunkTokens;
+    const int64_t rows = static_cast<int64_t>(num_pages) * num_kv_heads * page_size;
+    CUtensorMap tk_p, tv_p, tk, tv;
+    // the prefix pass loads one head's 64 rows (or a page of them) per box
+    st = encode_pool_map(&tk_p, k_cache, true, head_dim, rows, box_rows);
+    if (st != PKV_OK) return st;
+    st = encode_pool_map(&tv_p, v_cache, true, head_dim, rows, box_rows);
+    if (st != PKV_OK) return st;
+    // the split-K kernel's boxes (both heads of a 64-token page at once)
+    const int box_rows_s = page_size == pkv::kChunkTokens ? 2 * pkv::kChunkTokens : box_rows;
+    st = encode_pool_map(&tk, k_cache, true, head_dim, rows, box_rows_s);
+    if (st != PKV_OK) return st;
+    st = encode_pool_map(&tv, v_cache, true, head_dim, rows, box_rows_s);
+    if (st != PKV_OK) return st;
+
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const float qk_scale = sm_scale * k_scale * 1.4426950408889634f;
+    pkv::PrefixArgs pa{};
+    pa.q = q;
+    pa.page_table = page_table;
+    pa.seq_lens = seq_lens;
+    pa.abort = abort;
+    pa.status = reinterpret_cast<uint32_t*>(ws);
+    pa.pfx_ml = reinterpret_cast<float*>(ws + pl.pml_off);
+    pa.pfx_o = reinterpret_cast<float*>(ws + pl.po_off);
+    pa.link = reinterpret_cast<int32_t*>(ws + pl.link_off);
+    pa.leader = reinterpret_cast<int32_t*>(ws + pl.leader_off);
+    pa.refkey = reinterpret_cast<unsigned long long*>(ws + pl.refkey_off);
+    pa.ref = reinterpret_cast<int32_t*>(ws + pl.ref_off);
+    pa.share = reinterpret_cast<int32_t*>(ws + pl.share_off);
+    pa.chunk_begin = reinterpret_cast<int32_t*>(ws + pl.cbeg_off);
+    pa.tiles = reinterpret_cast<int32_t*>(ws + pl.tiles_off);
+    pa.num_tiles = reinterpret_cast<int32_t*>(ws + pl.ntiles_off);
+    pa.batch = batch;
+    pa.max_pages = max_pages;
+    pa.num_q_heads = num_q_heads;
+    pa.num_kv_heads = num_kv_heads;
+    pa.group = group;
+    pa.page_size = page_size;
+    pa.num_pages = num_pages;
+    pa.box_rows = box_rows;
+    pa.items_per_req = num_kv_heads / 2;
+    pa.members_per_tile = 64 / group;
+    pa.min_chunks = pkv::kPfxMinChunks;
+    pa.qk_scale = qk_scale;
+    pa.v_scale = v_scale;
+
+    cudaStream_t s = as_stream(stream);
+    cudaError_t e = pkv::launch_prefix_plan(s, pa);
+    if (e != cudaSuccess) return cuda_fail(e, "shared-prefix plan launch");
+    // two tile CTAs per SM, each looping over the tiles
+    e = pkv::launch_prefix_attn(2 * info->sms, s, tk_p, tv_p, pa);
+    if (e != cudaSuccess) return cuda_fail(e, "shared-prefix attention launch");
+
+    pkv::AttnArgs a{};
+    a.q = q;
+    a.page_table = page_table;
+    a.seq_lens = seq_lens;
+    a.abort = abort;
+    a.out = out;
+    a.lse = lse;
+    a.ws_status = reinterpret_cast<uint32_t*>(ws);
+    a.ws_ml = reinterpret_cast<float*>(ws + wl.ml_off);
+    a.ws_o = reinterpret_cast<float*>(ws + wl.o_off);
+    a.batch = batch;
+    a.max_pages = max_pages;
+    a.num_q_heads = num_q_heads;
+    a.num_kv_heads = num_kv_heads;
+    a.kv_per_item = 2;
+    a.items_per_req = num_kv_heads / 2;
+    a.group = group;
+    a.page_size = page_size;
+    a.num_pages = num_pages;
+    a.num_ctas = plan.grid;
+    a.box_rows = box_rows_s;
+    a.cluster_size = 0;
+    a.num_clusters = 0;
+    a.qk_scale = qk_scale;
+    a.v_scale = v_scale;
+    a.chunk_begin = pa.chunk_begin;
+    a.pfx_ml = pa.pfx_ml;
+    a.pfx_o = pa.pfx_o;
+    e = pkv::launch_attn_partial(true, head_dim, group_pad_of(group), 2, plan.grid, s, tk, tv, a);
+    if (e != cudaSuccess) return cuda_fail(e, "attention partial launch");
+    e = pkv::launch_attn_merge(head_dim, s, a);
+    if (e != cudaSuccess) return cuda_fail(e, "attention merge launch");
+    if (chunk_begin_out != nullptr) {
+        e = cudaMemcpyAsync(chunk_begin_out, pa.chunk_begin, static_cast<size_t>(batch) * 4,
+                            cudaMemcpyDeviceToDevice, s);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync");
     }
     return PKV_OK;
 }
@@ -657,6 +848,40 @@ pkv_status paged_decode_attn_fp8(const uint16_t* q, const uint8_t* k_cache,
     return attn_impl(true, q, k_cache, v_cache, k_scale, v_scale, page_table, max_pages, seq_lens,
                      batch, num_q_heads, num_kv_heads, head_dim, page_size, num_pages, sm_scale,
                      abort, out, lse, workspace, workspace_bytes, num_ctas, stream);
+}
+
+size_t paged_decode_attn_fp8_prefix_workspace_size(int32_t batch, int32_t num_q_heads,
+                                                   int32_t num_kv_heads, int32_t head_dim,
+                                                   int32_t num_ctas) {
+    if (batch < 0 || num_kv_heads < 1 || num_q_heads < 1 || num_q_heads % num_kv_heads != 0 ||
+        !supported_head_dim(head_dim) || num_ctas < 0) {
+        fail(PKV_ERR_INVALID_ARG, "invalid sizes for the shared-prefix workspace query");
+        return 0;
+    }
+    const int group = num_q_heads / num_kv_heads;
+    if (!prefix_supported(num_kv_heads, group, head_dim))
+        return paged_decode_attn_workspace_size(PKV_KV_FP8, batch, num_q_heads, num_kv_heads,
+                                                head_dim, num_ctas);
+    int grid = num_ctas;
+    if (grid == 0 && default_ctas(true, head_dim, group, 2, &grid) != PKV_OK) return 0;
+    const size_t base = pkv::workspace_layout(batch, group, num_kv_heads, 2, head_dim, grid).total;
+    return prefix_layout(base, batch, num_kv_heads, group).total;
+}
+
+pkv_status paged_decode_attn_fp8_prefix(const uint16_t* q, const uint8_t* k_cache,
+                                        const uint8_t* v_cache, float k_scale, float v_scale,
+                                        const int32_t* page_table, int32_t max_pages,
+                                        const int32_t* seq_lens, int32_t batch,
+                                        int32_t num_q_heads, int32_t num_kv_heads,
+                                        int32_t head_dim, int32_t page_size, int32_t num_pages,
+                                        float sm_scale, const uint8_t* abort, uint16_t* out,
+                                        float* lse, void* workspace, size_t workspace_bytes,
+                                        int32_t num_ctas, int32_t* chunk_begin_out,
+                                        void* stream) {
+    return prefix_impl(q, k_cache, v_cache, k_scale, v_scale, page_table, max_pages, seq_lens,
+                       batch, num_q_heads, num_kv_heads, head_dim, page_size, num_pages, sm_scale,
+                       abort, out, lse, workspace, workspace_bytes, num_ctas, chunk_begin_out,
+                       stream);
 }
 
 pkv_status paged_decode_attn_bf16(const uint16_t* q, const uint16_t* k_cache,

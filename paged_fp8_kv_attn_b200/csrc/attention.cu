@@ -124,12 +124,15 @@ struct Segment {
 
 // Walks a CTA's unit range [u, u_hi) segment by segment.  Every warp runs an
 // identical copy, so producer and consumers agree without communicating.
+// Units of an item are its chunks from the request's first chunk (0, or
+// chunk_begin[b] in shared-prefix mode) to its last.
 struct Walker {
     const int32_t* seq_lens;
+    const int32_t* chunk_begin;   // null: every request from chunk 0
     int64_t max_tokens;
     int num_kv_heads;
     int batch;
-    int b, h, ch, n, L;
+    int b, h, ch, n, L, cb;
     int64_t u, u_hi;
 
     __device__ __forceinline__ int chunks_of(int32_t len) const {
@@ -137,17 +140,26 @@ struct Walker {
                    ? (len + kChunkTokens - 1) / kChunkTokens
                    : 0;
     }
+    __device__ __forceinline__ int begin_of(int bb) const {
+        return chunk_begin != nullptr ? chunk_begin[bb] : 0;
+    }
+    // units of one item of request bb
+    __device__ __forceinline__ int units_of(int bb, int32_t len) const {
+        const int c = chunks_of(len);
+        return c > 0 ? c - begin_of(bb) : 0;
+    }
     __device__ __forceinline__ void init(int b0, int pre0, int64_t ulo, int64_t uhi) {
         u = ulo;
         u_hi = uhi;
         b = b0;
-        h = ch = n = L = 0;
+        h = ch = n = L = cb = 0;
         if (u < u_hi) {
             L = seq_lens[b];
             n = chunks_of(L);
+            cb = begin_of(b);
             const int64_t off = ulo - static_cast<int64_t>(num_kv_heads) * pre0;
-            h = static_cast<int>(off / n);
-            ch = static_cast<int>(off % n);
+            h = static_cast<int>(off / (n - cb));
+            ch = cb + static_cast<int>(off % (n - cb));
         }
     }
     __device__ __forceinline__ bool next(Segment& s) {
@@ -166,7 +178,6 @@ struct Walker {
         u += take;
         ch += take;
         if (u < u_hi && ch == n) {
-            ch = 0;
             if (++h == num_kv_heads) {
                 h = 0;
                 do {
@@ -174,7 +185,9 @@ struct Walker {
                     L = seq_lens[b];
                     n = chunks_of(L);
                 } while (n == 0 && b + 1 < batch);
+                cb = begin_of(b);
             }
+            ch = cb;
         }
         return true;
     }
@@ -402,11 +415,15 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int64_t max_tokens = static_cast<int64_t>(a.max_pages) * a.page_size;
 
     launch_dependents();
+    // Shared-prefix mode: the chunk begins the partition needs come from the
+    // plan kernels that precede this one.
+    if (a.chunk_begin != nullptr) grid_dependency_wait();
     // The call's status word starts at zero.  Clearing it before the grid
     // dependency wait is safe: no kernel reads it (the caller reads it in
     // stream order, after the call), and a bounded wait of this call can only
     // expire seconds after CTA 0, the first to be scheduled, has run this.
-    if (blockIdx.x == 0 && tid == 0) *a.ws_status = 0u;
+    // (in shared-prefix mode the plan kernel that opens the call clears it)
+    if (blockIdx.x == 0 && tid == 0 && a.chunk_begin == nullptr) *a.ws_status = 0u;
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full_bar[s], 1);
@@ -422,6 +439,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
     // ---- partition: exclusive scan of chunk counts over the batch --------
     Walker walk;
     walk.seq_lens = a.seq_lens;
+    walk.chunk_begin = a.chunk_begin;
     walk.max_tokens = max_tokens;
     walk.num_kv_heads = IPR;
     walk.batch = B;
@@ -429,7 +447,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int b_lo = min(B, tid * per);
     const int b_hi = min(B, b_lo + per);
     int local = 0;
-    for (int b = b_lo; b < b_hi; ++b) local += walk.chunks_of(a.seq_lens[b]);
+    for (int b = b_lo; b < b_hi; ++b) local += walk.units_of(b, a.seq_lens[b]);
     int incl = local;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -469,7 +487,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int i1 = static_cast<int>(static_cast<int64_t>(cid + 1) * I / a.num_clusters);
         int run = run0;
         for (int b = b_lo; b < b_hi; ++b) {
-            const int n = walk.chunks_of(a.seq_lens[b]);
+            const int n = walk.units_of(b, a.seq_lens[b]);
             if (b == i0 / IPR) { scratch[11] = run; scratch[12] = n; }
             if (b == i1 / IPR) { scratch[13] = run; scratch[14] = n; }
             run += n;
@@ -485,7 +503,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
     {
         int run = run0;
         for (int b = b_lo; b < b_hi; ++b) {
-            const int n = walk.chunks_of(a.seq_lens[b]);
+            const int n = walk.units_of(b, a.seq_lens[b]);
             if (n > 0 && u_lo < u_hi && static_cast<int64_t>(IPR) * run <= u_lo &&
                 u_lo < static_cast<int64_t>(IPR) * (run + n)) {
                 scratch[8] = b;
@@ -1239,17 +1257,21 @@ attn_merge_kernel(const AttnArgs a) {
     if (hq0 >= G) return;
     const int NH = min(kHPC, G - hq0);       // this CTA's heads
     const int64_t head0 = static_cast<int64_t>(b) * a.num_q_heads + h * G + hq0;
-    // Chunk counts of the requests before b, of b and of the batch, from the
-    // lengths (an input no kernel writes), before the grid-dependency wait:
-    // this overlaps the partial kernel's tail.
+    // Shared-prefix mode: the chunk begins come from the plan kernels, which
+    // precede the partial kernel.
+    if (a.chunk_begin != nullptr) grid_dependency_wait();
+    // Unit counts (chunks from the request's first) of the requests before b,
+    // of b and of the batch, from the lengths (an input no kernel writes),
+    // before the grid-dependency wait: this overlaps the partial kernel's tail.
     {
         const int64_t max_tokens = static_cast<int64_t>(a.max_pages) * a.page_size;
         int pre_part = 0, tot_part = 0;
         for (int bb = tid; bb < a.batch; bb += kMergeThreads) {
             const int32_t len = a.seq_lens[bb];
-            const int nb = (len >= 1 && static_cast<int64_t>(len) <= max_tokens)
-                               ? (len + kChunkTokens - 1) / kChunkTokens
-                               : 0;
+            int nb = (len >= 1 && static_cast<int64_t>(len) <= max_tokens)
+                         ? (len + kChunkTokens - 1) / kChunkTokens
+                         : 0;
+            if (nb > 0 && a.chunk_begin != nullptr) nb -= a.chunk_begin[bb];
             tot_part += nb;
             if (bb < b) pre_part += nb;
             if (bb == b) s_nb = nb;
@@ -1286,10 +1308,14 @@ attn_merge_kernel(const AttnArgs a) {
     const int64_t u0 = static_cast<int64_t>(IPR) * pre + static_cast<int64_t>(h) * n;
     const int64_t c0 = cta_of_unit(u0, U, NE);
     const int64_t c1 = cta_of_unit(u0 + n - 1, U, NE);
-    if (c0 == c1) return;   // finished by the partial kernel
+    // the shared-prefix pass's record of this item, if it has one: one more
+    // segment, after the CTAs' ones
+    const int pfx = (a.chunk_begin != nullptr && a.chunk_begin[b] > 0) ? 1 : 0;
+    if (c0 == c1 && pfx == 0) return;   // finished by the partial kernel
     const int nseg = static_cast<int>(c1 - c0 + 1);
+    const int ntot = nseg + pfx;
     const int64_t stride = static_cast<int64_t>(G) * kD;
-    if (nseg <= kMergeFastSegs) {
+    if (ntot <= kMergeFastSegs) {
         // Few segments: thread -> (head, 4 dims); every segment's (m, l, lr)
         // and output quad are requested at once (one round trip).
         constexpr int kQuads = kD / 4;
@@ -1298,18 +1324,21 @@ attn_merge_kernel(const AttnArgs a) {
         float4 ml[kMergeFastSegs], x[kMergeFastSegs];
 #pragma unroll
         for (int k = 0; k < kMergeFastSegs; ++k) {
-            if (k < nseg) {
+            if (k < ntot) {
                 const int64_t slot = c0 + k + item;
-                ml[k] = *reinterpret_cast<const float4*>(a.ws_ml + (slot * G + hq0 + hq) * 4);
-                x[k] = *reinterpret_cast<const float4*>(a.ws_o + slot * stride +
-                                                        static_cast<int64_t>(hq0 + hq) * kD + 4 * q);
+                const float* mp = k < nseg ? a.ws_ml + (slot * G + hq0 + hq) * 4
+                                           : a.pfx_ml + (static_cast<int64_t>(item) * G + hq0 + hq) * 4;
+                const float* op = (k < nseg ? a.ws_o + slot * stride : a.pfx_o + item * stride) +
+                                  static_cast<int64_t>(hq0 + hq) * kD + 4 * q;
+                ml[k] = *reinterpret_cast<const float4*>(mp);
+                x[k] = *reinterpret_cast<const float4*>(op);
             }
         }
         float M = kNegInf;
         int dead = 0;
 #pragma unroll
         for (int k = 0; k < kMergeFastSegs; ++k) {
-            if (k < nseg) {
+            if (k < ntot) {
                 M = fmaxf(M, ml[k].x);
                 dead |= ml[k].y < 0.f;
             }
@@ -1318,7 +1347,7 @@ attn_merge_kernel(const AttnArgs a) {
         float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int k = 0; k < kMergeFastSegs; ++k) {
-            if (k < nseg) {
+            if (k < ntot) {
                 const float wt = (ml[k].x == kNegInf) ? 0.f : exp2f(ml[k].x - M);
                 Lsum += wt * ml[k].y;
                 Lr += wt * ml[k].z;
@@ -1350,14 +1379,19 @@ attn_merge_kernel(const AttnArgs a) {
 #pragma unroll
     for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
 
-    for (int t0 = 0; t0 < nseg; t0 += kMergeTile) {
-        const int tn = min(kMergeTile, nseg - t0);
+    // tiles of the CTAs' segments, then (shared-prefix mode) a tile of the
+    // prefix record alone
+    for (int t0 = 0; t0 < ntot;) {
+        const bool ptile = t0 >= nseg;
+        const int tn = ptile ? 1 : min(kMergeTile, nseg - t0);
         // (1) the tile's (m, l, lr) of this CTA's heads into shared memory:
         // one round trip
         for (int e = tid; e < tn * NH; e += kMergeThreads) {
             const int sg = e / NH, hq = e % NH;
             const int64_t slot = c0 + t0 + sg + item;
-            const float4 ml = *reinterpret_cast<const float4*>(a.ws_ml + (slot * G + hq0 + hq) * 4);
+            const float* mp = ptile ? a.pfx_ml + (static_cast<int64_t>(item) * G + hq0 + hq) * 4
+                                    : a.ws_ml + (slot * G + hq0 + hq) * 4;
+            const float4 ml = *reinterpret_cast<const float4*>(mp);
             s_w[sg][hq] = ml.x;
             s_l[sg][hq] = ml.y;
             s_lr[sg][hq] = ml.z;
@@ -1402,7 +1436,8 @@ attn_merge_kernel(const AttnArgs a) {
         }
         __syncthreads();
         // (3) outputs: segment-major, kPer x kUnroll independent loads in flight
-        const float* base = a.ws_o + (c0 + t0 + item) * stride + static_cast<int64_t>(hq0) * kD;
+        const float* base = (ptile ? a.pfx_o + item * stride : a.ws_o + (c0 + t0 + item) * stride) +
+                            static_cast<int64_t>(hq0) * kD;
 #pragma unroll
         for (int k = 0; k < kPer; ++k) {
             const int e = tid + k * kMergeThreads;
@@ -1426,6 +1461,7 @@ attn_merge_kernel(const AttnArgs a) {
             }
         }
         __syncthreads();
+        t0 += tn;
     }
 #pragma unroll
     for (int k = 0; k < kPer; ++k) {

@@ -42,7 +42,57 @@ struct AttnArgs {
     int32_t num_clusters;       // cluster mode: clusters in the grid
     float qk_scale;             // sm_scale * k_scale * log2(e)
     float v_scale;              // per-tensor V scale (1 for BF16)
+    // Shared-prefix mode (all null otherwise): the split-K kernels cover
+    // chunks [chunk_begin[b], n_b) of request b; the shared-prefix pass left
+    // one record per item of the requests with chunk_begin[b] > 0, which the
+    // merge kernel adds to the item's own records.
+    const int32_t* chunk_begin;  // [B]
+    const float* pfx_ml;         // [items][G][4]
+    const float* pfx_o;          // [items][G][D]
 };
+
+// Shared-prefix pass (prefix.cu): FP8, head_dim 128, two KV heads per item.
+constexpr int kPfxRows = 128;         // rows of one tensor-core tile (query heads of its members)
+constexpr int kPfxThreads = 160;      // 4 row warps + 1 TMA warp
+constexpr int kPfxPlanThreads = 1024;
+constexpr int kPfxMinChunks = 4;      // shared chunks that make a request join a group
+
+struct PrefixArgs {
+    const uint16_t* q;          // [B][Hq][128] bf16
+    const int32_t* page_table;  // [B][MP]
+    const int32_t* seq_lens;    // [B]
+    const uint8_t* abort;       // [B] or null
+    uint32_t* status;           // workspace status word
+    float* pfx_ml;              // [items][2G][4]
+    float* pfx_o;               // [items][2G][128]
+    int32_t* link;              // [B]  shared chunks with request b - 1
+    int32_t* leader;            // [B]  first request of b's group
+    unsigned long long* refkey; // [B]  per group leader: (full chunks + 1, ~index) of its reference
+    int32_t* ref;               // [B]  the reference row of b's group
+    int32_t* share;             // [B]  shared chunks with the reference row
+    int32_t* chunk_begin;       // [B]
+    int32_t* tiles;             // [B / 2 + 1][4]: page-table row, first member, members, chunks
+    int32_t* num_tiles;         // [1]
+    int32_t batch;
+    int32_t max_pages;
+    int32_t num_q_heads;
+    int32_t num_kv_heads;
+    int32_t group;
+    int32_t page_size;
+    int32_t num_pages;
+    int32_t box_rows;           // min(page_size, 64)
+    int32_t items_per_req;      // num_kv_heads / 2
+    int32_t members_per_tile;   // 64 / group
+    int32_t min_chunks;
+    float qk_scale;             // sm_scale * k_scale * log2(e)
+    float v_scale;
+};
+size_t prefix_attn_smem_bytes();
+cudaError_t prefix_set_smem_attr();
+// the plan kernels (two launches)
+cudaError_t launch_prefix_plan(cudaStream_t stream, const PrefixArgs& args);
+cudaError_t launch_prefix_attn(int grid, cudaStream_t stream, const CUtensorMap& tmap_k,
+                               const CUtensorMap& tmap_v, const PrefixArgs& args);
 
 // Sets the message pkv_last_error() returns on this thread.
 void set_last_error(const char* message);

@@ -160,6 +160,16 @@ def custom(lens, page_size=64, num_q_heads=64, num_kv_heads=8, head_dim=128, see
                    head_dim, device)
 
 
+def from_table(lens, page_table, num_pages, page_size=64, num_q_heads=64, num_kv_heads=8,
+               head_dim=128, seed=0, device="cpu", name="from_table") -> DecodeBatch:
+    """Given lengths and page table (pages may be shared between rows); the
+    contents of the pools, queries and new tokens are drawn as everywhere."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    table = np.asarray(page_table, dtype=np.int32)
+    return _finish(name, seed, rng, lens, table, num_pages, page_size, num_q_heads, num_kv_heads,
+                   head_dim, device)
+
+
 def tiny_decode(seed=1, device="cpu") -> DecodeBatch:
     """2 sequences of 37 and 100 tokens, P=16, Hq=4, Hkv=1, D=64, a pool of 16
     pages assigned by a seeded permutation, random tags with one stale

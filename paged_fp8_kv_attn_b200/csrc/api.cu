@@ -398,8 +398,8 @@ pkv_status attn_impl(bool fp8, const uint16_t* q, const void* k_cache, const voi
 // Shared-prefix mode: the split-K workspace, then the prefix records and the
 // plan arrays.
 struct PrefixLayout {
-    size_t pml_off, po_off, link_off, leader_off, refkey_off, ref_off, share_off, cbeg_off, tiles_off,
-        ntiles_off, total;
+    size_t pml_off, po_off, link_off, leader_off, refkey_off, ref_off, share_off, pshare_off,
+        cbeg_off, tiles_off, ntiles_off, total;
 };
 
 bool prefix_supported(int32_t num_kv_heads, int32_t group, int32_t head_dim) {
@@ -418,7 +418,8 @@ PrefixLayout prefix_layout(size_t base, int32_t batch, int32_t num_kv_heads, int
     l.refkey_off = round_up(l.leader_off + B * 4, 256);
     l.ref_off = round_up(l.refkey_off + B * 8, 256);
     l.share_off = round_up(l.ref_off + B * 4, 256);
-    l.cbeg_off = round_up(l.share_off + B * 4, 256);
+    l.pshare_off = round_up(l.share_off + B * 4, 256);
+    l.cbeg_off = round_up(l.pshare_off + B * 4, 256);
     l.tiles_off = round_up(l.cbeg_off + B * 4, 256);
     l.ntiles_off = round_up(l.tiles_off + (B / 2 + 1) * 4 * 4, 256);
     l.total = round_up(l.ntiles_off + 4, 256);
@@ -469,27 +470,40 @@ pkv_status prefix_impl(const uint16_t* q, const uint8_t* k_cache, const uint8_t*
     st = plan_attention(true, batch, num_kv_heads, group, head_dim, max_pages, page_size, num_ctas,
                         &plan, /*allow_cluster=*/false);
     if (st != PKV_OK) return st;
+    const DeviceInfo* info = nullptr;
+    st = device_info(&info);
+    if (st != PKV_OK) return st;
     const pkv::WorkspaceLayout wl =
         pkv::workspace_layout(batch, group, num_kv_heads, 2, head_dim, plan.grid);
     const PrefixLayout pl = prefix_layout(wl.total, batch, num_kv_heads, group);
     if (workspace_bytes < pl.total)
         return fail(PKV_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes,
                     pl.total);
-    const DeviceInfo* info = nullptr;
-    st = device_info(&info);
-    if (st != PKV_OK) return st;
+    int pfx_blocks = 1;   // resident shared-prefix CTAs per SM
     {
         static std::mutex m;
-        static bool ready[kMaxDevices] = {};
+        static int blocks[kMaxDevices] = {};
         int dev = 0;
         cudaError_t e = cudaGetDevice(&dev);
         if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
         std::lock_guard<std::mutex> lock(m);
-        if (!ready[dev]) {
+        if (blocks[dev] == 0) {
             e = pkv::prefix_set_smem_attr();
             if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-            ready[dev] = true;
+            int n = 0;
+            e = pkv::prefix_occupancy(&n);
+            if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
+            if (n < 1) {
+                int regs = 0, local = 0, maxt = 0;
+                pkv::prefix_attributes(&regs, &local, &maxt);
+                return fail(PKV_ERR_UNSUPPORTED,
+                            "the shared-prefix kernel does not fit on an SM of this device "
+                            "(%d registers, %d local bytes per thread, at most %d threads per CTA)",
+                            regs, local, maxt);
+            }
+            blocks[dev] = n;
         }
+        pfx_blocks = blocks[dev];
     }
 
     const int box_rows = page_size < pkv::kChunkTokens ? page_size : pkv::kChunkTokens;
@@ -522,6 +536,7 @@ pkv_status prefix_impl(const uint16_t* q, const uint8_t* k_cache, const uint8_t*
     pa.refkey = reinterpret_cast<unsigned long long*>(ws + pl.refkey_off);
     pa.ref = reinterpret_cast<int32_t*>(ws + pl.ref_off);
     pa.share = reinterpret_cast<int32_t*>(ws + pl.share_off);
+    pa.pshare = reinterpret_cast<int32_t*>(ws + pl.pshare_off);
     pa.chunk_begin = reinterpret_cast<int32_t*>(ws + pl.cbeg_off);
     pa.tiles = reinterpret_cast<int32_t*>(ws + pl.tiles_off);
     pa.num_tiles = reinterpret_cast<int32_t*>(ws + pl.ntiles_off);
@@ -536,14 +551,17 @@ pkv_status prefix_impl(const uint16_t* q, const uint8_t* k_cache, const uint8_t*
     pa.items_per_req = num_kv_heads / 2;
     pa.members_per_tile = 64 / group;
     pa.min_chunks = pkv::kPfxMinChunks;
+    pa.tail_chunks = pkv::kPfxTailChunks;
+    pa.out = out;
+    pa.lse = lse;
     pa.qk_scale = qk_scale;
     pa.v_scale = v_scale;
 
     cudaStream_t s = as_stream(stream);
     cudaError_t e = pkv::launch_prefix_plan(s, pa);
     if (e != cudaSuccess) return cuda_fail(e, "shared-prefix plan launch");
-    // two tile CTAs per SM, each looping over the tiles
-    e = pkv::launch_prefix_attn(2 * info->sms, s, tk_p, tv_p, pa);
+    // one wave of tile CTAs, each looping over the tiles
+    e = pkv::launch_prefix_attn(pfx_blocks * info->sms, s, tk_p, tv_p, pa);
     if (e != cudaSuccess) return cuda_fail(e, "shared-prefix attention launch");
 
     pkv::AttnArgs a{};

@@ -180,12 +180,14 @@ struct Walker {
         if (u < u_hi && ch == n) {
             if (++h == num_kv_heads) {
                 h = 0;
+                // (requests with no units: invalid lengths, and in shared-prefix
+                // mode requests the shared pass finishes)
                 do {
                     ++b;
                     L = seq_lens[b];
                     n = chunks_of(L);
-                } while (n == 0 && b + 1 < batch);
-                cb = begin_of(b);
+                    cb = begin_of(b);
+                } while ((n == 0 || cb >= n) && b + 1 < batch);
             }
             ch = cb;
         }
@@ -1245,7 +1247,7 @@ attn_merge_kernel(const AttnArgs a) {
     __shared__ float s_lr[kMergeTile][kHPC];  // lr_s (weights as rounded for the PV product)
     __shared__ float s_m[kHPC], s_sum[kHPC], s_sumr[kHPC], s_scale[kHPC];
     __shared__ int s_dead;
-    __shared__ int s_red[2][kMergeThreads / 32], s_nb;
+    __shared__ int s_red[2][kMergeThreads / 32], s_nb, s_nc;
     launch_dependents();
     const int tid = threadIdx.x;
     constexpr int kGroups = 16 / kHPC;       // CTAs per item
@@ -1271,7 +1273,9 @@ attn_merge_kernel(const AttnArgs a) {
             int nb = (len >= 1 && static_cast<int64_t>(len) <= max_tokens)
                          ? (len + kChunkTokens - 1) / kChunkTokens
                          : 0;
+            const int nc = nb;
             if (nb > 0 && a.chunk_begin != nullptr) nb -= a.chunk_begin[bb];
+            if (bb == b) s_nc = nc;
             tot_part += nb;
             if (bb < b) pre_part += nb;
             if (bb == b) s_nb = nb;
@@ -1295,6 +1299,7 @@ attn_merge_kernel(const AttnArgs a) {
     }
     const int32_t n = s_nb;
     grid_dependency_wait();
+    if (n == 0 && s_nc > 0) return;   // finished by the shared-prefix pass
     if (n == 0) {
         for (int e = tid; e < NH * kD; e += kMergeThreads) {
             const int hq = e / kD, d = e % kD;

@@ -53,9 +53,11 @@ struct AttnArgs {
 
 // Shared-prefix pass (prefix.cu): FP8, head_dim 128, two KV heads per item.
 constexpr int kPfxRows = 128;         // rows of one tensor-core tile (query heads of its members)
-constexpr int kPfxThreads = 160;      // 4 row warps + 1 TMA warp
+constexpr int kPfxRowThreads = 256;   // two threads per tile row
+constexpr int kPfxThreads = 2 * (kPfxRowThreads + 32);   // two halves of 8 row warps + 1 TMA warp
 constexpr int kPfxPlanThreads = 1024;
 constexpr int kPfxMinChunks = 4;      // shared chunks that make a request join a group
+constexpr int kPfxTailChunks = 2;     // own chunks a tile finishes for a member
 
 struct PrefixArgs {
     const uint16_t* q;          // [B][Hq][128] bf16
@@ -70,7 +72,8 @@ struct PrefixArgs {
     unsigned long long* refkey; // [B]  per group leader: (full chunks + 1, ~index) of its reference
     int32_t* ref;               // [B]  the reference row of b's group
     int32_t* share;             // [B]  shared chunks with the reference row
-    int32_t* chunk_begin;       // [B]
+    int32_t* pshare;            // [B]  chunks the shared pass covers for b's rows
+    int32_t* chunk_begin;       // [B]  first chunk of the split-K kernels (n_b: none left)
     int32_t* tiles;             // [B / 2 + 1][4]: page-table row, first member, members, chunks
     int32_t* num_tiles;         // [1]
     int32_t batch;
@@ -84,11 +87,17 @@ struct PrefixArgs {
     int32_t items_per_req;      // num_kv_heads / 2
     int32_t members_per_tile;   // 64 / group
     int32_t min_chunks;
+    int32_t tail_chunks;        // a member with at most this many chunks after its shared
+                                // ones is finished by its tile (final outputs, no merge)
     float qk_scale;             // sm_scale * k_scale * log2(e)
     float v_scale;
+    uint16_t* out;              // [B][Hq][128] bf16 (members the tile finishes)
+    float* lse;                 // [B][Hq]
 };
 size_t prefix_attn_smem_bytes();
 cudaError_t prefix_set_smem_attr();
+cudaError_t prefix_occupancy(int* blocks_per_sm);
+cudaError_t prefix_attributes(int* regs, int* local_bytes, int* max_threads);
 // the plan kernels (two launches)
 cudaError_t launch_prefix_plan(cudaStream_t stream, const PrefixArgs& args);
 cudaError_t launch_prefix_attn(int grid, cudaStream_t stream, const CUtensorMap& tmap_k,

@@ -50,6 +50,7 @@ namespace {
 
 constexpr float kPfxLog2RescaleThreshold = 8.0f;
 constexpr float kPfxNegInf = -__builtin_huge_valf();
+constexpr float kPfxLn2 = 0.6931471805599453f;
 constexpr int kPfxD = 128;
 // shared memory: Q tile, converted K (token rows) or V^T (dim rows) tile,
 // raw FP8 K and V of one chunk of both heads, barriers
@@ -60,8 +61,15 @@ constexpr int kPfxRawBytes = 2 * kChunkTokens * kPfxD;   // one FP8 operand of b
 constexpr int kPfxRawKOff = kPfxKVOff + 2 * kPfxAtom;
 constexpr int kPfxRawVOff = kPfxRawKOff + kPfxRawBytes;
 constexpr int kPfxBarOff = kPfxRawVOff + kPfxRawBytes;
-constexpr int kPfxSmemBytes = kPfxBarOff + 5 * 8 + 16 + 1024;   // + alignment slack
-constexpr uint32_t kPfxTmemCols = 256;   // S / P: columns 0-127; O: 128-255
+constexpr int kPfxXOff = kPfxBarOff + 64;
+// The CTA holds two independent halves (a CTA that allocates tensor memory
+// gets an SM to itself), each with its own 8 row warps, TMA warp, shared
+// memory region and 256 tensor-memory columns.
+constexpr int kPfxHalfBytes = (kPfxXOff + 3 * kPfxRowThreads * 4 + 1023) / 1024 * 1024;
+constexpr int kPfxSmemBytes = 2 * kPfxHalfBytes + 1024;   // + alignment slack
+constexpr int kPfxRowWarps = kPfxRowThreads / 32;
+constexpr int kPfxHalfWarps = kPfxRowWarps + 1;
+constexpr uint32_t kPfxTmemCols = 512;   // per half: S / P 128 columns, then O 128
 constexpr uint32_t kPfxOCol = 128;
 
 }  // namespace
@@ -229,8 +237,19 @@ __global__ void __launch_bounds__(kPfxPlanThreads) prefix_tile_kernel(const Pref
             d[2] = nm;     // members
             d[3] = mx;     // chunks
         }
-        for (int k = 0; k < nm; ++k)
-            a.chunk_begin[b + k] = tile ? (b + k == r ? mx : a.share[b + k]) : 0;
+        for (int k = 0; k < nm; ++k) {
+            const int m = b + k;
+            const int ps = tile ? (m == r ? mx : a.share[m]) : 0;
+            int cbeg = ps;
+            if (tile) {
+                // a member with few chunks after its shared ones is finished by
+                // the tile itself
+                const int n = full_chunks(a, m) + 1;
+                if (n - ps <= a.tail_chunks) cbeg = n;
+            }
+            a.pshare[m] = ps;
+            a.chunk_begin[m] = cbeg;
+        }
     }
     __syncthreads();
     if (tid == 0) *a.num_tiles = s_count;
@@ -256,12 +275,23 @@ __device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
     asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
-// The 64 tokens of chunk c of KV head h (rows of the [page][kv_head][slot][dim]
-// pool) into 64 consecutive 128-byte rows at dst, as boxes of box_rows rows.
+// Boxes of chunk c that lie in the request's first `npages` pages (all of
+// them except in the last chunk of a request with pages under 64 tokens).
+__device__ __forceinline__ int chunk_boxes(const PrefixArgs& a, int c, int npages) {
+    const int br = a.box_rows;
+    int n = 0;
+    for (int i = 0; i < kChunkTokens / br; ++i)
+        if ((c * kChunkTokens + i * br) / a.page_size < npages) ++n;
+    return n;
+}
+
+// The tokens of chunk c of KV head h (rows of the [page][kv_head][slot][dim]
+// pool) into consecutive 128-byte rows at dst, as `boxes` boxes of box_rows
+// rows (the later rows keep what they held: those tokens are masked).
 __device__ __forceinline__ void load_chunk_rows(uint32_t dst, const CUtensorMap* map, const PrefixArgs& a,
-                                                const int32_t* prow, int c, int h, uint64_t* bar) {
+                                                const int32_t* prow, int c, int h, int boxes, uint64_t* bar) {
     const int P = a.page_size, br = a.box_rows;
-    for (int i = 0; i < kChunkTokens / br; ++i) {
+    for (int i = 0; i < boxes; ++i) {
         const int tok0 = c * kChunkTokens + i * br;
         int32_t pid = prow[tok0 / P];
         // (the plan admits only chunks whose page ids are valid; the clamp
@@ -274,31 +304,42 @@ __device__ __forceinline__ void load_chunk_rows(uint32_t dst, const CUtensorMap*
 
 }  // namespace
 
-__global__ void __launch_bounds__(kPfxThreads, 2)
+// (at most 96 registers: 576 threads in one CTA, registers allocated per 4 warps)
+__global__ void __maxnreg__(96)
 prefix_attn_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                    const __grid_constant__ PrefixArgs a) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
+    uint8_t* smem0 = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int half = warp / kPfxHalfWarps;
+    const int lwarp = warp - half * kPfxHalfWarps;            // warp within the half
+    uint8_t* smem = smem0 + half * kPfxHalfBytes;
     uint64_t* full_k = reinterpret_cast<uint64_t*>(smem + kPfxBarOff);
     uint64_t* empty_k = full_k + 1;
     uint64_t* full_v = full_k + 2;
     uint64_t* empty_v = full_k + 3;
     uint64_t* mma_bar = full_k + 4;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(full_k + 5);
-    volatile int* failed = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-    const int tid = threadIdx.x;
-    const int warp = tid >> 5;
-    const int lane = tid & 31;
+    // (shared by both halves: in the first half's region)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem0 + kPfxBarOff + 40);
+    volatile int* failed = reinterpret_cast<volatile int*>(smem0 + kPfxBarOff + 44);
+    // exchange between the two threads of a row: maxima, then l and lr
+    float* s_xmax = reinterpret_cast<float*>(smem + kPfxXOff);   // [256]
+    float* s_xl = s_xmax + kPfxRowThreads;                       // [256]
+    float* s_xlr = s_xl + kPfxRowThreads;                        // [256]
 
     launch_dependents();
     if (tid == 0) {
-        mbar_init(full_k, 1);
-        mbar_init(empty_k, 4);
-        mbar_init(full_v, 1);
-        mbar_init(empty_v, 4);
-        mbar_init(mma_bar, 1);
+        for (int hf = 0; hf < 2; ++hf) {
+            uint64_t* fb = reinterpret_cast<uint64_t*>(smem0 + hf * kPfxHalfBytes + kPfxBarOff);
+            mbar_init(fb, 1);                   // K full
+            mbar_init(fb + 1, kPfxRowWarps);    // K empty
+            mbar_init(fb + 2, 1);               // V full
+            mbar_init(fb + 3, kPfxRowWarps);    // V empty
+            mbar_init(fb + 4, 1);               // tensor-core commits
+        }
         *failed = 0;
         fence_barrier_init();
     }
@@ -309,74 +350,105 @@ prefix_attn_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_cons
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem = *tmem_slot + 256u * static_cast<uint32_t>(half);   // this half's columns
 
     // the plan and the abort flags come from the preceding kernels
     grid_dependency_wait();
     const int IPR = a.items_per_req;
     const int total = *a.num_tiles * IPR;
     const uint32_t base = smem_addr(smem);
+    // A tile's steps: its shared chunks (read through the reference row), then
+    // for each member the tile finishes (chunk_begin = all its chunks) the
+    // chunks after its shared ones (read through its own row).
+    auto n_chunks = [&](int bb) { return (a.seq_lens[bb] + kChunkTokens - 1) / kChunkTokens; };
+    auto finished = [&](int bb) { return a.chunk_begin[bb] == n_chunks(bb); };
 
-    if (warp == 4) {
+    if (lwarp == kPfxRowWarps) {
         // ================= producer =================
         if (lane == 0) {
             prefetch_tensormap(&tmap_k);
             prefetch_tensormap(&tmap_v);
             uint32_t it = 0;
-            for (int ti = blockIdx.x; ti < total; ti += gridDim.x) {
+            auto load = [&](const int32_t* prow, int c, int p, int npages) {
+                const int boxes = chunk_boxes(a, c, npages);
+                const uint32_t bytes = 2u * boxes * a.box_rows * 128u;
+                if (it > 0 && !gemv_wait(empty_k, (it - 1) & 1, failed, a.status)) return false;
+                mbar_arrive_expect_tx(full_k, bytes);
+                for (int hh = 0; hh < 2; ++hh)
+                    load_chunk_rows(base + kPfxRawKOff + hh * (kPfxRawBytes / 2), &tmap_k, a, prow, c, 2 * p + hh,
+                                    boxes, full_k);
+                if (it > 0 && !gemv_wait(empty_v, (it - 1) & 1, failed, a.status)) return false;
+                mbar_arrive_expect_tx(full_v, bytes);
+                for (int hh = 0; hh < 2; ++hh)
+                    load_chunk_rows(base + kPfxRawVOff + hh * (kPfxRawBytes / 2), &tmap_v, a, prow, c, 2 * p + hh,
+                                    boxes, full_v);
+                ++it;
+                return true;
+            };
+            for (int ti = 2 * blockIdx.x + half; ti < total && !*failed; ti += 2 * gridDim.x) {
                 const int t = ti / IPR, p = ti - t * IPR;
                 const int32_t* prow = a.page_table + static_cast<int64_t>(a.tiles[4 * t]) * a.max_pages;
-                const int nch = a.tiles[4 * t + 3];
-                for (int c = 0; c < nch; ++c, ++it) {
-                    if (it > 0 && !gemv_wait(empty_k, (it - 1) & 1, failed, a.status)) break;
-                    mbar_arrive_expect_tx(full_k, kPfxRawBytes);
-                    for (int hh = 0; hh < 2; ++hh)
-                        load_chunk_rows(base + kPfxRawKOff + hh * (kPfxRawBytes / 2), &tmap_k, a, prow, c,
-                                        2 * p + hh, full_k);
-                    if (it > 0 && !gemv_wait(empty_v, (it - 1) & 1, failed, a.status)) break;
-                    mbar_arrive_expect_tx(full_v, kPfxRawBytes);
-                    for (int hh = 0; hh < 2; ++hh)
-                        load_chunk_rows(base + kPfxRawVOff + hh * (kPfxRawBytes / 2), &tmap_v, a, prow, c,
-                                        2 * p + hh, full_v);
+                const int b_first = a.tiles[4 * t + 1], nm = a.tiles[4 * t + 2], nch = a.tiles[4 * t + 3];
+                for (int c = 0; c < nch; ++c)
+                    if (!load(prow, c, p, INT_MAX)) break;
+                for (int k = 0; k < nm; ++k) {
+                    const int bb = b_first + k;
+                    if (!finished(bb)) continue;
+                    const int32_t* own = a.page_table + static_cast<int64_t>(bb) * a.max_pages;
+                    const int npages = (a.seq_lens[bb] + a.page_size - 1) / a.page_size;
+                    for (int c = a.pshare[bb]; c < n_chunks(bb); ++c)
+                        if (!load(own, c, p, npages)) break;
                 }
-                if (*failed) break;
             }
         }
     } else {
-        // ================= tile rows: warps 0-3 =================
-        const int r = tid;                                   // tile row = tensor-memory lane
-        const uint32_t tl = tmem + (static_cast<uint32_t>(32 * warp) << 16);
+        // ============ tile rows: warps 0-7, two threads per row ============
+        // Row r = tensor-memory lane (warp w reaches lanes 32 (w mod 4) ..);
+        // rows 0-63 hold the members' query heads of the pair's first KV
+        // head, rows 64-127 of the second, so a warp's rows share a head.
+        // The thread's half h2 picks half of the row's columns (S, P, O) and
+        // of its dims (Q).
+        // (a warp reaches the tensor-memory lanes 32 (w mod 4) .. of its
+        // index w in the CTA)
+        const int r = 32 * (warp & 3) + lane;
+        const int h2 = lwarp >> 2;
+        const int xi = h2 * kPfxRows + r;                    // this thread's exchange slot
+        const bool issuer = lwarp == 0 && lane == 0;         // issues the half's tensor-core work
+        const uint32_t tl = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
         const int G = a.group;
-        const int mrow = r / (2 * G);                        // member
-        const int hh = (r / G) & 1;                          // KV head of the pair
-        const int g = r - (r / G) * G;                       // query head in the group
+        const int hh = r >> 6;                               // KV head of the pair
+        const int rr = r & 63;
+        const int mrow = rr / G;                             // member
+        const int g = rr - mrow * G;                         // query head in the group
         constexpr uint32_t idesc = mma_idesc_f16(128);
         uint32_t it = 0, mma_phase = 0;
+        auto row_sync = [&]() { named_barrier_sync(1 + half, kPfxRowThreads); };
         auto mma_wait = [&]() {
             gemv_wait(mma_bar, mma_phase & 1, failed, a.status);
             ++mma_phase;
             tc_fence_after();
         };
-        for (int ti = blockIdx.x; ti < total; ti += gridDim.x) {
+        for (int ti = 2 * blockIdx.x + half; ti < total; ti += 2 * gridDim.x) {
             const int t = ti / IPR, p = ti - t * IPR;
             const int b_first = a.tiles[4 * t + 1], nm = a.tiles[4 * t + 2], nch = a.tiles[4 * t + 3];
-            const bool real = mrow < nm && r < (a.members_per_tile * 2 * G);
+            const bool real = mrow < nm && rr < a.members_per_tile * G;
             const int b = b_first + (real ? mrow : 0);
-            const int cb = real ? a.chunk_begin[b] : 0;
+            const int ps = real ? a.pshare[b] : 0;
+            const bool fin = real && finished(b);
             const bool dead = real && a.abort != nullptr && a.abort[b] != 0;
             const int hq = (2 * p + hh) * G + g;             // query head in the request
 
             // ---- Q row -> f16 scaled by 2^shift (exact), K-major swizzled tile ----
             float qs = 0.f;
             {
-                uint4 w[16];
+                uint4 w[8];
                 const uint4* src = reinterpret_cast<const uint4*>(
-                    a.q + (static_cast<int64_t>(b) * a.num_q_heads + hq) * kPfxD);
+                    a.q + (static_cast<int64_t>(b) * a.num_q_heads + hq) * kPfxD + 64 * h2);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) w[j] = real ? src[j] : make_uint4(0u, 0u, 0u, 0u);
+                for (int j = 0; j < 8; ++j) w[j] = real ? src[j] : make_uint4(0u, 0u, 0u, 0u);
                 float amax = 0.f;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
+                for (int j = 0; j < 8; ++j) {
                     const uint32_t x[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
@@ -384,6 +456,9 @@ prefix_attn_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_cons
                         amax = fmaxf(amax, fabsf(bf16_bits_to_f32(x[i] >> 16)));
                     }
                 }
+                s_xmax[xi] = amax;
+                row_sync();
+                amax = fmaxf(s_xmax[r], s_xmax[r + kPfxRows]);
                 // 2^shift brings amax into [128, 256) (see the split-K kernel)
                 int shift = 0;
                 if (amax > 0.f && isfinite(amax)) {
@@ -393,46 +468,62 @@ prefix_attn_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_cons
                 const float up = __uint_as_float(static_cast<uint32_t>(shift + 127) << 23);
                 qs = a.qk_scale * __uint_as_float(static_cast<uint32_t>(127 - shift) << 23);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
+                for (int j = 0; j < 8; ++j) {
                     const uint32_t x[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
                     uint32_t h[4];
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
                         h[i] = pack_f16x2(bf16_bits_to_f32(x[i] & 0xFFFFu) * up,
                                           bf16_bits_to_f32(x[i] >> 16) * up);
-                    // dims 8j .. 8j + 7: atom j / 8, chunk j mod 8
-                    sts128(base + kPfxQOff + (j >> 3) * kPfxAtom + atom_off(r, j & 7), h[0], h[1], h[2], h[3]);
+                    // dims 64 h2 + 8j .. + 7: atom h2, chunk j
+                    sts128(base + kPfxQOff + h2 * kPfxAtom + atom_off(r, j), h[0], h[1], h[2], h[3]);
                 }
             }
             fence_proxy_async_smem();
-            named_barrier_sync(1, 128);
+            row_sync();
 
             float m_run = kPfxNegInf, l_sum = 0.f, lr_sum = 0.f;
-            for (int c = 0; c < nch; ++c, ++it) {
-                // ---- K (row r = token r mod 64 of head r / 64) -> f16 token rows ----
+            // The tile's steps: shared chunks c < nch (member k = -1), then the
+            // own chunks of each member the tile finishes.  Per step, `act`
+            // says whether this row attends to the chunk, `valid` how many of
+            // its 64 tokens exist (the others are masked, their V rows zero).
+            int c = 0, cend = nch, k_mem = -1, len_k = 0;
+            for (int step = 0;; ++step) {
+                if (c >= cend) {
+                    do {
+                        ++k_mem;
+                    } while (k_mem < nm && !finished(b_first + k_mem));
+                    if (k_mem >= nm) break;
+                    c = a.pshare[b_first + k_mem];
+                    cend = n_chunks(b_first + k_mem);
+                    len_k = a.seq_lens[b_first + k_mem];
+                }
+                const bool act = real && !dead && (k_mem < 0 ? c < ps : mrow == k_mem);
+                const int valid = k_mem < 0 ? kChunkTokens : min(kChunkTokens, len_k - c * kChunkTokens);
+                // ---- K: row r = token r mod 64 of head r / 64; dims 64 h2 .. ----
                 gemv_wait(full_k, it & 1, failed, a.status);
                 {
                     const uint32_t src = base + kPfxRawKOff + r * 128;
+                    const uint32_t at = base + kPfxKVOff + h2 * kPfxAtom;
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const uint4 x = lds128(src + ((static_cast<uint32_t>(j) ^ (r & 7u)) << 4));
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const uint32_t j = static_cast<uint32_t>(4 * h2 + jj);   // raw dims 16j .. 16j + 15
+                        const uint4 x = lds128(src + ((j ^ (r & 7u)) << 4));
                         uint32_t f[8];
                         e4m3x4_to_f16x2x2(x.x, f[0], f[1]);
                         e4m3x4_to_f16x2x2(x.y, f[2], f[3]);
                         e4m3x4_to_f16x2x2(x.z, f[4], f[5]);
                         e4m3x4_to_f16x2x2(x.w, f[6], f[7]);
-                        // dims 16j .. 16j + 15: atom j / 4, chunks 2j, 2j + 1 (mod 8)
-                        const uint32_t at = base + kPfxKVOff + (j >> 2) * kPfxAtom;
-                        sts128(at + atom_off(r, (2 * j) & 7), f[0], f[1], f[2], f[3]);
-                        sts128(at + atom_off(r, (2 * j + 1) & 7), f[4], f[5], f[6], f[7]);
+                        sts128(at + atom_off(r, (2 * jj) & 7), f[0], f[1], f[2], f[3]);
+                        sts128(at + atom_off(r, (2 * jj + 1) & 7), f[4], f[5], f[6], f[7]);
                     }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(empty_k);
                 fence_proxy_async_smem();
                 tc_fence_before();
-                named_barrier_sync(1, 128);
-                if (tid == 0) {
+                row_sync();
+                if (issuer) {
                     tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
@@ -445,18 +536,22 @@ prefix_attn_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_cons
                 mma_wait();   // S is in tensor memory; the converted tile is free
 
                 // ---- V -> f16 V^T: row = dim, columns = tokens (head 0 | head 1) ----
+                // warp w: head w / 4, dims 32 (w mod 4) ..; lane: tokens 2 lane, 2 lane + 1
                 gemv_wait(full_v, it & 1, failed, a.status);
                 {
-                    const int hv = warp >> 1, dh = warp & 1;   // head, dims 64 dh .. 64 dh + 63
+                    const int hv = lwarp >> 2, dq = lwarp & 3;
                     const uint32_t t0 = static_cast<uint32_t>(hv * kChunkTokens + 2 * lane);
                     const uint32_t s0 = base + kPfxRawVOff + t0 * 128, s1 = s0 + 128;
                     const uint32_t at = base + kPfxKVOff + hv * kPfxAtom;
                     const uint32_t wofs = static_cast<uint32_t>(lane & 3) * 4;
+                    const bool z0 = 2 * lane >= valid, z1 = 2 * lane + 1 >= valid;
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const uint32_t j = static_cast<uint32_t>(4 * dh + jj);   // dims 16j .. 16j + 15
-                        const uint4 x0 = lds128(s0 + ((j ^ (t0 & 7u)) << 4));
-                        const uint4 x1 = lds128(s1 + ((j ^ ((t0 + 1) & 7u)) << 4));
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const uint32_t j = static_cast<uint32_t>(2 * dq + jj);   // dims 16j .. 16j + 15
+                        uint4 x0 = lds128(s0 + ((j ^ (t0 & 7u)) << 4));
+                        uint4 x1 = lds128(s1 + ((j ^ ((t0 + 1) & 7u)) << 4));
+                        if (z0) x0 = make_uint4(0u, 0u, 0u, 0u);
+                        if (z1) x1 = make_uint4(0u, 0u, 0u, 0u);
                         const uint32_t a0[4] = {x0.x, x0.y, x0.z, x0.w};
                         const uint32_t a1[4] = {x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
@@ -479,28 +574,29 @@ prefix_attn_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_cons
                 if (lane == 0) mbar_arrive(empty_v);
                 fence_proxy_async_smem();
 
-                // ---- online softmax of this row; P (f16) over S in tensor memory ----
-                // (tensor-memory loads and stores are warp-wide with one column
-                // address: every lane loads both heads' columns and keeps its own)
+                // ---- online softmax; P (f16) over S in tensor memory ----
+                // this thread: tokens 32 h2 .. 32 h2 + 31 of the row's head
                 {
-                    const bool active = real && !dead && c < cb;
-                    float sc[64];
+                    float sc[32];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint32_t v0[16], v1[16];
-                        tmem_ld16(tl + static_cast<uint32_t>(16 * q), v0);
-                        tmem_ld16(tl + static_cast<uint32_t>(64 + 16 * q), v1);
-                        tmem_wait_ld(v0);
-                        tmem_wait_ld(v1);
+                    for (int q = 0; q < 2; ++q) {
+                        uint32_t v[16];
+                        tmem_ld16(tl + static_cast<uint32_t>(hh * 64 + 32 * h2 + 16 * q), v);
+                        tmem_wait_ld(v);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) sc[16 * q + i] = __uint_as_float(hh ? v1[i] : v0[i]) * qs;
+                        for (int i = 0; i < 16; ++i)
+                            sc[16 * q + i] = (32 * h2 + 16 * q + i < valid) ? __uint_as_float(v[i]) * qs : kPfxNegInf;
                     }
-                    float mx = sc[0];
+                    float m4[4] = {sc[0], sc[1], sc[2], sc[3]};
 #pragma unroll
-                    for (int i = 1; i < 64; ++i) mx = fmaxf(mx, sc[i]);
+                    for (int i = 4; i < 32; ++i) m4[i & 3] = fmaxf(m4[i & 3], sc[i]);
+                    s_xmax[xi] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+                    row_sync();
+                    const float mx = fmaxf(s_xmax[r], s_xmax[r + kPfxRows]);
                     // the running maximum grows past the threshold: rescale l, lr and
-                    // this row of O (empty before the row's first chunk, which resets it)
-                    const bool need = active && mx > m_run + kPfxLog2RescaleThreshold;
+                    // this thread's half of the row of O (empty before the row's
+                    // first chunk, which resets it)
+                    const bool need = act && mx > m_run + kPfxLog2RescaleThreshold;
                     const float alpha = (need && m_run != kPfxNegInf) ? exp2f(m_run - mx) : 1.f;
                     if (need) {
                         l_sum *= alpha;
@@ -509,71 +605,84 @@ prefix_attn_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_cons
                     }
                     if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
+                        for (int q = 0; q < 4; ++q) {
                             uint32_t v[16];
-                            tmem_ld16(tl + kPfxOCol + 16 * q, v);
+                            const uint32_t col = tl + kPfxOCol + 64 * h2 + 16 * q;
+                            tmem_ld16(col, v);
                             tmem_wait_ld(v);
 #pragma unroll
                             for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-                            tmem_st16(tl + kPfxOCol + 16 * q, v);
+                            tmem_st16(col, v);
                         }
                     }
-                    uint32_t pw[32];
+                    uint32_t pw[16];
+                    float ls[2] = {0.f, 0.f}, lrs[2] = {0.f, 0.f};
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        pw[i] = 0u;
-                        if (active) {
-                            const float p0 = exp2f(sc[2 * i] - m_run), p1 = exp2f(sc[2 * i + 1] - m_run);
-                            l_sum += p0 + p1;
-                            pw[i] = pack_f16x2(p0, p1);
-                            float r0, r1;
-                            f16x2_to_f32x2(pw[i], r0, r1);
-                            lr_sum += r0 + r1;
-                        }
+                    for (int i = 0; i < 16; ++i) {
+                        const float p0 = exp2f(sc[2 * i] - m_run), p1 = exp2f(sc[2 * i + 1] - m_run);
+                        pw[i] = act ? pack_f16x2(p0, p1) : 0u;
+                        float r0, r1;
+                        f16x2_to_f32x2(pw[i], r0, r1);
+                        ls[i & 1] += act ? p0 + p1 : 0.f;
+                        lrs[i & 1] += r0 + r1;
                     }
-                    // P columns 0-31: tokens of head 0, 32-63: head 1; a row's
-                    // other head's columns are zero
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const bool mine = (q >> 1) == hh;
-                        uint32_t v[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) v[i] = mine ? pw[16 * (q & 1) + i] : 0u;
-                        tmem_st16(tl + static_cast<uint32_t>(16 * q), v);
-                    }
+                    l_sum += ls[0] + ls[1];
+                    lr_sum += lrs[0] + lrs[1];
+                    // P columns 0-31: tokens of head 0, 32-63: head 1; this
+                    // thread writes its 16 columns of its head and zeros in the
+                    // matching columns of the other head
+                    tmem_st16(tl + static_cast<uint32_t>(32 * hh + 16 * h2), pw);
+                    tmem_st16_zero(tl + static_cast<uint32_t>(32 * (1 - hh) + 16 * h2));
                     tmem_wait_st();
                 }
                 tc_fence_before();
-                named_barrier_sync(1, 128);
-                if (tid == 0) {
+                row_sync();
+                if (issuer) {
                     tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         const uint32_t off = (k >> 2) * kPfxAtom + 32 * (k & 3);
                         tc_mma_ts(tmem + kPfxOCol, tmem + 8 * k, sw128_kmajor_desc(base + kPfxKVOff + off),
-                                  idesc, (c > 0 || k > 0) ? 1u : 0u);
+                                  idesc, (step > 0 || k > 0) ? 1u : 0u);
                     }
                     tc_commit(mma_bar);
                 }
                 mma_wait();   // O updated; P, S and the converted tile are free
+                ++c;
+                ++it;
             }
 
-            // ---- this row's record: (m, l, lr, 0) and O (V scale applied) ----
-            // (every lane reads its O row: the loads are warp-wide)
+            // ---- this row: final output (a member the tile finishes) or the
+            // record (m, l, lr, 0) and O with the V scale applied ----
+            // (every lane reads its half of the O row: the loads are warp-wide)
             {
+                s_xl[xi] = l_sum;
+                s_xlr[xi] = lr_sum;
+                row_sync();
+                const float l_tot = s_xl[r] + s_xl[r + kPfxRows];
+                const float lr_tot = s_xlr[r] + s_xlr[r + kPfxRows];
                 const int64_t item = static_cast<int64_t>(b) * IPR + p;
                 const int IQ = 2 * G;
                 const int hi = hh * G + g;                    // head within the item
-                float4* o = reinterpret_cast<float4*>(a.pfx_o + (item * IQ + hi) * kPfxD);
-                float4* ml = reinterpret_cast<float4*>(a.pfx_ml + (item * IQ + hi) * 4);
-                const bool live = real && !dead && nch > 0;
+                const bool live = real && !dead;
+                const int64_t orow = static_cast<int64_t>(b) * a.num_q_heads + hq;
+                const float k_out = live ? a.v_scale / lr_tot : 0.f;
                 const float vs = live ? a.v_scale : 0.f;
+                float4* o = reinterpret_cast<float4*>(a.pfx_o + (item * IQ + hi) * kPfxD + 64 * h2);
+                uint32_t* dst = reinterpret_cast<uint32_t*>(a.out + orow * kPfxD + 64 * h2);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
+                for (int q = 0; q < 4; ++q) {
                     uint32_t v[16];
-                    tmem_ld16(tl + kPfxOCol + 16 * q, v);
+                    tmem_ld16(tl + kPfxOCol + 64 * h2 + 16 * q, v);
                     tmem_wait_ld(v);
-                    if (real) {
+                    if (fin) {
+                        uint32_t pk[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * k_out, __uint_as_float(v[2 * i + 1]) * k_out);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) dst[8 * q + i] = pk[i];
+                    } else if (real) {
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
                             o[4 * q + i] = make_float4(__uint_as_float(v[4 * i]) * vs, __uint_as_float(v[4 * i + 1]) * vs,
@@ -581,13 +690,20 @@ prefix_attn_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_cons
                                                        __uint_as_float(v[4 * i + 3]) * vs);
                     }
                 }
-                if (real)
-                    *ml = live ? make_float4(m_run, l_sum, lr_sum, 0.f) : make_float4(kPfxNegInf, -1.f, -1.f, 0.f);
+                if (h2 == 0 && real) {
+                    if (fin) {
+                        a.lse[orow] = live ? (m_run + log2f(l_tot)) * kPfxLn2 : kPfxNegInf;
+                    } else {
+                        float4* ml = reinterpret_cast<float4*>(a.pfx_ml + (item * IQ + hi) * 4);
+                        *ml = live ? make_float4(m_run, l_tot, lr_tot, 0.f) : make_float4(kPfxNegInf, -1.f, -1.f, 0.f);
+                    }
+                }
+                tc_fence_before();
+                row_sync();
             }
-            tc_fence_before();
             // the next tile rewrites Q, whose last reader (the final S product)
-            // has completed, and O, read above by every row before this barrier
-            named_barrier_sync(1, 128);
+            // has completed, O, read above by every row, and the exchange
+            // arrays, read above (the next writes follow another barrier)
         }
     }
 
@@ -596,7 +712,7 @@ prefix_attn_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_cons
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, kPfxTmemCols);
+        tmem_dealloc(*tmem_slot, kPfxTmemCols);
     }
 }
 
@@ -606,7 +722,26 @@ prefix_attn_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_cons
 size_t prefix_attn_smem_bytes() { return kPfxSmemBytes; }
 
 cudaError_t prefix_set_smem_attr() {
-    return cudaFuncSetAttribute(prefix_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPfxSmemBytes);
+    cudaError_t e =
+        cudaFuncSetAttribute(prefix_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPfxSmemBytes);
+    if (e != cudaSuccess) return e;
+    // all of the SM's on-chip memory as shared memory: two CTAs per SM
+    return cudaFuncSetAttribute(prefix_attn_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                cudaSharedmemCarveoutMaxShared);
+}
+
+cudaError_t prefix_occupancy(int* blocks_per_sm) {
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, prefix_attn_kernel, kPfxThreads,
+                                                         kPfxSmemBytes);
+}
+
+cudaError_t prefix_attributes(int* regs, int* local_bytes, int* max_threads) {
+    cudaFuncAttributes at;
+    cudaError_t e = cudaFuncGetAttributes(&at, prefix_attn_kernel);
+    *regs = at.numRegs;
+    *local_bytes = static_cast<int>(at.localSizeBytes);
+    *max_threads = at.maxThreadsPerBlock;
+    return e;
 }
 
 cudaError_t launch_prefix_plan(cudaStream_t stream, const PrefixArgs& args) {

@@ -22,6 +22,7 @@ pytestmark = pytest.mark.gpu
 
 CHUNK = 64
 MIN_CHUNKS = 4
+TAIL_CHUNKS = 2
 
 
 def expected_begin(lens, table, page_size, num_pages, max_pages, group):
@@ -32,7 +33,9 @@ def expected_begin(lens, table, page_size, num_pages, max_pages, group):
     a tie) and each member's chunks are those it shares with the reference;
     runs of 64 / group consecutive members (from the group's first request)
     form a tile if they have 2 members and a non-reference member with >= 4
-    chunks, and the reference, if in the run, takes the run's largest count."""
+    chunks, and the reference, if in the run, takes the run's largest count;
+    a tile member with at most 2 chunks after those is finished by the tile
+    (all of its chunks count)."""
     B = len(lens)
     max_tok = max_pages * page_size
 
@@ -80,7 +83,9 @@ def expected_begin(lens, table, page_size, num_pages, max_pages, group):
         mx = max([share[m] for m in members if m != refrow[b]], default=0)
         if len(members) >= 2 and mx >= MIN_CHUNKS:
             for m in members:
-                begin[m] = mx if m == refrow[b] else share[m]
+                ps = mx if m == refrow[b] else share[m]
+                n = full(m) + 1
+                begin[m] = n if n - ps <= TAIL_CHUNKS else ps
     return begin
 
 

@@ -16,7 +16,11 @@
 //
 // Design (tcgen05 / tensor memory):
 //  * Used for batches above 16 (int4_gemv_mma.cu covers smaller ones).
-//  * One CTA per 128 weight rows.  Warp 4 streams, with 2-D TMA loads, the
+//  * One half-CTA per 128 weight rows: a CTA holds two independent halves
+//    (warps 0-5 and 6-11), each with its own shared memory, barriers and
+//    tensor-memory columns (a CTA that allocates tensor memory is the only
+//    one on its SM).  Below, warp numbers are within a half.  Warp 4 streams,
+//    with 2-D TMA loads, the
 //    rows' codes (one contiguous 16 KiB tile per 256 columns) and the two
 //    groups' scales into one ring of shared-memory stages (lane 0), and the
 //    matching columns of x for the whole batch (zero-filled up to N = 32 or 64
@@ -60,7 +64,7 @@ struct GemvCfg {
     static constexpr int kWStageBytes = (kWBytes + kSBytes + 1023) / 1024 * 1024;
     static constexpr int kXBoxBytes = kN * 128;                     // kN rows x 64 columns (bf16)
     static constexpr int kXStageBytes = (kGemvKTile / 64) * kXBoxBytes;
-    // two CTAs per SM; the depths fill what is left of the shared memory
+    // two halves per CTA; the depths fill what is left of the shared memory
     static constexpr int kXStages = 2;
     static constexpr int kWStages = kN == 32 ? 4 : 2;
     static constexpr int kXOff = kWStages * kWStageBytes;
@@ -70,7 +74,13 @@ struct GemvCfg {
     // then the TMA warp and the MMA warp
     static constexpr int kSplit = 1;
     static constexpr int kConverters = 4 * kSplit;
-    static constexpr int kThreads = 32 * (kConverters + 2);
+    static constexpr int kHalfThreads = 32 * (kConverters + 2);
+    static constexpr int kHalfWarps = kHalfThreads / 32;
+    // Two independent halves per CTA, each with its own warps, shared memory
+    // and 256 tensor-memory columns, each working one row block: a CTA that
+    // allocates tensor memory gets an SM to itself, and two row blocks in
+    // flight let one half's expansion overlap the other's MMAs.
+    static constexpr int kThreads = 2 * kHalfThreads;
     static constexpr int kPartN = kN / kSplit;                     // accumulator columns per converter
     static constexpr int kPartUnits = 4 / kSplit;                  // 16-byte code units per group
     static constexpr int kGroupCols = kGemvGroup / 2;              // A columns of one group (bf16x2)
@@ -79,70 +89,87 @@ struct GemvCfg {
     static constexpr int kTmemCols = 256;
     static constexpr int kBarOff = kXOff + kXStages * kXStageBytes;
     static constexpr int kBars = 2 * kWStages + 2 * kXStages + 4;
-    static constexpr int kSmemBytes = kBarOff + kBars * 8 + 16 + 1024;   // + alignment slack
+    static constexpr int kHalfBytes = (kBarOff + kBars * 8 + 16 + 1023) / 1024 * 1024;
+    static constexpr int kSmemBytes = 2 * kHalfBytes + 1024;   // + alignment slack
     static_assert(kN == 32 || kN == 64, "batch columns");
     static_assert(kDCol + 2 * kN <= kTmemCols, "tensor memory");
 };
 
 template <int kN>
-__global__ void __launch_bounds__(GemvCfg<kN>::kThreads, 2)
+__global__ void __launch_bounds__(GemvCfg<kN>::kThreads, 1)
 int4_gemv_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                  const __grid_constant__ CUtensorMap tmap_s, const GemvArgs a) {
     using C = GemvCfg<kN>;
     constexpr int SW = C::kWStages;
     constexpr int SX = C::kXStages;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
+    uint8_t* smem0 = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int half = warp / C::kHalfWarps;
+    const int lwarp = warp - half * C::kHalfWarps;     // warp within the half
+    const int rb = 2 * static_cast<int>(blockIdx.x) + half;   // this half's row block
+    const bool active = rb < a.n / kGemvRows;
+    uint8_t* smem = smem0 + half * C::kHalfBytes;
     uint64_t* full_w = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
     uint64_t* empty_w = full_w + SW;
     uint64_t* full_x = empty_w + SW;
     uint64_t* empty_x = full_x + SX;
     uint64_t* a_ready = empty_x + SX;     // [2] A buffer written (the converter warps)
     uint64_t* d_ready = a_ready + 2;      // [2] group's MMAs complete (tcgen05.commit)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(d_ready + 2);
+    // (shared by both halves: in the first half's region)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem0 + C::kBarOff + C::kBars * 8);
     volatile int* failed = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-    const int tid = threadIdx.x;
-    const int warp = tid >> 5;
-    const int lane = tid & 31;
-    const int row0 = blockIdx.x * kGemvRows;
+    const int row0 = rb * kGemvRows;
     const int KT = a.k / kGemvKTile;
     const int NG = KT * (kGemvKTile / kGemvGroup);    // groups
 
     launch_dependents();
     if (tid == 0) {
-        for (int s = 0; s < SW; ++s) {
-            mbar_init(&full_w[s], 1);
-            mbar_init(&empty_w[s], C::kConverters);
-        }
-        for (int s = 0; s < SX; ++s) {
-            mbar_init(&full_x[s], 1);
-            mbar_init(&empty_x[s], 1);              // the MMA commit
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&a_ready[b], C::kConverters);
-            mbar_init(&d_ready[b], 1);
+        for (int hf = 0; hf < 2; ++hf) {
+            uint64_t* fw = reinterpret_cast<uint64_t*>(smem0 + hf * C::kHalfBytes + C::kBarOff);
+            uint64_t* ew = fw + SW;
+            uint64_t* fx = ew + SW;
+            uint64_t* ex = fx + SX;
+            uint64_t* ar = ex + SX;
+            uint64_t* dr = ar + 2;
+            for (int s = 0; s < SW; ++s) {
+                mbar_init(&fw[s], 1);
+                mbar_init(&ew[s], C::kConverters);
+            }
+            for (int s = 0; s < SX; ++s) {
+                mbar_init(&fx[s], 1);
+                mbar_init(&ex[s], 1);              // the MMA commit
+            }
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(&ar[b], C::kConverters);
+                mbar_init(&dr[b], 1);
+            }
         }
         *failed = 0;
         fence_barrier_init();
     }
     if (warp == 0) {
-        tmem_alloc(smem_addr(tmem_slot), C::kTmemCols);
+        tmem_alloc(smem_addr(tmem_slot), 2 * C::kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem = *tmem_slot + static_cast<uint32_t>(half * C::kTmemCols);   // this half's columns
 
-    if (warp == C::kConverters) {
+    if (!active) {
+        // (an odd number of row blocks: this half has none)
+    } else if (lwarp == C::kConverters) {
         // ================= TMA producers: lane 0 codes, lane 1 x =================
         if (lane == 0) {
             prefetch_tensormap(&tmap_w);
             prefetch_tensormap(&tmap_s);
             // the first code tiles into L2 while the preceding kernel finishes
-            const int tile0 = blockIdx.x * KT;     // first code tile of the row block
+            const int tile0 = rb * KT;     // first code tile of the row block
             for (int t = 0; t < SW && t < KT; ++t) tma_prefetch_l2_2d(&tmap_w, 0, (tile0 + t) * kGemvRows);
             grid_dependency_wait();
             for (int t = 0; t < KT; ++t) {
@@ -152,7 +179,7 @@ int4_gemv_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
                 mbar_arrive_expect_tx(&full_w[stage], C::kWBytes + C::kSBytes);
                 tma_load_2d(base, &tmap_w, 0, (tile0 + t) * kGemvRows, &full_w[stage]);
                 tma_load_2d(base + C::kWBytes, &tmap_s, 0,
-                            blockIdx.x * (a.k / kGemvGroup) + t * (kGemvKTile / kGemvGroup), &full_w[stage]);
+                            rb * (a.k / kGemvGroup) + t * (kGemvKTile / kGemvGroup), &full_w[stage]);
             }
         } else if (lane == 1) {
             prefetch_tensormap(&tmap_x);
@@ -167,7 +194,7 @@ int4_gemv_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
                     tma_load_2d(base + i * C::kXBoxBytes, &tmap_x, t * kGemvKTile + i * 64, 0, &full_x[stage]);
             }
         }
-    } else if (warp == C::kConverters + 1) {
+    } else if (lwarp == C::kConverters + 1) {
         // ================= MMA issuer =================
         if (lane == 0) {
             constexpr uint32_t idesc = mma_idesc_bf16(kN);
@@ -199,8 +226,10 @@ int4_gemv_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
         // (thread = row = tensor-memory lane; the part picks 1 / kSplit of a
         // group's columns for A and of the batch columns for the output)
         constexpr int PU = C::kPartUnits;
+        // (a warp reaches the tensor-memory lanes 32 (w mod 4) .. of its
+        // index w in the CTA)
         const int quarter = warp & 3;
-        const int part = warp >> 2;
+        const int part = lwarp >> 2;
         const int r = 32 * quarter + lane;                         // row in the tile
         const uint32_t tlane = tmem + (static_cast<uint32_t>(32 * quarter) << 16);
         float acc[C::kPartN];
@@ -289,7 +318,7 @@ int4_gemv_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, C::kTmemCols);
+        tmem_dealloc(*tmem_slot, 2 * C::kTmemCols);
     }
 }
 
@@ -311,7 +340,8 @@ cudaError_t gemv_set_smem_attr(int ncols) {
 cudaError_t launch_int4_gemv(int ncols, cudaStream_t stream, const CUtensorMap& tmap_w,
                              const CUtensorMap& tmap_x, const CUtensorMap& tmap_s, const GemvArgs& args) {
     PKV_GEMV_DISPATCH(ncols, {
-        PdlLaunch l(dim3(args.n / kGemvRows), dim3(GemvCfg<N>::kThreads), GemvCfg<N>::kSmemBytes, stream);
+        PdlLaunch l(dim3((args.n / kGemvRows + 1) / 2), dim3(GemvCfg<N>::kThreads), GemvCfg<N>::kSmemBytes,
+                    stream);
         return cudaLaunchKernelEx(&l.cfg, int4_gemv_kernel<N>, tmap_w, tmap_x, tmap_s, args);
     })
 }

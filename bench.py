@@ -775,6 +775,23 @@ def config_lines(args, rank, peak):
     t_a, _ = time_per_call(ga.replay, steps, args.warmup)
     torch.cuda.synchronize()
     assert pkv_status_ok(st) and not bool(st.abort.any())
+    # the shared-prefix call on the same batch (groups found on the device)
+    import paged_fp8_kv_attn_b200 as pkv
+    B, Hq, D = wl.q.shape
+    wsp = pkv.alloc_prefix_workspace(B, Hq, wl.num_kv_heads, D)
+    begin = torch.zeros(B, dtype=torch.int32, device="cuda")
+
+    def attend_prefix():
+        pkv.paged_decode_attn_fp8_prefix(st.q, st.k_cache, st.v_cache, wl.k_scale, wl.v_scale,
+                                         st.page_table, st.seq_lens, wl.sm_scale, st.out, st.lse,
+                                         wsp, abort=st.abort, chunk_begin_out=begin)
+
+    gp = _graph(attend_prefix)
+    t_p, _ = time_per_call(gp.replay, steps, args.warmup)
+    torch.cuda.synchronize()
+    assert pkv.workspace_status(wsp) == 0
+    n_chunks = np.asarray([(int(L) + 63) // 64 for L in wl.seq_lens])
+    cb = begin.cpu().numpy()
     lens = wl.seq_lens.astype(np.int64)
     out["ragged_prefix"] = {
         "batch": wl.batch, "logical_tokens": int(lens.sum()), "unique_tokens": u_tok,
@@ -784,8 +801,13 @@ def config_lines(args, rank, peak):
         "step_us": round(t_step, 2), "tokens_per_s": round(wl.batch / (t_step * 1e-6), 1),
         "attn_us": round(t_a, 2),
         "attn_logical_gbs": round(logical / (t_a * 1e-6) / 1e9, 1),
-        "attn_unique": _kv_row(unique, t_a, peak)}
-    del gf, ga, st, wl
+        "attn_unique": _kv_row(unique, t_a, peak),
+        "shared_prefix_call": {
+            "attn_us": round(t_p, 2), "attn_unique": _kv_row(unique, t_p, peak),
+            "requests_in_tiles": int((cb > 0).sum()),
+            "requests_finished_in_tiles": int(((cb > 0) & (cb == n_chunks)).sum()),
+            "chunks_in_tiles": int(cb.sum())}}
+    del gf, ga, gp, st, wl, wsp
     torch.cuda.empty_cache()
     return out
 

@@ -999,10 +999,11 @@ def main():
     ap.add_argument("--no-int4", action="store_true")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the capacity, integrity-stress and ragged + prefix workloads")
-    ap.add_argument("--kernel-only", choices=["fp8", "bf16", "int4"], default=None,
+    ap.add_argument("--kernel-only", choices=["fp8", "bf16", "int4", "prefix"], default=None,
                     help="profiling target: run only the decode step (fp8/bf16) on a --batch "
-                         "request concurrency-sweep batch, or only the INT4 GEMV at --batch; "
-                         "warmup + steps times; prints nothing")
+                         "request concurrency-sweep batch, only the INT4 GEMV at --batch, or "
+                         "only the shared-prefix attention call on a --batch request ragged "
+                         "prefix-reuse batch; warmup + steps times; prints nothing")
     ap.add_argument("--batch", type=int, default=16)
     args = ap.parse_args()
     if args.warmup < 3:
@@ -1027,6 +1028,22 @@ def main():
             pkv.int4_dequant_gemv(case.x, case.w_tiles, case.scales, y, case.group, status=status)
         torch.cuda.synchronize()
         assert int(status.item()) == 0
+        return
+    if args.kernel_only == "prefix":
+        import paged_fp8_kv_attn_b200 as pkv
+        import workloads
+        wl = workloads.ragged_prefix(device="cuda", batch=args.batch)
+        st = Step(wl, "fp8")
+        del wl.k_pool, wl.v_pool     # (the FP8 caches are built)
+        torch.cuda.empty_cache()
+        B, Hq, D = wl.q.shape
+        wsp = pkv.alloc_prefix_workspace(B, Hq, wl.num_kv_heads, D)
+        for _ in range(args.warmup + args.steps):
+            pkv.paged_decode_attn_fp8_prefix(st.q, st.k_cache, st.v_cache, wl.k_scale, wl.v_scale,
+                                             st.page_table, st.seq_lens, wl.sm_scale, st.out,
+                                             st.lse, wsp, abort=st.abort)
+        torch.cuda.synchronize()
+        assert pkv.workspace_status(wsp) == 0
         return
     if args.kernel_only:
         import workloads

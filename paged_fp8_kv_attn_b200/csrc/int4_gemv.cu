@@ -19,16 +19,16 @@
 //  * One half-CTA per 128 weight rows: a CTA holds two independent halves
 //    (warps 0-5 and 6-11), each with its own shared memory, barriers and
 //    tensor-memory columns (a CTA that allocates tensor memory is the only
-//    one on its SM).  Below, warp numbers are within a half.  Warp 4 streams,
-//    with 2-D TMA loads, the
-//    rows' codes (one contiguous 16 KiB tile per 256 columns) and the two
+//    one on its SM).  Below, warp numbers are within a half.  Warp 4
+//    streams, with 2-D TMA loads, the rows' codes (one contiguous 16 KiB
+//    tile per 256 columns) and the two
 //    groups' scales into one ring of shared-memory stages (lane 0), and the
 //    matching columns of x for the whole batch (zero-filled up to N = 32 or 64
 //    rows) into a second ring (lane 1); the first code tiles are
 //    prefetched into L2 before the grid-dependency wait.
-//  * Warps 0-3 convert: warp w owns rows 32 w .. 32 w + 31 (thread = row =
-//    tensor-memory lane).  Per 128-column group a thread expands its row's
-//    128 codes to bf16 in
+//  * Warps 0-3 convert: each owns the 32 rows of its tensor-memory lane
+//    quarter (the warp's index in the CTA mod 4; thread = row = lane).  Per
+//    128-column group a thread expands its row's 128 codes to bf16 in
 //    registers (per pair of columns: one shift, one LOP3 that puts the two
 //    offset-binary nibbles into the mantissas of 128.0, one bf16x2 FMA that
 //    subtracts 136) and writes them to a tensor-memory A buffer with

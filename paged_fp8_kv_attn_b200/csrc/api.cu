@@ -271,12 +271,13 @@ pkv_status plan_attention(bool fp8, int32_t batch, int32_t num_kv_heads, int32_t
     // when the batch has no more items than one wave of CTAs (measured on
     // B200: faster than split-K plus merge at every such size of the
     // concurrency sweep; larger batches, which can be ragged, keep the
-    // balanced split-K partition), or requested with num_ctas = -C.  When
-    // even clusters of the largest size
-    // would leave SMs idle with two KV heads per item (a handful of
-    // requests), the library's choice takes one KV head per item, which
-    // doubles the CTAs (cluster mode needs the workspace for its status word
-    // only, so the workspace size does not depend on this).
+    // balanced split-K partition), or requested with num_ctas = -C.  With at
+    // most a quarter as many two-head items as SMs (up to 9 requests at 8 KV
+    // heads), the library's choice takes one KV head per item, which doubles
+    // the items and the CTAs that share them (measured on B200 at 8,192
+    // tokens: 13% faster at 4 requests, unchanged at 1 and 8, 4-5% slower at
+    // 16 and 32; cluster mode needs the workspace for its status word only,
+    // so the workspace size does not depend on this).
     int64_t items = static_cast<int64_t>(batch) * (num_kv_heads / kv_per_item);
     int cluster = 0, nclusters = 0;
     if (allow_cluster && (num_ctas < 0 || (num_ctas == 0 && items <= grid))) {
@@ -284,7 +285,7 @@ pkv_status plan_attention(bool fp8, int32_t batch, int32_t num_kv_heads, int32_t
             const DeviceInfo* info = nullptr;
             st = device_info(&info);
             if (st != PKV_OK) return st;
-            if (items * pkv::kMaxCluster <= info->sms) {
+            if (items * 4 <= info->sms) {
                 kv_per_item = 1;
                 items *= 2;
             }

@@ -560,6 +560,12 @@ def gpu_arm(args, rank, world):
 
     e2e_run(max(args.warmup, 2))
     torch.cuda.synchronize()
+    # the same ~1 s of sustained load as before the device-timed steps, so
+    # that both figures are taken at the clocks that load settles at
+    soak_until = time.perf_counter() + 1.0
+    while time.perf_counter() < soak_until:
+        e2e_run(50)
+        torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     e0.record()
@@ -653,7 +659,8 @@ def gpu_arm(args, rank, world):
                 "api": "python binding -> C ABI, eager calls; one pinned H2D copy of the "
                        "packed inputs and one D2H copy of the packed results per step, "
                        "double-buffered on two copy streams (step i+1 in and step i-1 out "
-                       "while step i computes)"},
+                       "while step i computes); timed after ~1 s of the same load, as the "
+                       "device-timed steps are"},
         "gpu_launches": (1 + attn_launches) * args.steps,   # check+append, then attention
         "clocks": clk,
         "int4_gemv": int4,

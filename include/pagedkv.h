@@ -327,13 +327,16 @@ PKV_API pkv_status paged_decode_attn_fp8(const uint16_t* q, const uint8_t* k_cac
  * token (the first on a tie); each member shares with the group the leading
  * chunks it has in common with the reference row (same rule).  Runs of up to
  * 64 / G consecutive members from the group's first request
- * (G = num_q_heads / num_kv_heads) form tensor-core tiles of two KV heads,
- * if a run has 2 members and one of them other than the reference shares at
- * least 4 chunks; the tile covers the run's largest share, which the
- * reference, if in the run, takes as its own.  Those chunks are attended for
- * all members of the tile together, each member's remaining chunks by the
- * split-K kernel, and a merge kernel combines the two.  Supported: head_dim 128, an even num_kv_heads and G <= 8;
- * other shapes run paged_decode_attn_fp8 unchanged (nothing shared).
+ * (G = num_q_heads / num_kv_heads) form tensor-core tiles of two KV heads
+ * when a run has at least 2 members and one of them other than the
+ * reference shares at least 4 chunks; the tile covers the run's largest
+ * share, which the reference, if in the run, takes as its own.  Those
+ * chunks are attended for all members of the tile together; a member with
+ * at most 2 chunks after them is finished in the tile too, the others'
+ * remaining chunks go through the split-K kernel, and a merge kernel
+ * combines the two.  Supported: head_dim 128, an even num_kv_heads and
+ * G <= 8; other shapes run paged_decode_attn_fp8 unchanged (nothing
+ * shared).
  *
  * workspace: at least paged_decode_attn_fp8_prefix_workspace_size(...)
  * bytes (the split-K workspace plus one partial record per (request, pair of
@@ -342,7 +345,8 @@ PKV_API pkv_status paged_decode_attn_fp8(const uint16_t* q, const uint8_t* k_cac
  * library's split-K grid) or N > 0 (split-K over N CTAs); cluster mode is
  * not used (PKV_ERR_INVALID_ARG for num_ctas < 0).  chunk_begin_out: NULL,
  * or a device [batch] int32 array that receives, per request, the number of
- * leading chunks the shared pass covered (0 = none), in stream order.
+ * leading chunks attended in its tile (0 = none; all of its chunks when the
+ * tile finished it), in stream order.
  * Kernels: four plan kernels, the shared-prefix kernel, the split-K partial
  * kernel and the merge kernel, all chained with programmatic dependent
  * launch; none of them reads the cache, the page table or abort before the

@@ -360,8 +360,8 @@ def paged_decode_attn_fp8_prefix(q, k_cache, v_cache, k_scale, v_scale, page_tab
                                  chunk_begin_out=None, stream=None):
     """paged_decode_attn_fp8 for batches whose consecutive requests share leading
     pages: the shared chunks are attended once per group.  chunk_begin_out
-    (optional int32 [batch] CUDA tensor) receives the chunks the shared pass
-    covered per request."""
+    (optional int32 [batch] CUDA tensor) receives, per request, the leading
+    chunks attended in its tile (all of them when the tile finished it)."""
     _need(k_cache, torch.uint8, 4, "k_cache")
     _need(v_cache, torch.uint8, 4, "v_cache")
     B, Hq, D, NP, Hkv, P = _attn_common(q, k_cache, page_table, seq_lens, out, lse, workspace,

@@ -28,8 +28,9 @@
 //    streams the raw FP8 K and V rows of both heads (TMA, 128-byte swizzle);
 //    warps 0-3 (thread = row = tensor-memory lane) convert K to f16 token
 //    rows (exact), thread 0 issues S = Q K^T (M = 128, N = 128 tokens of both
-//    heads, K = 128 dims) into tensor memory; while it runs the warps convert
-//    V to f16 V^T; each thread then reads its row of S (its own head's 64
+//    heads, K = 128 dims) into tensor memory; then the warps convert V to
+//    f16 token rows (the MN-major operand of the product, so no transpose);
+//    each thread then reads its row of S (its own head's 64
 //    columns), updates its online softmax and writes P (f16, the other head's
 //    columns zero: the product is block-diagonal) back into tensor memory
 //    over S; thread 0 issues O += P V (A = P from tensor memory, K = 128
@@ -52,11 +53,11 @@ constexpr float kPfxLog2RescaleThreshold = 8.0f;
 constexpr float kPfxNegInf = -__builtin_huge_valf();
 constexpr float kPfxLn2 = 0.6931471805599453f;
 constexpr int kPfxD = 128;
-// shared memory: Q tile, converted K (token rows) or V^T (dim rows) tile,
+// shared memory: Q tile, converted K or V tile (token rows of 64-dim blocks),
 // raw FP8 K and V of one chunk of both heads, barriers
 constexpr int kPfxAtom = kPfxRows * 128;                 // 128 rows x 128 bytes: 64 f16 columns
 constexpr int kPfxQOff = 0;                               // 2 atoms (dims 0-63, 64-127)
-constexpr int kPfxKVOff = kPfxQOff + 2 * kPfxAtom;        // 2 atoms (K: dims; V^T: tokens of each head)
+constexpr int kPfxKVOff = kPfxQOff + 2 * kPfxAtom;        // 2 atoms (dims 0-63, 64-127)
 constexpr int kPfxRawBytes = 2 * kChunkTokens * kPfxD;   // one FP8 operand of both heads: 16 KiB
 constexpr int kPfxRawKOff = kPfxKVOff + 2 * kPfxAtom;
 constexpr int kPfxRawVOff = kPfxRawKOff + kPfxRawBytes;
@@ -271,8 +272,13 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, ui
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                  : "memory");
 }
-__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
-    asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+// 2^x with the hardware approximation (relative error near 2^-22; results
+// below the smallest normal float flush to zero): the softmax weights, which
+// are rounded to f16 for the product anyway.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 // Boxes of chunk c that lie in the request's first `npages` pages (all of
@@ -421,6 +427,7 @@ prefix_attn_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_cons
         const int mrow = rr / G;                             // member
         const int g = rr - mrow * G;                         // query head in the group
         constexpr uint32_t idesc = mma_idesc_f16(128);
+        constexpr uint32_t idesc_pv = mma_idesc_f16_bmn(128);   // V: N = dims contiguous
         uint32_t it = 0, mma_phase = 0;
         auto row_sync = [&]() { named_barrier_sync(1 + half, kPfxRowThreads); };
         auto mma_wait = [&]() {
@@ -535,39 +542,26 @@ prefix_attn_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_cons
                 }
                 mma_wait();   // S is in tensor memory; the converted tile is free
 
-                // ---- V -> f16 V^T: row = dim, columns = tokens (head 0 | head 1) ----
-                // warp w: head w / 4, dims 32 (w mod 4) ..; lane: tokens 2 lane, 2 lane + 1
+                // ---- V: row r = token r mod 64 of head r / 64; dims 64 h2 .. ----
+                // (token rows of 64-dim blocks, as the MN-major operand of
+                // O += P V: no transpose; the rows of missing tokens are zero)
                 gemv_wait(full_v, it & 1, failed, a.status);
                 {
-                    const int hv = lwarp >> 2, dq = lwarp & 3;
-                    const uint32_t t0 = static_cast<uint32_t>(hv * kChunkTokens + 2 * lane);
-                    const uint32_t s0 = base + kPfxRawVOff + t0 * 128, s1 = s0 + 128;
-                    const uint32_t at = base + kPfxKVOff + hv * kPfxAtom;
-                    const uint32_t wofs = static_cast<uint32_t>(lane & 3) * 4;
-                    const bool z0 = 2 * lane >= valid, z1 = 2 * lane + 1 >= valid;
+                    const bool zero = rr >= valid;
+                    const uint32_t src = base + kPfxRawVOff + r * 128;
+                    const uint32_t at = base + kPfxKVOff + h2 * kPfxAtom;
 #pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) {
-                        const uint32_t j = static_cast<uint32_t>(2 * dq + jj);   // dims 16j .. 16j + 15
-                        uint4 x0 = lds128(s0 + ((j ^ (t0 & 7u)) << 4));
-                        uint4 x1 = lds128(s1 + ((j ^ ((t0 + 1) & 7u)) << 4));
-                        if (z0) x0 = make_uint4(0u, 0u, 0u, 0u);
-                        if (z1) x1 = make_uint4(0u, 0u, 0u, 0u);
-                        const uint32_t a0[4] = {x0.x, x0.y, x0.z, x0.w};
-                        const uint32_t a1[4] = {x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            uint32_t v0, v1, v2, v3;   // dims 4i .. 4i + 3 of the unit: (token t0, t0 + 1)
-                            e4m3x4_to_f16x2x2(prmt(a0[i], a1[i], 0x5140u), v0, v1);
-                            e4m3x4_to_f16x2x2(prmt(a0[i], a1[i], 0x7362u), v2, v3);
-                            const uint32_t d = 16 * j + 4 * i;
-                            const uint32_t vs[4] = {v0, v1, v2, v3};
-#pragma unroll
-                            for (int k = 0; k < 4; ++k) {
-                                const uint32_t dd = d + k;
-                                sts32(at + dd * 128 + (((static_cast<uint32_t>(lane) >> 2) ^ (dd & 7u)) << 4) + wofs,
-                                      vs[k]);
-                            }
-                        }
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const uint32_t j = static_cast<uint32_t>(4 * h2 + jj);   // raw dims 16 j .. 16 j + 15
+                        uint4 x = lds128(src + ((j ^ (r & 7u)) << 4));
+                        if (zero) x = make_uint4(0u, 0u, 0u, 0u);
+                        uint32_t f[8];
+                        e4m3x4_to_f16x2x2(x.x, f[0], f[1]);
+                        e4m3x4_to_f16x2x2(x.y, f[2], f[3]);
+                        e4m3x4_to_f16x2x2(x.z, f[4], f[5]);
+                        e4m3x4_to_f16x2x2(x.w, f[6], f[7]);
+                        sts128(at + atom_off(r, (2 * jj) & 7), f[0], f[1], f[2], f[3]);
+                        sts128(at + atom_off(r, (2 * jj + 1) & 7), f[4], f[5], f[6], f[7]);
                     }
                 }
                 __syncwarp();
@@ -615,19 +609,22 @@ prefix_attn_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_cons
                             tmem_st16(col, v);
                         }
                     }
+                    // lr sums the weights as rounded to f16 for the product:
+                    // their f16 exponent and mantissa fields, moved under the
+                    // binary32 ones, read as the weight times 2^-112 exactly
+                    // (subnormals included), so the sum is scaled once
                     uint32_t pw[16];
                     float ls[2] = {0.f, 0.f}, lrs[2] = {0.f, 0.f};
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const float p0 = exp2f(sc[2 * i] - m_run), p1 = exp2f(sc[2 * i + 1] - m_run);
+                        const float p0 = ex2_approx(sc[2 * i] - m_run), p1 = ex2_approx(sc[2 * i + 1] - m_run);
                         pw[i] = act ? pack_f16x2(p0, p1) : 0u;
-                        float r0, r1;
-                        f16x2_to_f32x2(pw[i], r0, r1);
                         ls[i & 1] += act ? p0 + p1 : 0.f;
-                        lrs[i & 1] += r0 + r1;
+                        lrs[i & 1] += __uint_as_float((pw[i] << 13) & 0x0FFFE000u) +
+                                      __uint_as_float((pw[i] >> 3) & 0x0FFFE000u);
                     }
                     l_sum += ls[0] + ls[1];
-                    lr_sum += lrs[0] + lrs[1];
+                    lr_sum += (lrs[0] + lrs[1]) * 0x1p112f;
                     // P columns 0-31: tokens of head 0, 32-63: head 1; this
                     // thread writes its 16 columns of its head and zeros in the
                     // matching columns of the other head
@@ -640,10 +637,10 @@ prefix_attn_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_cons
                 if (issuer) {
                     tc_fence_after();
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const uint32_t off = (k >> 2) * kPfxAtom + 32 * (k & 3);
-                        tc_mma_ts(tmem + kPfxOCol, tmem + 8 * k, sw128_kmajor_desc(base + kPfxKVOff + off),
-                                  idesc, (step > 0 || k > 0) ? 1u : 0u);
+                    for (int k = 0; k < 8; ++k) {   // tokens 16 k .. 16 k + 15: two 8-row atoms
+                        tc_mma_ts(tmem + kPfxOCol, tmem + 8 * k,
+                                  sw128_mnmajor_desc(base + kPfxKVOff + 2048 * k, kPfxAtom), idesc_pv,
+                                  (step > 0 || k > 0) ? 1u : 0u);
                     }
                     tc_commit(mma_bar);
                 }

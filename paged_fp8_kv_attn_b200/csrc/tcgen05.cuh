@@ -104,6 +104,17 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_byte_addr) {
            | (static_cast<uint64_t>(2) << 61);                       // 128-byte swizzle
 }
 
+// Shared-memory descriptor of an MN-major operand tile with the 128-byte
+// swizzle: K rows of 128 bytes (64 16-bit MN elements), 8-row atoms 1024
+// bytes apart along K, and the next 64 MN elements `mn_stride` bytes on.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_byte_addr, uint32_t mn_stride) {
+    return static_cast<uint64_t>((smem_byte_addr >> 4) & 0x3FFFu)   // start address / 16
+           | (static_cast<uint64_t>((mn_stride >> 4) & 0x3FFFu) << 16)   // leading offset: next 64 MN
+           | (static_cast<uint64_t>(1024 >> 4) << 32)                // stride offset: next 8 K rows
+           | (static_cast<uint64_t>(1) << 46)                        // descriptor version
+           | (static_cast<uint64_t>(2) << 61);                       // 128-byte swizzle
+}
+
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
 // K-major, M = 128, N = n.
 __host__ __device__ constexpr uint32_t mma_idesc_bf16(int n) {
@@ -116,5 +127,7 @@ __host__ __device__ constexpr uint32_t mma_idesc_bf16(int n) {
 __host__ __device__ constexpr uint32_t mma_idesc_f16(int n) {
     return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
 }
+// The same with B MN-major (its N elements contiguous in each K row).
+__host__ __device__ constexpr uint32_t mma_idesc_f16_bmn(int n) { return mma_idesc_f16(n) | (1u << 16); }
 
 }  // namespace pkv

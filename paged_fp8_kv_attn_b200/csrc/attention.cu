@@ -980,7 +980,7 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const float ref = (m[nb][i & 1] == kNegInf) ? 0.f : m[nb][i & 1];
-                    p[nb][i] = exp2f(p[nb][i] - ref);
+                    p[nb][i] = ex2_approx(p[nb][i] - ref);
                 }
                 l[nb][0] += p[nb][0] + p[nb][2];
                 l[nb][1] += p[nb][1] + p[nb][3];
@@ -989,16 +989,18 @@ attn_partial_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 if constexpr (kFp8) {
                     h01 = pack_f16x2(p[nb][0], p[nb][1]);
                     h23 = pack_f16x2(p[nb][2], p[nb][3]);
-                    f16x2_to_f32x2(h01, r0, r1);
-                    f16x2_to_f32x2(h23, r2, r3);
+                    f16x2_nonneg_scaled(h01, r0, r1);   // (x 2^-112)
+                    f16x2_nonneg_scaled(h23, r2, r3);
+                    lr[nb][0] = fmaf(r0 + r2, 0x1p112f, lr[nb][0]);
+                    lr[nb][1] = fmaf(r1 + r3, 0x1p112f, lr[nb][1]);
                 } else {
                     h01 = pack_bf16x2(p[nb][0], p[nb][1]);
                     h23 = pack_bf16x2(p[nb][2], p[nb][3]);
                     bf16x2_to_f32x2(h01, r0, r1);
                     bf16x2_to_f32x2(h23, r2, r3);
+                    lr[nb][0] += r0 + r2;
+                    lr[nb][1] += r1 + r3;
                 }
-                lr[nb][0] += r0 + r2;
-                lr[nb][1] += r1 + r3;
                 pb[nb][0] = movmatrix_trans(h01);
                 pb[nb][1] = movmatrix_trans(h23);
             }

@@ -223,6 +223,22 @@ __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float hi, float lo) {
         : "f"(hi), "f"(lo));
     return r;
 }
+// 2^x with the hardware approximation (relative error near 2^-22; results
+// below the smallest normal float flush to zero): softmax weights, which
+// are rounded to f16 or bf16 for the PV product anyway.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// The f16 pair x, both halves >= 0 (sign bits clear), as binary32 values
+// times 2^-112, exactly (subnormals included): the f16 exponent and mantissa
+// fields moved under the binary32 ones.  Summing these and scaling the sum by
+// 2^112 once replaces two conversions per pair.
+__device__ __forceinline__ void f16x2_nonneg_scaled(uint32_t x, float& lo, float& hi) {
+    lo = __uint_as_float((x << 13) & 0x0FFFE000u);
+    hi = __uint_as_float((x >> 3) & 0x0FFFE000u);
+}
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

@@ -272,14 +272,6 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, ui
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                  : "memory");
 }
-// 2^x with the hardware approximation (relative error near 2^-22; results
-// below the smallest normal float flush to zero): the softmax weights, which
-// are rounded to f16 for the product anyway.
-__device__ __forceinline__ float ex2_approx(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
 
 // Boxes of chunk c that lie in the request's first `npages` pages (all of
 // them except in the last chunk of a request with pages under 64 tokens).
@@ -609,10 +601,8 @@ prefix_attn_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_cons
                             tmem_st16(col, v);
                         }
                     }
-                    // lr sums the weights as rounded to f16 for the product:
-                    // their f16 exponent and mantissa fields, moved under the
-                    // binary32 ones, read as the weight times 2^-112 exactly
-                    // (subnormals included), so the sum is scaled once
+                    // lr sums the weights as rounded to f16 for the product
+                    // (read as binary32 times 2^-112, the sum scaled once)
                     uint32_t pw[16];
                     float ls[2] = {0.f, 0.f}, lrs[2] = {0.f, 0.f};
 #pragma unroll
@@ -620,8 +610,9 @@ prefix_attn_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_cons
                         const float p0 = ex2_approx(sc[2 * i] - m_run), p1 = ex2_approx(sc[2 * i + 1] - m_run);
                         pw[i] = act ? pack_f16x2(p0, p1) : 0u;
                         ls[i & 1] += act ? p0 + p1 : 0.f;
-                        lrs[i & 1] += __uint_as_float((pw[i] << 13) & 0x0FFFE000u) +
-                                      __uint_as_float((pw[i] >> 3) & 0x0FFFE000u);
+                        float r0, r1;
+                        f16x2_nonneg_scaled(pw[i], r0, r1);
+                        lrs[i & 1] += r0 + r1;
                     }
                     l_sum += ls[0] + ls[1];
                     lr_sum += (lrs[0] + lrs[1]) * 0x1p112f;

@@ -32,8 +32,9 @@ def expected_begin(lens, table, page_size, num_pages, max_pages, group):
     is its member with the most chunks before its newest token (the first on
     a tie) and each member's chunks are those it shares with the reference;
     runs of 64 / group consecutive members (from the group's first request)
-    form a tile if they have 2 members and a non-reference member with >= 4
-    chunks, and the reference, if in the run, takes the run's largest count;
+    form a tile if they have at least 2 members and a non-reference member
+    with >= 4 chunks, and the reference, if in the run, takes the run's
+    largest count;
     a tile member with at most 2 chunks after those is finished by the tile
     (all of its chunks count)."""
     B = len(lens)

@@ -40,9 +40,9 @@
  *  - Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).
  *    Every call only enqueues work: it returns before the GPU runs it, and
  *    never synchronises.
- *  - Launch chaining: every kernel except the cluster-mode attention kernel
- *    is launched with programmatic dependent launch, so it may be scheduled
- *    while the previous kernel on the stream is still running.  Each kernel
+ *  - Launch chaining: every kernel is launched with programmatic dependent
+ *    launch, so it may be scheduled while the previous kernel on the stream
+ *    is still running.  Each kernel
  *    waits for that kernel to finish before it touches memory that kernel
  *    may write, with one exception documented at paged_decode_attn_fp8:
  *    before waiting, attention reads q, seq_lens and page_table and

@@ -63,6 +63,8 @@ pkv_status device_info(const DeviceInfo** out) {
     if (!info.ready) {
         e = cudaDeviceGetAttribute(&info.sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+        e = pkv::step_kernels_set_carveout();
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         for (int f = 0; f < 2; ++f)
             for (int d = 0; d < 2; ++d)
                 for (int gp = 0; gp < 2; ++gp)
@@ -643,6 +645,11 @@ pkv_status kv_tag_check(const uint32_t* page_tags, int32_t num_pages, const int3
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(num_aborted)");
     }
     if (batch == 0) return PKV_OK;
+    {
+        const DeviceInfo* info = nullptr;   // per-device set-up (kernel attributes)
+        const pkv_status ds = device_info(&info);
+        if (ds != PKV_OK) return ds;
+    }
     cudaError_t e = pkv::launch_tag_check(page_tags, num_pages, page_table, expected_tags,
                                           max_pages, seq_lens, batch, page_size, abort_out,
                                           num_aborted, as_stream(stream));
@@ -667,6 +674,11 @@ static pkv_status append_impl(bool fp8, const uint16_t* k_new, const uint16_t* v
     if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) ||
         !aligned(v_cache, 16))
         return fail(PKV_ERR_INVALID_ARG, "k_new, v_new and the caches must be 16-byte aligned");
+    {
+        const DeviceInfo* info = nullptr;   // per-device set-up (kernel attributes)
+        const pkv_status ds = device_info(&info);
+        if (ds != PKV_OK) return ds;
+    }
     cudaError_t e = pkv::launch_append(fp8, k_new, v_new, page_table, max_pages, seq_lens, batch,
                                        num_kv_heads, head_dim, page_size, k_scale, v_scale,
                                        k_cache, v_cache, num_pages, abort, as_stream(stream));
@@ -717,6 +729,11 @@ static pkv_status check_append_impl(bool fp8, const uint32_t* page_tags, int32_t
     if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) ||
         !aligned(v_cache, 16))
         return fail(PKV_ERR_INVALID_ARG, "k_new, v_new and the caches must be 16-byte aligned");
+    {
+        const DeviceInfo* info = nullptr;   // per-device set-up (kernel attributes)
+        const pkv_status ds = device_info(&info);
+        if (ds != PKV_OK) return ds;
+    }
     cudaError_t e = pkv::launch_check_append(fp8, page_tags, num_pages, page_table, expected_tags,
                                              max_pages, seq_lens, batch, page_size, k_new, v_new,
                                              num_kv_heads, head_dim, k_scale, v_scale, k_cache,

@@ -1493,18 +1493,7 @@ static cudaError_t launch_variant(int grid, cudaStream_t stream, const CUtensorM
                                   const CUtensorMap& tv, const AttnArgs& args) {
     using C = AttnCfg<kFp8, kD, kGP, kH>;
     PdlLaunch l(dim3(grid), dim3(kAttnThreads), C::kSmemBytes, stream);
-    if (args.cluster_size > 0) {
-        // Cluster launches go without programmatic dependent launch.  Measured
-        // on B200: launched early, beside the resident CTAs of the preceding
-        // kernel (the check + append kernel, with 256 or with 128 threads),
-        // a grid sized to every cluster the device holds could not place one
-        // or two of its clusters, and those started only when other clusters
-        // of the grid exited, about 1.6x the call's time.  Launched after the
-        // preceding kernel, every cluster starts at once.
-        l.set_cluster(args.cluster_size);
-        l.cfg.attrs = &l.attr[1];
-        l.cfg.numAttrs = 1;
-    }
+    if (args.cluster_size > 0) l.set_cluster(args.cluster_size);
     return cudaLaunchKernelEx(&l.cfg, attn_partial_kernel<kFp8, kD, kGP, kH>, tk, tv, args);
 }
 

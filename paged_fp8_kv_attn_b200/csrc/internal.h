@@ -150,6 +150,8 @@ cudaError_t launch_append(bool fp8, const uint16_t* k_new, const uint16_t* v_new
                           void* v_cache, int32_t num_pages, const uint8_t* abort,
                           cudaStream_t stream);
 
+// all of the SM's on-chip memory as shared memory for the step's first kernels
+cudaError_t step_kernels_set_carveout();
 cudaError_t launch_check_append(bool fp8, const uint32_t* page_tags, int32_t num_pages,
                                 const int32_t* page_table, const uint32_t* expected_tags,
                                 int32_t max_pages, const int32_t* seq_lens, int32_t batch,

@@ -364,4 +364,19 @@ cudaError_t launch_requant(const uint16_t* src_pool, int32_t src_num_pages,
                               dst_pool, dst_num_pages, dst_pages, num_pairs, page_elems, scale);
 }
 
+// The step's first kernels run beside the attention grid that programmatic
+// dependent launch starts early: an SM running one of them must already have
+// its on-chip memory configured as the attention kernel wants it (all of it
+// shared), or the attention CTAs can join that SM only after it drains.
+cudaError_t step_kernels_set_carveout() {
+    const int c = cudaSharedmemCarveoutMaxShared;
+    const cudaFuncAttribute at = cudaFuncAttributePreferredSharedMemoryCarveout;
+    cudaError_t e = cudaFuncSetAttribute(tag_check_kernel, at, c);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(append_kernel<true>, at, c);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(append_kernel<false>, at, c);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(check_append_kernel<true>, at, c);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(check_append_kernel<false>, at, c);
+    return e;
+}
+
 }  // namespace pkv

@@ -385,9 +385,11 @@ def time_per_call(fn, steps, warmup, flush=None):
 
 
 def time_pair(fn_a, fn_b, steps, warmup, flush=None):
-    """Device times (us) of two calls measured alternately (a, b, a, b, ...)
-    so that clock and thermal drift affect both alike: (median a, median b,
-    samples a, samples b), sample i of a and of b forming one pair."""
+    """Device times (us) of two calls measured alternately so that clock and
+    thermal drift affect both alike, the order within a pair swapped every
+    other pair (a b, b a, a b, ...) so that neither call always follows the
+    other: (median a, median b, samples a, samples b), sample i of a and of
+    b forming one pair."""
     import torch
     for _ in range(warmup):
         fn_a()
@@ -395,7 +397,8 @@ def time_pair(fn_a, fn_b, steps, warmup, flush=None):
     torch.cuda.synchronize()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
     for i in range(steps):
-        for j, fn in enumerate((fn_a, fn_b)):
+        order = ((0, fn_a), (1, fn_b)) if i % 2 == 0 else ((1, fn_b), (0, fn_a))
+        for j, fn in order:
             if flush is not None:
                 flush()
             ev[i][2 * j].record()

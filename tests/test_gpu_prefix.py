@@ -162,7 +162,7 @@ def check_case(wl, num_ctas, label, items=None):
 
 
 @pytest.mark.parametrize("num_ctas", [0, 7, 64])
-@pytest.mark.parametrize("page_size", [16, 64, 128])
+@pytest.mark.parametrize("page_size", [16, 32, 64, 128])
 def test_prefix_groups(cuda_device, page_size, num_ctas):
     scale = 64 // page_size if page_size <= 64 else None
     specs = []
@@ -174,6 +174,28 @@ def test_prefix_groups(cuda_device, page_size, num_ctas):
     wl = make_batch(specs, page_size=page_size, seed=page_size + num_ctas)
     begin = check_case(wl, num_ctas, f"P={page_size} ctas={num_ctas}")
     assert begin.sum() > 0
+
+
+def test_prefix_nan_code_in_a_shared_page_reaches_every_member(cuda_device):
+    """A NaN code in a shared page's K reaches, through the shared pass, every
+    member's query heads of that KV head (as in the oracle and the plain
+    call), and no other head."""
+    specs = [(0, 6, 600), (0, 6, 700), (0, 6, 650), (0, 6, 800)]
+    wl = make_batch(specs, seed=9)
+    G = wl.num_q_heads // wl.num_kv_heads
+    db = DeviceBatch(wl, kv_dtype="fp8")
+    db.check_append()
+    pid = int(wl.page_table[0, 2])
+    assert all(int(wl.page_table[b, 2]) == pid for b in range(len(specs)))
+    db.k_cache[pid, 1, 5, 9] = 0x7F               # KV head 1, token 5 of chunk 2, dim 9
+    begin, ws = run_prefix(db)
+    assert int(begin.min()) > 2                    # chunk 2 went through the shared pass
+    out, lse = db.outputs()
+    for b in range(len(specs)):
+        assert np.isnan(lse[b, G:2 * G]).all() and np.isnan(out[b, G:2 * G]).all()
+        assert np.isfinite(lse[b, :G]).all() and np.isfinite(out[b, :G]).all()
+        assert np.isfinite(lse[b, 2 * G:]).all() and np.isfinite(out[b, 2 * G:]).all()
+    assert pkv.workspace_status(ws) == 0
 
 
 def test_prefix_large_groups_and_lone_member(cuda_device):

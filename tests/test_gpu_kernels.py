@@ -424,6 +424,25 @@ def test_attention_tiny_decode_with_check(cuda_device, kv):
 
 
 @pytest.mark.parametrize("kv", ["fp8", "bf16"])
+@pytest.mark.parametrize("num_ctas", [0, 5, -4])
+def test_attention_full_page_table_rows(cuda_device, kv, num_ctas):
+    """Requests at the longest length their page-table rows allow (every entry
+    used, the new token in the last slot of the last page) beside a one-token
+    request, in the library's split, split-K over 5 CTAs and clusters of 4."""
+    lens = [2048, 1, 2048, 1000]
+    wl = workloads.custom(lens, page_size=64, num_q_heads=64, num_kv_heads=8, head_dim=128,
+                          seed=91)
+    assert wl.page_table.shape[1] * wl.page_size == max(lens)
+    db = DeviceBatch(wl, kv_dtype=kv)
+    db.step(check=False, append=True, num_ctas=num_ctas)
+    out, lse = db.outputs()
+    items = list(range(wl.batch * wl.num_kv_heads))
+    ref_o, ref_l, _ = oracle_step(wl, items, kv_dtype=kv, check=False, append=True)
+    compare(wl, items, out, lse, ref_o, ref_l, label=f"{kv} full rows ctas={num_ctas}")
+    assert pkv.workspace_status(db.ws) == 0
+
+
+@pytest.mark.parametrize("kv", ["fp8", "bf16"])
 def test_attention_dead_requests(cuda_device, kv):
     lens = [100, 100, 100, 100, 300, 5]
     wl = workloads.custom(lens, page_size=16, num_q_heads=16, num_kv_heads=2, head_dim=128,
